@@ -1,0 +1,500 @@
+/*
+ * sage_oracle.c -- plain, slow CPU oracle for SageAttention-style quantized
+ * attention.  TEST INFRASTRUCTURE ONLY: it exists so that tests/, the smoke
+ * check and the benchmark's CPU-baseline leg can check the CUDA library
+ * against an independent statement of the method.  Nothing in the product
+ * path may call it, and it shares no code with the CUDA sources.
+ *
+ * Every routine follows the method in the order the pages give it:
+ *
+ *   [SA2]  "SageAttention2" paper summary (sgqg.cn/news/89714),
+ *          sections 相关工作 (SageAttention bullet) and SageAttention2方法
+ *          (smooth Q; per-thread quantization; FP8 quantization of P~V;
+ *          FP32 buffer for the FP22 accumulator).
+ *   [KAI]  "Kairos的注意力加速利器SageAttention INT8/FP8量化内核..." (mhpq.cn),
+ *          section 二, 2.1 (kernel table: fp32 / fp32+fp32 accumulation,
+ *          per_warp granularity) and 2.2 (block INT8 quantization, smoothing,
+ *          two-level accumulation).
+ *   [GUIDE] "SageAttention量化加速框架完整指南" (mhpq.cn), sections 五分钟跑通
+ *          (sageattn(q,k,v,tensor_layout,is_causal)) and 性能调优实战
+ *          (pv_accum_dtype).
+ *
+ * The pages give no formulas, block sizes or rounding rules.  The readings
+ * taken where they are silent are stated at each routine and listed in the
+ * design notes: round-to-nearest-even everywhere, symmetric INT8 codes in
+ * [-127, 127], the group shapes of orc_q_group/orc_k_group, 128-key tiles in
+ * increasing order for the online softmax, the row sum taken over the
+ * unquantized P~, a static FP8 scale of 448 (the E4M3 maximum) for P~.
+ *
+ * Precision: floating point in fp64 except where the method itself fixes a
+ * float32 value that decides an integer code (the smoothed K/Q fed to the
+ * INT8 quantizer, the scale products, the P~*448 fed to the E4M3 encoder);
+ * those steps are written in float32 so that both sides decide each code in
+ * the same precision.  Build with -ffp-contract=off: no fused multiply-adds.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+
+#define ORC_EXPORT __attribute__((visibility("default")))
+
+/* ------------------------------------------------------------------------ */
+/* OCP 8-bit floating point, E4M3 ("FN": no infinities).                     */
+/* Bias 7, 3 mantissa bits, largest finite 448 = 1.75 * 2^8 (code 0x7E),     */
+/* smallest subnormal 2^-9 (code 0x01), S.1111.111 is NaN.                   */
+/* The pages name only the E4M3 flavour [SA2, FP8 quantization of P~V]; the   */
+/* format is the OCP one that tensor cores implement.  Conversion: round to  */
+/* nearest, ties to even, then saturate to +-448 ("satfinite"); NaN stays    */
+/* NaN, +-Inf saturates.                                                     */
+/* ------------------------------------------------------------------------ */
+ORC_EXPORT float orc_e4m3_to_float(uint8_t c) {
+    int s = c >> 7, e = (c >> 3) & 0xF, m = c & 7;
+    double v;
+    if (e == 0xF && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);               /* subnormal: m/8 * 2^-6 */
+    else v = ldexp(1.0 + m / 8.0, e - 7);
+    return (float)(s ? -v : v);
+}
+
+ORC_EXPORT uint8_t orc_e4m3_from_float(float x) {
+    uint8_t sign = signbit(x) ? 0x80 : 0x00;
+    double a = fabs((double)x);
+    if (isnan(x)) return sign | 0x7F;
+    if (a >= 448.0) return sign | 0x7E;                  /* saturate (incl. Inf) */
+    if (a < ldexp(1.0, -6)) {                            /* subnormal range */
+        double q = nearbyint(a * 512.0);                 /* units of 2^-9, RNE */
+        /* q == 8 is exactly the smallest normal 2^-6, whose code is 0x08. */
+        return sign | (uint8_t)q;
+    }
+    int e;
+    double f = frexp(a, &e);                             /* a = f * 2^e, f in [0.5, 1) */
+    e -= 1;                                              /* a = (2f) * 2^e, 2f in [1, 2) */
+    double mant = nearbyint((2.0 * f - 1.0) * 8.0);      /* 3 fraction bits, RNE */
+    if (mant == 8.0) { mant = 0.0; e += 1; }
+    if (e > 8 || (e == 8 && mant > 6.0)) return sign | 0x7E;   /* rounds past 448 */
+    return sign | (uint8_t)(((e + 7) << 3) | (int)mant);
+}
+
+ORC_EXPORT void orc_e4m3_from_float_array(const float* x, uint8_t* out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_e4m3_from_float(x[i]);
+}
+ORC_EXPORT void orc_e4m3_to_float_array(const uint8_t* c, float* out, int64_t n) {
+    for (int64_t i = 0; i < n; ++i) out[i] = orc_e4m3_to_float(c[i]);
+}
+
+/* IEEE binary16 / bfloat16 rounding of a double (RNE), used for the 16-bit
+ * P~ of the FP16-PV mode [KAI 2.1, sm80 row: INT8 QK^T, FP16 PV].            */
+static double round_to_f16(double x) {
+    if (x == 0.0 || isnan(x)) return x;
+    double a = fabs(x);
+    int e;
+    frexp(a, &e);                                        /* a in [2^(e-1), 2^e) */
+    int ulp_exp = (e - 1) - 10;                          /* 10 fraction bits */
+    if (ulp_exp < -24) ulp_exp = -24;                    /* subnormal spacing 2^-24 */
+    double r = ldexp(nearbyint(ldexp(a, -ulp_exp)), ulp_exp);
+    if (r > 65504.0) r = INFINITY;
+    return x < 0 ? -r : r;
+}
+static double round_to_bf16(double x) {
+    float f = (float)x;                                  /* the P~ value is an fp32 */
+    uint32_t u;
+    memcpy(&u, &f, 4);
+    if ((u & 0x7FFFFFFFu) > 0x7F800000u) return x;
+    uint32_t lsb = (u >> 16) & 1u;
+    u = (u + 0x7FFFu + lsb) & 0xFFFF0000u;
+    memcpy(&f, &u, 4);
+    return (double)f;
+}
+
+ORC_EXPORT double orc_round_f16(double x) { return round_to_f16(x); }
+ORC_EXPORT double orc_round_bf16(double x) { return round_to_bf16(x); }
+
+/* ------------------------------------------------------------------------ */
+/* Quantization groups (reading; the pages name the granularities --        */
+/* per-block, per-warp [KAI 2.1/2.2], per-thread [SA2, per-thread           */
+/* quantization] -- but define none of them).  Tokens are counted from the  */
+/* start of their sequence.  Q is split in 128-token blocks, K in 128-token */
+/* blocks (two 64-token halves).  Within one block:                         */
+/*   per_block : Q one group of 128 rows;      K two groups of 64 rows.     */
+/*   per_warp  : Q four groups of 32 rows;     K two groups of 64 rows.     */
+/*   per_thread: Q rows of a 32-row slice with equal (row mod 8) -> 8 groups */
+/*               per slice, 32 per block;                                   */
+/*               K rows of a 64-row half with equal (row mod 8) -> 8 groups  */
+/*               per half, 16 per block.                                    */
+/* (per_thread mirrors the thread-to-row map of the m16n8k32 MMA fragments  */
+/* the pages' kernels were written for: a thread owns rows r and r+8 of     */
+/* each 16-row slab, hence one scale per residue mod 8.)                    */
+/* ------------------------------------------------------------------------ */
+enum { ORC_PER_BLOCK = 0, ORC_PER_WARP = 1, ORC_PER_THREAD = 2 };
+
+ORC_EXPORT int orc_q_groups_per_block(int gran) {
+    return gran == ORC_PER_BLOCK ? 1 : gran == ORC_PER_WARP ? 4 : 32;
+}
+ORC_EXPORT int orc_k_groups_per_block(int gran) {
+    return gran == ORC_PER_THREAD ? 16 : 2;
+}
+ORC_EXPORT int orc_q_group(int gran, int r) {           /* r: row within its 128-block */
+    if (gran == ORC_PER_BLOCK) return 0;
+    if (gran == ORC_PER_WARP) return r / 32;
+    return (r / 32) * 8 + (r % 8);
+}
+ORC_EXPORT int orc_k_group(int gran, int r) {
+    if (gran == ORC_PER_THREAD) return (r / 64) * 8 + (r % 8);
+    return r / 64;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Smooth K [SA2, 相关工作/SageAttention: K is preprocessed to protect the   */
+/* accuracy; KAI 2.2, smoothing]: subtract the per-channel mean of K over   */
+/* the tokens of its sequence (reading: all tokens, also under a causal     */
+/* mask).  Softmax rows are invariant to it: q.(k_j - mu) = q.k_j - q.mu,   */
+/* a constant shift of the whole score row.                                 */
+/*                                                                          */
+/* The mean is fixed to the last bit: the sum is exact (fp16 inputs are     */
+/* integers times 2^-24 and are summed in int64; bf16 inputs are summed in  */
+/* fp64, which is exact unless the values span more than ~45 binary orders) */
+/* then mean = float( double(sum) / L ).                                    */
+/*   x: [L][D] values (exactly the fp16/bf16 inputs), mu: [D] float out.    */
+/* ------------------------------------------------------------------------ */
+ORC_EXPORT void orc_channel_mean(const double* x, int64_t L, int D, int is_fp16, float* mu) {
+    for (int c = 0; c < D; ++c) {
+        double mean;
+        if (is_fp16) {
+            int64_t acc = 0;
+            for (int64_t t = 0; t < L; ++t) acc += (int64_t)ldexp(x[t * D + c], 24);
+            mean = ldexp((double)acc, -24) / (double)L;
+        } else {
+            double acc = 0.0;
+            for (int64_t t = 0; t < L; ++t) acc += x[t * D + c];
+            mean = acc / (double)L;
+        }
+        mu[c] = L > 0 ? (float)mean : 0.0f;
+    }
+}
+
+/* xs[t][c] = float(x[t][c] - mu[c]): one float32 subtraction (x is exactly a
+ * float32 value).  mu == NULL means no smoothing.                           */
+ORC_EXPORT void orc_subtract_channel(const double* x, int64_t L, int D, const float* mu, float* xs) {
+    for (int64_t t = 0; t < L; ++t)
+        for (int c = 0; c < D; ++c) {
+            float v = (float)x[t * D + c];
+            xs[t * D + c] = mu ? v - mu[c] : v;
+        }
+}
+
+/* Smooth Q [SA2, 平滑Q]: subtract the mean of each 128-token Q block.       *
+ * QK^T = (Q - mu_Q) K^T + mu_Q K^T: the first product runs on the INT8     *
+ * tensor cores, the second is a per-block row vector added to the scores   *
+ * (orc_smooth_q_bias).  Block means: exact fp64 sum of the block's tokens  *
+ * (at most 128 fp16/bf16 values), mean = float(sum / n).                   *
+ *   mu_blk: [ceil(L/128)][D] float out; xs: [L][D] float out.               */
+ORC_EXPORT void orc_smooth_q_blocks(const double* x, int64_t L, int D, float* mu_blk, float* xs) {
+    int64_t nblk = (L + 127) / 128;
+    for (int64_t b = 0; b < nblk; ++b) {
+        int64_t t0 = b * 128, t1 = t0 + 128 < L ? t0 + 128 : L;
+        for (int c = 0; c < D; ++c) {
+            double acc = 0.0;
+            for (int64_t t = t0; t < t1; ++t) acc += x[t * D + c];
+            float m = (float)(acc / (double)(t1 - t0));
+            mu_blk[b * D + c] = m;
+            for (int64_t t = t0; t < t1; ++t) xs[t * D + c] = (float)x[t * D + c] - m;
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Symmetric INT8 quantization per group [KAI 2.2 block INT8 quantization;  */
+/* SA2 per-thread quantization].  For a group G:                            */
+/*   amax  = max |x| over G  (valid tokens only)                            */
+/*   delta = amax / 127                      (float32 IEEE division)        */
+/*   code  = clamp(rne(x * (127 / amax)), -127, 127)                        */
+/* with 127/amax one float32 division per group and the product rounded to  */
+/* float32 before the round-to-nearest-even to an integer (reading: the     */
+/* pages give neither rounding nor range; x/delta is taken as x times the   */
+/* reciprocal of delta expressed as 127/amax).  amax == 0 gives delta = 0   */
+/* and all codes 0.                                                         */
+/*   xs: [L][D] float (already smoothed), is_q selects the Q or K groups.   */
+/*   codes: [L][D]; scales: [nblk][groups_per_block].                       */
+/* ------------------------------------------------------------------------ */
+ORC_EXPORT void orc_quant_int8(const float* xs, int64_t L, int D, int is_q, int gran,
+                               int8_t* codes, float* scales) {
+    int ng = is_q ? orc_q_groups_per_block(gran) : orc_k_groups_per_block(gran);
+    int64_t nblk = (L + 127) / 128;
+    float* amax = (float*)malloc(sizeof(float) * ng);
+    for (int64_t b = 0; b < nblk; ++b) {
+        for (int g = 0; g < ng; ++g) amax[g] = 0.0f;
+        for (int r = 0; r < 128 && b * 128 + r < L; ++r) {
+            int g = is_q ? orc_q_group(gran, r) : orc_k_group(gran, r);
+            const float* row = xs + (b * 128 + r) * D;
+            for (int c = 0; c < D; ++c) {
+                float a = fabsf(row[c]);
+                if (a > amax[g]) amax[g] = a;
+            }
+        }
+        for (int g = 0; g < ng; ++g) scales[b * ng + g] = amax[g] / 127.0f;
+        for (int r = 0; r < 128 && b * 128 + r < L; ++r) {
+            int g = is_q ? orc_q_group(gran, r) : orc_k_group(gran, r);
+            float inv = amax[g] > 0.0f ? 127.0f / amax[g] : 0.0f;
+            const float* row = xs + (b * 128 + r) * D;
+            int8_t* out = codes + (b * 128 + r) * D;
+            for (int c = 0; c < D; ++c) {
+                float y = row[c] * inv;                    /* float32 product */
+                double q = nearbyint((double)y);           /* ties to even */
+                if (q > 127.0) q = 127.0;
+                if (q < -127.0) q = -127.0;
+                out[c] = (int8_t)q;
+            }
+        }
+    }
+    free(amax);
+}
+
+/* Per-row view of the group scales: rs[t] = scale of the group of token t. */
+ORC_EXPORT void orc_row_scales(const float* scales, int64_t L, int is_q, int gran, float* rs) {
+    int ng = is_q ? orc_q_groups_per_block(gran) : orc_k_groups_per_block(gran);
+    for (int64_t t = 0; t < L; ++t) {
+        int r = (int)(t % 128);
+        int g = is_q ? orc_q_group(gran, r) : orc_k_group(gran, r);
+        rs[t] = scales[(t / 128) * ng + g];
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* V to FP8 E4M3 per channel [SA2, FP8 quantization of P~V: per channel]:   */
+/*   amax_c = max_t |V[t][c]|; delta_c = amax_c / 448; code = E4M3(V * (448 */
+/*   / amax_c)) with the product rounded to float32 (same reading of x /    */
+/*   delta as for INT8; 448 is the largest finite E4M3 value).              */
+/*   v: [L][D] values; codes [L][D]; dv [D].                                 */
+/* ------------------------------------------------------------------------ */
+ORC_EXPORT void orc_quant_v_fp8(const double* v, int64_t L, int D, uint8_t* codes, float* dv) {
+    for (int c = 0; c < D; ++c) {
+        float amax = 0.0f;
+        for (int64_t t = 0; t < L; ++t) {
+            float a = fabsf((float)v[t * D + c]);
+            if (a > amax) amax = a;
+        }
+        dv[c] = amax / 448.0f;
+        float inv = amax > 0.0f ? 448.0f / amax : 0.0f;
+        for (int64_t t = 0; t < L; ++t) {
+            float y = (float)v[t * D + c] * inv;
+            codes[t * D + c] = orc_e4m3_from_float(y);
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* INT8 QK^T with int32 accumulation [SA2 / KAI 2.2]: exact integer dot     */
+/* products, |S| <= D * 127^2 < 2^22.  out: [Lq][Lk].                        */
+/* ------------------------------------------------------------------------ */
+ORC_EXPORT void orc_scores_int32(const int8_t* qc, const int8_t* kc, int64_t Lq, int64_t Lk,
+                                 int D, int32_t* out) {
+    #pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < Lq; ++i)
+        for (int64_t j = 0; j < Lk; ++j) {
+            int32_t acc = 0;
+            for (int c = 0; c < D; ++c) acc += (int32_t)qc[i * D + c] * (int32_t)kc[j * D + c];
+            out[i * Lk + j] = acc;
+        }
+}
+
+/* Smooth-Q score correction [SA2, 平滑Q]: bias[b][j] = sum_c mu_Q[b][c] *   *
+ * Khat[j][c] with Khat = delta_K(j) * K_code the dequantized smoothed K     *
+ * (reading: the only choice that needs no second pass over full-precision  *
+ * K).  Evaluated in fp64.  bias: [nqblk][Lk].                               */
+ORC_EXPORT void orc_smooth_q_bias(const float* mu_blk, int64_t nqblk, const int8_t* kc,
+                                  const float* k_rs, int64_t Lk, int D, double* bias) {
+    for (int64_t b = 0; b < nqblk; ++b)
+        for (int64_t j = 0; j < Lk; ++j) {
+            double acc = 0.0;
+            for (int c = 0; c < D; ++c) acc += (double)mu_blk[b * D + c] * (double)kc[j * D + c];
+            bias[b * Lk + j] = acc * (double)k_rs[j];
+        }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Quantized attention for one (sequence, head), following the FlashAttention */
+/* tiling the method is built on [SA2, 相关工作: SageAttention reuses the    */
+/* FlashAttention block decomposition]:                                     */
+/*                                                                          */
+/*  for each query row i, for each 128-key tile in increasing order          */
+/*  (reading: the tile size is the kernel's; the online-softmax state then   */
+/*  matches the kernel's, which matters because P~ is rounded to FP8        */
+/*  relative to the running maximum), skipping tiles with no visible key:   */
+/*    c_ij   = float(float(dQ_i * dK_j) * float(sm_scale * log2 e))          */
+/*    s_ij   = float(S_ij * c_ij)          (+ smooth-Q bias, see below)      */
+/*    m_new  = max(m, max_j s_ij);  alpha = 2^(m - m_new)                    */
+/*    p_ij   = 2^(s_ij - m_new)            (P~ <= 1)                         */
+/*    l      = alpha * l + sum_j p_ij      (unquantized P~; reading)        */
+/*    FP8 mode  [SA2, FP8 quantization of P~V: static scale for P~,         */
+/*               per-channel for V]:                                        */
+/*       P8_ij = E4M3(float(p_ij * 448))   (static scale 1/448; reading)     */
+/*       Opart = sum_j P8_ij * V8_j        (exact products, fp64 sum)        */
+/*    16-bit mode [KAI 2.1, sm80 row]: Ph = rne16(p), Opart = sum Ph * V_j   */
+/*    O = alpha * O + Opart               (two-level: per-tile partial sums  */
+/*                                         added into an outer accumulator   */
+/*                                         [SA2, FP32 MMA buffer]; in exact  */
+/*                                         arithmetic the one-level "fp32"   */
+/*                                         mode computes the same value)     */
+/*  out_i = O * dV / (448 * l)  (FP8)      or  O / l  (16-bit)               */
+/*                                                                          */
+/* Causal (reading): top-left aligned, key j visible to query i iff j <= i.  */
+/* Smooth Q: s_ij += bias[i/128][j] * float(sm_scale * log2 e).              */
+/*                                                                          */
+/*   qc [Lq][D] int8, q_rs [Lq] row scales; kc [Lk][D], k_rs [Lk];           */
+/*   pv_mode 0: v8 [Lk][D] E4M3 codes, dv [D];                               */
+/*   pv_mode 1: v16 [Lk][D] 16-bit V values (exact), v_is_bf16 picks the    */
+/*              16-bit type P~ is rounded to;                               */
+/*   bias [ceil(Lq/128)][Lk] or NULL; rows [row0, row1) are computed.        */
+/*   out [Lq][D] (only the computed rows are written).                       */
+/* ------------------------------------------------------------------------ */
+ORC_EXPORT void orc_attn_quant_head(const int8_t* qc, const float* q_rs, const int8_t* kc,
+                                    const float* k_rs, const uint8_t* v8, const float* dv,
+                                    const double* v16, int pv_mode, int v_is_bf16,
+                                    const double* bias, int64_t Lq, int64_t Lk, int D,
+                                    int causal, float sm_scale, int64_t row0, int64_t row1,
+                                    double* out) {
+    const float sl2 = sm_scale * 1.44269504f;             /* float(log2 e) */
+    int64_t ntile = (Lk + 127) / 128;
+    #pragma omp parallel
+    {
+        double* O = (double*)malloc(sizeof(double) * D);
+        double* Op = (double*)malloc(sizeof(double) * D);
+        float* s = (float*)malloc(sizeof(float) * 128);
+        double* v8f = NULL;
+        if (pv_mode == 0) v8f = (double*)malloc(sizeof(double) * 256);
+        if (v8f) for (int c = 0; c < 256; ++c) v8f[c] = (double)orc_e4m3_to_float((uint8_t)c);
+        #pragma omp for schedule(dynamic, 4)
+        for (int64_t i = row0; i < row1; ++i) {
+            float m = -INFINITY;
+            double l = 0.0;
+            for (int c = 0; c < D; ++c) O[c] = 0.0;
+            for (int64_t t = 0; t < ntile; ++t) {
+                int64_t j0 = t * 128, j1 = j0 + 128 < Lk ? j0 + 128 : Lk;
+                if (causal && j1 > i + 1) j1 = i + 1;
+                if (j1 <= j0) continue;                    /* fully masked tile */
+                float mt = -INFINITY;
+                for (int64_t j = j0; j < j1; ++j) {
+                    int32_t S = 0;
+                    for (int c = 0; c < D; ++c) S += (int32_t)qc[i * D + c] * (int32_t)kc[j * D + c];
+                    float cij = (q_rs[i] * k_rs[j]) * sl2;
+                    float sj = (float)S * cij;
+                    if (bias) sj = (float)((double)sj + bias[(i / 128) * Lk + j] * (double)sl2);
+                    s[j - j0] = sj;
+                    if (sj > mt) mt = sj;
+                }
+                float mn = m > mt ? m : mt;
+                double alpha = (m == -INFINITY) ? 0.0 : exp2((double)m - (double)mn);
+                double lt = 0.0;
+                for (int c = 0; c < D; ++c) Op[c] = 0.0;
+                for (int64_t j = j0; j < j1; ++j) {
+                    double p = exp2((double)s[j - j0] - (double)mn);
+                    lt += p;
+                    if (pv_mode == 0) {
+                        double p8 = v8f[orc_e4m3_from_float((float)(p * 448.0))];
+                        const uint8_t* vr = v8 + j * D;
+                        for (int c = 0; c < D; ++c) Op[c] += p8 * v8f[vr[c]];
+                    } else {
+                        double ph = v_is_bf16 ? round_to_bf16(p) : round_to_f16((double)(float)p);
+                        const double* vr = v16 + j * D;
+                        for (int c = 0; c < D; ++c) Op[c] += ph * vr[c];
+                    }
+                }
+                l = alpha * l + lt;
+                for (int c = 0; c < D; ++c) O[c] = alpha * O[c] + Op[c];
+                m = mn;
+            }
+            for (int c = 0; c < D; ++c) {
+                double o;
+                if (l <= 0.0) o = 0.0;                     /* no visible key at all */
+                else if (pv_mode == 0) o = O[c] * (double)dv[c] / (448.0 * l);
+                else o = O[c] / l;
+                out[i * D + c] = o;
+            }
+        }
+        free(O); free(Op); free(s); free(v8f);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* The same tiled online softmax with quantization switched off (debug      */
+/* reading used only to pin the FlashAttention bookkeeping): fp64 scores    */
+/* q_i . k_j * sm_scale * log2 e, unrounded P~ and V.  With the tiling       */
+/* removed it is exactly softmax attention, so it must agree with           */
+/* orc_attn_exact_head to fp64 round-off.                                   */
+/*   q [Lq][D], k [Lk][D], v [Lk][D] fp64.                                    */
+/* ------------------------------------------------------------------------ */
+ORC_EXPORT void orc_attn_tiled_fp64_head(const double* q, const double* k, const double* v,
+                                         int64_t Lq, int64_t Lk, int D, int causal,
+                                         double sm_scale, double* out) {
+    const double sl2 = sm_scale * 1.4426950408889634;
+    int64_t ntile = (Lk + 127) / 128;
+    #pragma omp parallel
+    {
+        double* O = (double*)malloc(sizeof(double) * D);
+        double* s = (double*)malloc(sizeof(double) * 128);
+        #pragma omp for schedule(dynamic, 4)
+        for (int64_t i = 0; i < Lq; ++i) {
+            double m = -INFINITY, l = 0.0;
+            for (int c = 0; c < D; ++c) O[c] = 0.0;
+            for (int64_t t = 0; t < ntile; ++t) {
+                int64_t j0 = t * 128, j1 = j0 + 128 < Lk ? j0 + 128 : Lk;
+                if (causal && j1 > i + 1) j1 = i + 1;
+                if (j1 <= j0) continue;
+                double mt = -INFINITY;
+                for (int64_t j = j0; j < j1; ++j) {
+                    double d = 0.0;
+                    for (int c = 0; c < D; ++c) d += q[i * D + c] * k[j * D + c];
+                    s[j - j0] = d * sl2;
+                    if (s[j - j0] > mt) mt = s[j - j0];
+                }
+                double mn = m > mt ? m : mt;
+                double alpha = (m == -INFINITY) ? 0.0 : exp2(m - mn);
+                for (int c = 0; c < D; ++c) O[c] *= alpha;
+                l *= alpha;
+                for (int64_t j = j0; j < j1; ++j) {
+                    double p = exp2(s[j - j0] - mn);
+                    l += p;
+                    for (int c = 0; c < D; ++c) O[c] += p * v[j * D + c];
+                }
+                m = mn;
+            }
+            for (int c = 0; c < D; ++c) out[i * D + c] = l > 0.0 ? O[c] / l : 0.0;
+        }
+        free(O); free(s);
+    }
+}
+
+/* ------------------------------------------------------------------------ */
+/* Exact attention, the quantity the method approximates: softmax(q k^T *    */
+/* sm_scale [+ causal mask]) v, in fp64, one pass with the true row maximum. */
+/* sm_scale defaults to 1/sqrt(D) at the API (reading: the pages use the    */
+/* scaled_dot_product_attention convention they replace [GUIDE, 换进真实模型]). */
+/* ------------------------------------------------------------------------ */
+ORC_EXPORT void orc_attn_exact_head(const double* q, const double* k, const double* v,
+                                    int64_t Lq, int64_t Lk, int D, int causal, double sm_scale,
+                                    double* out) {
+    #pragma omp parallel
+    {
+        double* s = (double*)malloc(sizeof(double) * (Lk > 0 ? Lk : 1));
+        #pragma omp for schedule(dynamic, 4)
+        for (int64_t i = 0; i < Lq; ++i) {
+            int64_t n = causal ? (i + 1 < Lk ? i + 1 : Lk) : Lk;
+            double mx = -INFINITY;
+            for (int64_t j = 0; j < n; ++j) {
+                double d = 0.0;
+                for (int c = 0; c < D; ++c) d += q[i * D + c] * k[j * D + c];
+                s[j] = d * sm_scale;
+                if (s[j] > mx) mx = s[j];
+            }
+            double den = 0.0;
+            for (int64_t j = 0; j < n; ++j) { s[j] = exp(s[j] - mx); den += s[j]; }
+            for (int c = 0; c < D; ++c) {
+                double acc = 0.0;
+                for (int64_t j = 0; j < n; ++j) acc += s[j] * v[j * D + c];
+                out[i * D + c] = n > 0 ? acc / den : 0.0;
+            }
+        }
+        free(s);
+    }
+}
