@@ -1,0 +1,214 @@
+/*
+ * sage.h -- C ABI of the B200 (sm_100a) quantized attention library (libsage).
+ *
+ * The library computes SageAttention-style quantized attention forward:
+ *   out = softmax(Q K^T * sm_scale [+ causal mask]) V
+ * with K smoothed by its per-channel token mean, Q and K quantized to INT8
+ * (QK^T on INT8 tensor cores, int32 accumulation), FlashAttention-style online
+ * softmax over 128-key tiles, P~ quantized to FP8 E4M3 with a static scale and
+ * V to FP8 E4M3 per channel (P~V on FP8 tensor cores), or P~ and V kept in
+ * 16 bits.  Sources for the method:
+ *   - "SageAttention2" paper summary (sgqg.cn/news/89714), section
+ *     SageAttention2方法: smooth Q, per-thread quantization, FP8 P~V with a
+ *     static P~ scale and per-channel V scale, FP32 buffer for the PV sums;
+ *     section 相关工作: SageAttention quantizes Q/K to INT8 after smoothing K
+ *     inside FlashAttention's tiling.
+ *   - "Kairos的注意力加速利器SageAttention INT8/FP8量化内核..." (mhpq.cn),
+ *     section 二 2.1 (kernel table: INT8 QK^T with FP16 or FP8 PV, fp32 and
+ *     fp32+fp32 accumulation, per_warp granularity) and 2.2.
+ *   - "SageAttention量化加速框架完整指南" (mhpq.cn), section 五分钟跑通
+ *     (sageattn(q, k, v, tensor_layout="HND"|"NHD", is_causal); output has
+ *     q's shape), section 性能调优实战 (pv_accum_dtype), section 换进真实模型
+ *     (no attention mask), section 最容易踩的四个安装坑 (an unsupported GPU
+ *     architecture is an error).
+ *   - "SageAttention: Thư viện Attention lượng tử hóa" (topgit.dev), section
+ *     Tính năng chính: variable-length batches (sageattn_varlen) and native
+ *     grouped-query attention.
+ *
+ * Conventions for every entry point:
+ *   - Pointers named q, k, v, out, ws, cu_seqlens_* are DEVICE pointers of
+ *     the current CUDA device; the caller owns all memory.  The library never
+ *     allocates or frees device memory.  q, k, v, out must be 16-byte aligned;
+ *     ws must be 256-byte aligned.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  All work is enqueued asynchronously on it; no entry point
+ *     synchronizes except sage_get_device_error.
+ *   - Argument errors are reported synchronously and nothing is launched.
+ *     A CUDA launch error is reported as SAGE_ERR_CUDA.
+ *   - Device-side timeouts (a pipeline wait that never completes) never hang:
+ *     the kernel records the failure in the workspace's error word, releases
+ *     its resources and returns; sage_get_device_error reports it.
+ *   - Element (b, h, s, d) of a dense tensor lives at
+ *       HND: ((b*H + h)*S + s)*D + d        NHD: ((b*S + s)*H + h)*D + d
+ *     and of a packed variable-length tensor at (t*H + h)*D + d with
+ *     t = cu_seqlens[b] + s.  out has q's layout and dtype.
+ *   - D (head dim) is 64 or 128.  Hq % Hkv == 0; query head h reads KV head
+ *     h / (Hq / Hkv).  sm_scale <= 0 selects 1/sqrt(D).
+ *   - Only NVIDIA B200-class devices (compute capability 10.0) are supported;
+ *     any other device gives SAGE_ERR_UNSUPPORTED.
+ */
+#ifndef SAGE_H_
+#define SAGE_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  SAGE_OK = 0,
+  SAGE_ERR_INVALID_ARG = 1,  /* null pointer, bad size, bad enum, misalignment */
+  SAGE_ERR_UNSUPPORTED = 2,  /* device is not sm_100, D not in {64,128}, ... */
+  SAGE_ERR_WORKSPACE = 3,    /* ws_bytes smaller than the planner's figure */
+  SAGE_ERR_CUDA = 4,         /* a CUDA runtime call or launch failed */
+  SAGE_ERR_TIMEOUT = 5       /* a device pipeline wait gave up (see above) */
+} sage_status_t;
+
+typedef enum { SAGE_HND = 0, SAGE_NHD = 1 } sage_layout_t;
+typedef enum { SAGE_F16 = 0, SAGE_BF16 = 1 } sage_dtype_t;
+
+/* Q/K quantization groups (the pages name the granularities but define
+ * none).  Tokens are counted from the start of their sequence, in blocks of
+ * 128; within a block:
+ *   PER_BLOCK : Q one group of 128 rows;  K two groups of 64 rows.
+ *   PER_WARP  : Q four groups of 32 rows; K two groups of 64 rows.
+ *   PER_THREAD: Q rows of each 32-row slice with equal (row mod 8) share a
+ *               scale (32 groups); K rows of each 64-row half with equal
+ *               (row mod 8) share a scale (16 groups).                        */
+typedef enum { SAGE_PER_BLOCK = 0, SAGE_PER_WARP = 1, SAGE_PER_THREAD = 2 } sage_gran_t;
+
+/* P~V precision: FP8 E4M3 (P~ scale 1/448 static, V scale per channel) or
+ * 16-bit (P~ rounded to the input's 16-bit type, V unquantized). */
+typedef enum { SAGE_PV_FP8 = 0, SAGE_PV_FP16 = 1 } sage_pv_t;
+
+/* P~V accumulation: FP32 = one FP32 tensor-memory accumulator across all KV
+ * tiles; FP32_FP32 = a fresh FP32 partial sum per 128-key tile added into a
+ * separate FP32 register accumulator (two-level accumulation). */
+typedef enum { SAGE_ACC_FP32 = 0, SAGE_ACC_FP32_FP32 = 1 } sage_acc_t;
+
+/* ------------------------------------------------------------------------ */
+/* Workspace.                                                               */
+/* ------------------------------------------------------------------------ */
+/* Bytes of device workspace a dense call (B sequences of S tokens) needs.
+ * Returns 0 for invalid sizes.  smooth_q adds the smooth-Q regions. */
+size_t sage_workspace_bytes(int B, int Hq, int Hkv, int S, int D, sage_pv_t pv, int smooth_q);
+
+/* Bytes for a packed variable-length call: n_seqs sequences with at most
+ * total_q / total_k tokens in all and max_seqlen tokens in the longest one. */
+size_t sage_varlen_workspace_bytes(int n_seqs, int total_q, int total_k, int max_seqlen,
+                                   int Hq, int Hkv, int D, sage_pv_t pv);
+
+/* Byte offsets of the workspace regions (for callers that read the quantized
+ * tensors, e.g. to cache K/V).  Quantized tiles hold 128 tokens; tile t of
+ * sequence b is global tile tile_off(b) + t (dense: b*ceil(S/128) + t).
+ *   q_codes : int8  [Hq ][tiles_q][128 rows][D]   swizzled, see below
+ *   q_scale : float [Hq ][tiles_q][32]            group g of the tile at [g]
+ *   k_codes : int8  [Hkv][tiles_k][128 rows][D]   swizzled
+ *   k_scale : float [Hkv][tiles_k][16]
+ *   k_mean  : float [n_seqs][Hkv][D]              (0 when smooth_k is off)
+ *   v_codes : [Hkv][tiles_k][D rows][128 keys]    E4M3 (1 byte) or 16-bit
+ *             (2 bytes, as two [D][64-key] halves of 128-byte rows)
+ *   v_scale : float [n_seqs][Hkv][D]              (FP8 mode)
+ *   q_mean  : float [Hq][tiles_q][D]              (smooth_q)
+ *   q_bias  : float [Hq][tiles_q][tiles_k_seq*128] (smooth_q, dense only)
+ * Swizzle of every 128-byte row r (D=128 codes, E4M3 V rows, 16-bit V halves):
+ * logical 16-byte chunk c is stored at chunk c ^ (r % 8).  For 64-byte rows
+ * (D=64 codes): chunk c (of 4) is stored at chunk c ^ ((r / 2) % 4).  This is
+ * the 128B / 64B swizzle of the tensor cores' shared-memory operand layout, so
+ * a tile is copied to shared memory as one contiguous block. */
+typedef struct {
+  size_t err;       /* uint32 device error word */
+  size_t tile_off_q, tile_off_k;   /* int32 [n_seqs+1] (varlen) */
+  size_t k_stat, v_stat;           /* pre-pass accumulators */
+  size_t k_mean, v_scale;
+  size_t q_codes, q_scale, k_codes, k_scale, v_codes;
+  size_t q_mean, q_bias;
+  size_t total;
+  int tiles_q, tiles_k;            /* tiles per head */
+} sage_ws_layout_t;
+
+sage_status_t sage_workspace_layout(int n_seqs, int total_q, int total_k, int max_seqlen,
+                                    int Hq, int Hkv, int D, sage_pv_t pv, int smooth_q,
+                                    int varlen, sage_ws_layout_t* out);
+
+/* ------------------------------------------------------------------------ */
+/* Pre-pass: smooth + quantize.                                             */
+/* ------------------------------------------------------------------------ */
+/* Smooth K (per-channel mean over each sequence's tokens, when smooth_k),
+ * optionally smooth Q (mean of each 128-token block, when smooth_q), and
+ * quantize Q and K to INT8 at granularity `gran` into ws.  [SageAttention2
+ * summary, 相关工作 and SageAttention2方法; Kairos page 2.2]
+ * Reads q [B,Hq,S,D] / [B,S,Hq,D] and k likewise with Hkv heads (dtype,
+ * layout).  Writes ws regions k_stat, k_mean, q_codes, q_scale, k_codes,
+ * k_scale (+ q_mean, q_bias when smooth_q). */
+sage_status_t sage_quant_qk(const void* q, const void* k, sage_dtype_t dtype, sage_layout_t layout,
+                            int B, int Hq, int Hkv, int S, int D, sage_gran_t gran,
+                            int smooth_k, int smooth_q, void* ws, size_t ws_bytes, void* stream);
+
+/* Quantize V per channel to E4M3 (pv == SAGE_PV_FP8) or re-lay it out in 16
+ * bits (SAGE_PV_FP16), transposed to [D][keys] tiles.  [SageAttention2
+ * summary, SageAttention2方法, FP8 quantization of P~V]  Writes v_stat,
+ * v_scale, v_codes. */
+sage_status_t sage_quant_v(const void* v, sage_dtype_t dtype, sage_layout_t layout, int B, int Hkv,
+                           int S, int D, sage_pv_t pv, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Attention.                                                               */
+/* ------------------------------------------------------------------------ */
+/* The whole forward pass: sage_quant_qk + sage_quant_v + the attention
+ * kernel.  out has q's shape, layout and dtype.  [Install/tuning guide,
+ * 五分钟跑通 and 性能调优实战] */
+sage_status_t sage_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                            sage_dtype_t dtype, int B, int Hq, int Hkv, int S, int D,
+                            sage_layout_t layout, int is_causal, float sm_scale,
+                            sage_gran_t gran, sage_pv_t pv, sage_acc_t pv_accum,
+                            int smooth_k, int smooth_q, void* ws, size_t ws_bytes, void* stream);
+
+/* The attention kernel alone, on a workspace already filled by
+ * sage_quant_qk and sage_quant_v for the same problem (lets callers keep
+ * quantized K/V; also what the benchmark times as the attention kernel). */
+sage_status_t sage_attn_quantized(void* out, sage_dtype_t dtype, int B, int Hq, int Hkv, int S,
+                                  int D, sage_layout_t layout, int is_causal, float sm_scale,
+                                  sage_gran_t gran, sage_pv_t pv, sage_acc_t pv_accum,
+                                  int smooth_q, const void* ws, size_t ws_bytes, void* stream);
+
+/* Packed variable-length batch with grouped-query attention [repo summary,
+ * Tính năng chính].  q [total_q, Hq, D], k/v [total_k, Hkv, D], out like q.
+ * cu_seqlens_q/k: device int32 [n_seqs+1], non-decreasing, starting at 0;
+ * sequence b holds tokens [cu[b], cu[b+1]).  max_seqlen bounds every
+ * sequence's length (larger lengths are an error reported through the device
+ * error word).  total_q/total_k are the token counts the buffers hold.
+ * Causal masking is top-left aligned: query i sees key j iff j <= i. */
+sage_status_t sage_attn_varlen_fwd(const void* q, const void* k, const void* v, void* out,
+                                   sage_dtype_t dtype, const int* cu_seqlens_q,
+                                   const int* cu_seqlens_k, int n_seqs, int total_q, int total_k,
+                                   int max_seqlen, int Hq, int Hkv, int D, int is_causal,
+                                   float sm_scale, sage_gran_t gran, sage_pv_t pv,
+                                   sage_acc_t pv_accum, int smooth_k, void* ws, size_t ws_bytes,
+                                   void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Diagnostics.                                                             */
+/* ------------------------------------------------------------------------ */
+/* Synchronizes `stream`, reads and clears the workspace error word.  Returns
+ * SAGE_OK, SAGE_ERR_TIMEOUT (a device wait gave up), SAGE_ERR_INVALID_ARG (a
+ * device-side argument check failed, e.g. a varlen length above max_seqlen)
+ * or SAGE_ERR_CUDA.  *bits (optional) receives the raw error word. */
+sage_status_t sage_get_device_error(void* ws, void* stream, uint32_t* bits);
+
+/* Debug: the int32 scores of one 128x128 tile, S = Q_codes(q tile) *
+ * K_codes(k tile)^T, computed by the same tensor-core MMA path as the
+ * attention kernel from a workspace filled by sage_quant_qk.  s_out: device
+ * int32 [128][128] (row = query, column = key).  Dense problems only. */
+sage_status_t sage_debug_qk_tile(const void* ws, int B, int Hq, int Hkv, int S, int D,
+                                 sage_pv_t pv, int smooth_q, int b, int h, int q_tile, int k_tile,
+                                 int32_t* s_out, void* stream);
+
+const char* sage_status_string(sage_status_t s);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SAGE_H_ */

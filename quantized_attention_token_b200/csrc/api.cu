@@ -1,0 +1,386 @@
+// api.cu -- the C ABI of libsage (declared in include/sage.h).
+//
+// Host side only: argument validation, the workspace planner, and the order
+// of launches on the caller's stream.  No device memory is allocated here and
+// no call synchronizes except sage_get_device_error.
+#include <climits>
+#include <cmath>
+#include <cstring>
+
+#include "sage.h"
+#include "sage_launch.cuh"
+
+#define SAGE_EXPORT extern "C" __attribute__((visibility("default")))
+
+namespace sage {
+namespace {
+
+// ---------------------------------------------------------------- device check
+sage_status_t check_device() {
+  static int cache[128] = {0};   // 0 unknown, 1 sm_100, -1 other
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (dev < 0 || dev >= 128) return SAGE_ERR_UNSUPPORTED;
+  if (cache[dev] == 0) {
+    int maj = 0, mnr = 0;
+    if (cudaDeviceGetAttribute(&maj, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&mnr, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
+      return SAGE_ERR_CUDA;
+    cache[dev] = (maj == 10 && mnr == 0) ? 1 : -1;
+  }
+  return cache[dev] == 1 ? SAGE_OK : SAGE_ERR_UNSUPPORTED;
+}
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+size_t up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+int cdiv(int a, int b) { return (a + b - 1) / b; }
+
+// ---------------------------------------------------------------- planner
+// Regions in order: error word, varlen tile offsets, K/V statistics, K/V
+// results, then the Q results (so the K/V part does not depend on Hq).
+sage_status_t plan(int nseq, int total_q, int total_k, int max_seqlen, int Hq, int Hkv, int D, int pv,
+                   int smooth_q, int varlen, sage_ws_layout_t* L) {
+  if (nseq <= 0 || max_seqlen <= 0 || Hq <= 0 || Hkv <= 0 || total_q < 0 || total_k < 0)
+    return SAGE_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return SAGE_ERR_UNSUPPORTED;
+  if (Hq % Hkv != 0) return SAGE_ERR_UNSUPPORTED;
+  if (pv != SAGE_PV_FP8 && pv != SAGE_PV_FP16) return SAGE_ERR_INVALID_ARG;
+  if (smooth_q && varlen) return SAGE_ERR_UNSUPPORTED;
+  if (max_seqlen > (1 << 24) || nseq > (1 << 20) || Hq > 4096) return SAGE_ERR_UNSUPPORTED;
+  const long long tps = cdiv(max_seqlen, kTile);
+  const long long tq = varlen ? (long long)total_q / kTile + nseq : (long long)nseq * tps;
+  const long long tk = varlen ? (long long)total_k / kTile + nseq : (long long)nseq * tps;
+  if (tq > INT_MAX / 2 || tk > INT_MAX / 2) return SAGE_ERR_UNSUPPORTED;
+  std::memset(L, 0, sizeof(*L));
+  L->tiles_q = (int)tq;
+  L->tiles_k = (int)tk;
+  size_t o = 0;
+  auto take = [&](size_t bytes, size_t align) { o = up(o, align); size_t r = o; o += bytes; return r; };
+  const size_t nd = (size_t)nseq * Hkv * D;
+  L->err = take(256, 256);
+  L->tile_off_q = take(varlen ? sizeof(int) * (nseq + 1) : 0, 256);
+  L->tile_off_k = take(varlen ? sizeof(int) * (nseq + 1) : 0, 256);
+  L->k_stat = take(nd * 8, 256);
+  L->v_stat = take(nd * 4, 256);
+  L->k_mean = take(nd * 4, 256);
+  L->v_scale = take(nd * 4, 256);
+  L->k_codes = take((size_t)Hkv * tk * kTile * D, 1024);
+  L->k_scale = take((size_t)Hkv * tk * kKGroupsMax * 4, 256);
+  // sized for 16-bit V in both modes, so every region's offset is the same
+  // whichever P~V precision a later call picks
+  L->v_codes = take((size_t)Hkv * tk * kTile * D * 2, 1024);
+  L->q_codes = take((size_t)Hq * tq * kTile * D, 1024);
+  L->q_scale = take((size_t)Hq * tq * kQGroupsMax * 4, 256);
+  L->q_mean = take(smooth_q ? (size_t)Hq * tq * D * 4 : 0, 256);
+  L->q_bias = take(smooth_q ? (size_t)Hq * tq * tps * kTile * 4 : 0, 256);
+  L->total = up(o, 256);
+  return SAGE_OK;
+}
+
+template <class T>
+T* at(void* ws, size_t off) { return reinterpret_cast<T*>(reinterpret_cast<char*>(ws) + off); }
+
+Strides dense_strides(sage_layout_t layout, int H, int S, int D) {
+  if (layout == SAGE_HND) return Strides{(long long)H * S * D, (long long)S * D, (long long)D};
+  return Strides{(long long)S * H * D, (long long)D, (long long)H * D};
+}
+
+sage_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA; }
+
+sage_status_t check_common(sage_dtype_t dtype, int D, sage_gran_t gran, sage_pv_t pv, sage_acc_t acc) {
+  if (dtype != SAGE_F16 && dtype != SAGE_BF16) return SAGE_ERR_INVALID_ARG;
+  if (gran != SAGE_PER_BLOCK && gran != SAGE_PER_WARP && gran != SAGE_PER_THREAD) return SAGE_ERR_INVALID_ARG;
+  if (pv != SAGE_PV_FP8 && pv != SAGE_PV_FP16) return SAGE_ERR_INVALID_ARG;
+  if (acc != SAGE_ACC_FP32 && acc != SAGE_ACC_FP32_FP32) return SAGE_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return SAGE_ERR_UNSUPPORTED;
+  return SAGE_OK;
+}
+
+PrepassParams base_params(void* ws, const sage_ws_layout_t& L, const Seqs& seqs, int bf16) {
+  PrepassParams p{};
+  p.seqs = seqs;
+  p.bf16 = bf16;
+  p.err = at<uint32_t>(ws, L.err);
+  p.k_stat = at<unsigned long long>(ws, L.k_stat);
+  p.v_stat = at<uint32_t>(ws, L.v_stat);
+  p.k_mean = at<float>(ws, L.k_mean);
+  p.v_scale = at<float>(ws, L.v_scale);
+  return p;
+}
+
+// Q/K pre-pass for dense or varlen problems (stats region zeroed here).
+sage_status_t run_quant_qk(const void* q, const void* k, int bf16, Strides sq, Strides sk, const Seqs& seqs,
+                           int nseq, int Hq, int Hkv, int D, int gran, int smooth_k, int smooth_q, void* ws,
+                           const sage_ws_layout_t& L, cudaStream_t s) {
+  if (cudaMemsetAsync(at<char>(ws, L.k_stat), 0, (size_t)nseq * Hkv * D * 8, s) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  PrepassParams pq = base_params(ws, L, seqs, bf16), pk = pq;
+  pq.x = static_cast<const uint16_t*>(q);
+  pq.st = sq;
+  pq.H = Hq;
+  pq.gran = gran;
+  pq.smooth = smooth_q;
+  pq.tiles = L.tiles_q;
+  pq.codes = at<int8_t>(ws, L.q_codes);
+  pq.scales = at<float>(ws, L.q_scale);
+  pq.q_mean = smooth_q ? at<float>(ws, L.q_mean) : nullptr;
+  pk.x = static_cast<const uint16_t*>(k);
+  pk.st = sk;
+  pk.H = Hkv;
+  pk.gran = gran;
+  pk.smooth = smooth_k;
+  pk.tiles = L.tiles_k;
+  pk.codes = at<int8_t>(ws, L.k_codes);
+  pk.scales = at<float>(ws, L.k_scale);
+  const int tps = cdiv(seqs.max_seqlen, kTile);
+  return cuda_status(prepass_qk(pq, pk, D, nseq, tps, tps, s));
+}
+
+sage_status_t run_quant_v(const void* v, int bf16, Strides sv, const Seqs& seqs, int nseq, int Hkv, int D,
+                          int pv, void* ws, const sage_ws_layout_t& L, cudaStream_t s) {
+  const bool pv8 = pv == SAGE_PV_FP8;
+  if (pv8 && cudaMemsetAsync(at<char>(ws, L.v_stat), 0, (size_t)nseq * Hkv * D * 4, s) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  PrepassParams p = base_params(ws, L, seqs, bf16);
+  p.x = static_cast<const uint16_t*>(v);
+  p.st = sv;
+  p.H = Hkv;
+  p.tiles = L.tiles_k;
+  p.v_codes = at<uint8_t>(ws, L.v_codes);
+  return cuda_status(prepass_v(p, D, pv8, nseq, cdiv(seqs.max_seqlen, kTile), s));
+}
+
+sage_status_t run_attn(void* out, int bf16, Strides so, const Seqs& seqs, int nseq, int Hq, int Hkv, int D,
+                       int causal, float sm_scale, int gran, int pv, int acc, const void* ws,
+                       const sage_ws_layout_t& L, cudaStream_t s) {
+  void* w = const_cast<void*>(ws);
+  AttnParams p{};
+  p.q_codes = at<int8_t>(w, L.q_codes);
+  p.q_scale = at<float>(w, L.q_scale);
+  p.k_codes = at<int8_t>(w, L.k_codes);
+  p.k_scale = at<float>(w, L.k_scale);
+  p.v_codes = at<uint8_t>(w, L.v_codes);
+  p.v_scale = at<float>(w, L.v_scale);
+  p.err = at<uint32_t>(w, L.err);
+  p.seqs = seqs;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.group = Hq / Hkv;
+  p.tiles_q = L.tiles_q;
+  p.tiles_k = L.tiles_k;
+  p.out = out;
+  p.os = so;
+  const float scale = sm_scale > 0.f ? sm_scale : 1.0f / sqrtf((float)D);
+  p.sl2 = scale * kLog2e;
+  p.gran = gran;
+  p.causal = causal ? 1 : 0;
+  p.out_bf16 = bf16;
+  return cuda_status(attn_forward(p, D, pv == SAGE_PV_FP8, acc == SAGE_ACC_FP32_FP32, seqs.max_seqlen, nseq, s));
+}
+
+Seqs dense_seqs(int S) {
+  Seqs q;
+  q.S = S;
+  q.tps = cdiv(S, kTile);
+  q.max_seqlen = S;
+  return q;
+}
+
+sage_status_t check_dense(int B, int Hq, int Hkv, int S, int D, sage_layout_t layout) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || S <= 0) return SAGE_ERR_INVALID_ARG;
+  if (layout != SAGE_HND && layout != SAGE_NHD) return SAGE_ERR_INVALID_ARG;
+  if (D != 64 && D != 128) return SAGE_ERR_UNSUPPORTED;
+  if (Hq % Hkv != 0) return SAGE_ERR_UNSUPPORTED;
+  if ((long long)B * S * Hq * D > (1ll << 40)) return SAGE_ERR_UNSUPPORTED;
+  return SAGE_OK;
+}
+
+}  // namespace
+}  // namespace sage
+
+using namespace sage;
+
+// ====================================================================== C ABI
+SAGE_EXPORT size_t sage_workspace_bytes(int B, int Hq, int Hkv, int S, int D, sage_pv_t pv, int smooth_q) {
+  sage_ws_layout_t L;
+  if (check_dense(B, Hq, Hkv, S, D, SAGE_HND) != SAGE_OK) return 0;
+  if (plan(B, B * S, B * S, S, Hq, Hkv, D, pv, smooth_q, 0, &L) != SAGE_OK) return 0;
+  return L.total;
+}
+
+SAGE_EXPORT size_t sage_varlen_workspace_bytes(int n_seqs, int total_q, int total_k, int max_seqlen, int Hq,
+                                               int Hkv, int D, sage_pv_t pv) {
+  sage_ws_layout_t L;
+  if (plan(n_seqs, total_q, total_k, max_seqlen, Hq, Hkv, D, pv, 0, 1, &L) != SAGE_OK) return 0;
+  return L.total;
+}
+
+SAGE_EXPORT sage_status_t sage_workspace_layout(int n_seqs, int total_q, int total_k, int max_seqlen, int Hq,
+                                                int Hkv, int D, sage_pv_t pv, int smooth_q, int varlen,
+                                                sage_ws_layout_t* out) {
+  if (!out) return SAGE_ERR_INVALID_ARG;
+  return plan(n_seqs, total_q, total_k, max_seqlen, Hq, Hkv, D, pv, smooth_q, varlen, out);
+}
+
+SAGE_EXPORT sage_status_t sage_quant_qk(const void* q, const void* k, sage_dtype_t dtype, sage_layout_t layout,
+                                        int B, int Hq, int Hkv, int S, int D, sage_gran_t gran, int smooth_k,
+                                        int smooth_q, void* ws, size_t ws_bytes, void* stream) {
+  sage_status_t st;
+  if ((st = check_dense(B, Hq, Hkv, S, D, layout)) != SAGE_OK) return st;
+  if ((st = check_common(dtype, D, gran, SAGE_PV_FP8, SAGE_ACC_FP32)) != SAGE_OK) return st;
+  if (!q || !k || !ws) return SAGE_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(ws, 256)) return SAGE_ERR_INVALID_ARG;
+  if (smooth_q) return SAGE_ERR_UNSUPPORTED;
+  sage_ws_layout_t L;
+  if ((st = plan(B, B * S, B * S, S, Hq, Hkv, D, SAGE_PV_FP8, smooth_q, 0, &L)) != SAGE_OK) return st;
+  if (ws_bytes < L.q_scale + (size_t)Hq * L.tiles_q * kQGroupsMax * 4) return SAGE_ERR_WORKSPACE;
+  if ((st = check_device()) != SAGE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return run_quant_qk(q, k, dtype == SAGE_BF16, dense_strides(layout, Hq, S, D), dense_strides(layout, Hkv, S, D),
+                      dense_seqs(S), B, Hq, Hkv, D, gran, smooth_k, smooth_q, ws, L, s);
+}
+
+SAGE_EXPORT sage_status_t sage_quant_v(const void* v, sage_dtype_t dtype, sage_layout_t layout, int B, int Hkv,
+                                       int S, int D, sage_pv_t pv, void* ws, size_t ws_bytes, void* stream) {
+  sage_status_t st;
+  if ((st = check_dense(B, Hkv, Hkv, S, D, layout)) != SAGE_OK) return st;
+  if ((st = check_common(dtype, D, SAGE_PER_BLOCK, pv, SAGE_ACC_FP32)) != SAGE_OK) return st;
+  if (!v || !ws || !aligned(v, 16) || !aligned(ws, 256)) return SAGE_ERR_INVALID_ARG;
+  sage_ws_layout_t L;
+  // the K/V regions do not depend on the number of query heads
+  if ((st = plan(B, B * S, B * S, S, Hkv, Hkv, D, pv, 0, 0, &L)) != SAGE_OK) return st;
+  if (ws_bytes < L.q_codes) return SAGE_ERR_WORKSPACE;
+  if ((st = check_device()) != SAGE_OK) return st;
+  return run_quant_v(v, dtype == SAGE_BF16, dense_strides(layout, Hkv, S, D), dense_seqs(S), B, Hkv, D, pv, ws, L,
+                     static_cast<cudaStream_t>(stream));
+}
+
+SAGE_EXPORT sage_status_t sage_attn_quantized(void* out, sage_dtype_t dtype, int B, int Hq, int Hkv, int S, int D,
+                                              sage_layout_t layout, int is_causal, float sm_scale,
+                                              sage_gran_t gran, sage_pv_t pv, sage_acc_t pv_accum, int smooth_q,
+                                              const void* ws, size_t ws_bytes, void* stream) {
+  sage_status_t st;
+  if ((st = check_dense(B, Hq, Hkv, S, D, layout)) != SAGE_OK) return st;
+  if ((st = check_common(dtype, D, gran, pv, pv_accum)) != SAGE_OK) return st;
+  if (!out || !ws || !aligned(out, 16) || !aligned(ws, 256)) return SAGE_ERR_INVALID_ARG;
+  if (!std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
+  if (smooth_q) return SAGE_ERR_UNSUPPORTED;
+  sage_ws_layout_t L;
+  if ((st = plan(B, B * S, B * S, S, Hq, Hkv, D, pv, smooth_q, 0, &L)) != SAGE_OK) return st;
+  if (ws_bytes < L.total) return SAGE_ERR_WORKSPACE;
+  if ((st = check_device()) != SAGE_OK) return st;
+  return run_attn(out, dtype == SAGE_BF16, dense_strides(layout, Hq, S, D), dense_seqs(S), B, Hq, Hkv, D,
+                  is_causal, sm_scale, gran, pv, pv_accum, ws, L, static_cast<cudaStream_t>(stream));
+}
+
+SAGE_EXPORT sage_status_t sage_attn_fwd(const void* q, const void* k, const void* v, void* out,
+                                        sage_dtype_t dtype, int B, int Hq, int Hkv, int S, int D,
+                                        sage_layout_t layout, int is_causal, float sm_scale, sage_gran_t gran,
+                                        sage_pv_t pv, sage_acc_t pv_accum, int smooth_k, int smooth_q, void* ws,
+                                        size_t ws_bytes, void* stream) {
+  sage_status_t st;
+  if ((st = check_dense(B, Hq, Hkv, S, D, layout)) != SAGE_OK) return st;
+  if ((st = check_common(dtype, D, gran, pv, pv_accum)) != SAGE_OK) return st;
+  if (!q || !k || !v || !out || !ws) return SAGE_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(ws, 256))
+    return SAGE_ERR_INVALID_ARG;
+  if (!std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
+  if (smooth_q) return SAGE_ERR_UNSUPPORTED;
+  sage_ws_layout_t L;
+  if ((st = plan(B, B * S, B * S, S, Hq, Hkv, D, pv, smooth_q, 0, &L)) != SAGE_OK) return st;
+  if (ws_bytes < L.total) return SAGE_ERR_WORKSPACE;
+  if ((st = check_device()) != SAGE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int bf16 = dtype == SAGE_BF16;
+  const Seqs seqs = dense_seqs(S);
+  if ((st = run_quant_qk(q, k, bf16, dense_strides(layout, Hq, S, D), dense_strides(layout, Hkv, S, D), seqs, B, Hq,
+                         Hkv, D, gran, smooth_k, smooth_q, ws, L, s)) != SAGE_OK)
+    return st;
+  if ((st = run_quant_v(v, bf16, dense_strides(layout, Hkv, S, D), seqs, B, Hkv, D, pv, ws, L, s)) != SAGE_OK)
+    return st;
+  return run_attn(out, bf16, dense_strides(layout, Hq, S, D), seqs, B, Hq, Hkv, D, is_causal, sm_scale, gran, pv,
+                  pv_accum, ws, L, s);
+}
+
+SAGE_EXPORT sage_status_t sage_attn_varlen_fwd(const void* q, const void* k, const void* v, void* out,
+                                               sage_dtype_t dtype, const int* cu_seqlens_q, const int* cu_seqlens_k,
+                                               int n_seqs, int total_q, int total_k, int max_seqlen, int Hq, int Hkv,
+                                               int D, int is_causal, float sm_scale, sage_gran_t gran, sage_pv_t pv,
+                                               sage_acc_t pv_accum, int smooth_k, void* ws, size_t ws_bytes,
+                                               void* stream) {
+  sage_status_t st;
+  if ((st = check_common(dtype, D, gran, pv, pv_accum)) != SAGE_OK) return st;
+  if (n_seqs <= 0 || max_seqlen <= 0 || total_q <= 0 || total_k <= 0 || Hq <= 0 || Hkv <= 0)
+    return SAGE_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return SAGE_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !out || !ws || !cu_seqlens_q || !cu_seqlens_k) return SAGE_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(ws, 256) ||
+      !aligned(cu_seqlens_q, 4) || !aligned(cu_seqlens_k, 4))
+    return SAGE_ERR_INVALID_ARG;
+  if (!std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
+  sage_ws_layout_t L;
+  if ((st = plan(n_seqs, total_q, total_k, max_seqlen, Hq, Hkv, D, pv, 0, 1, &L)) != SAGE_OK) return st;
+  if (ws_bytes < L.total) return SAGE_ERR_WORKSPACE;
+  if ((st = check_device()) != SAGE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  Seqs seqs;
+  seqs.cu_q = cu_seqlens_q;
+  seqs.cu_k = cu_seqlens_k;
+  seqs.toff_q = at<int>(ws, L.tile_off_q);
+  seqs.toff_k = at<int>(ws, L.tile_off_k);
+  seqs.max_seqlen = max_seqlen;
+  if (prepass_varlen_offsets(cu_seqlens_q, cu_seqlens_k, n_seqs, max_seqlen, L.tiles_q, L.tiles_k,
+                             at<int>(ws, L.tile_off_q), at<int>(ws, L.tile_off_k), at<uint32_t>(ws, L.err),
+                             s) != cudaSuccess)
+    return SAGE_ERR_CUDA;
+  const int bf16 = dtype == SAGE_BF16;
+  const Strides sq{0, (long long)D, (long long)Hq * D}, skv{0, (long long)D, (long long)Hkv * D};
+  if ((st = run_quant_qk(q, k, bf16, sq, skv, seqs, n_seqs, Hq, Hkv, D, gran, smooth_k, 0, ws, L, s)) != SAGE_OK)
+    return st;
+  if ((st = run_quant_v(v, bf16, skv, seqs, n_seqs, Hkv, D, pv, ws, L, s)) != SAGE_OK) return st;
+  return run_attn(out, bf16, sq, seqs, n_seqs, Hq, Hkv, D, is_causal, sm_scale, gran, pv, pv_accum, ws, L, s);
+}
+
+SAGE_EXPORT sage_status_t sage_get_device_error(void* ws, void* stream, uint32_t* bits) {
+  if (!ws || !aligned(ws, 256)) return SAGE_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t w = 0;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (cudaMemcpy(&w, ws, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (w && cudaMemset(ws, 0, sizeof(w)) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (bits) *bits = w;
+  if (w & (kErrTimeoutLoad | kErrTimeoutMma | kErrTimeoutSoftmax | kErrTimeoutCorr)) return SAGE_ERR_TIMEOUT;
+  if (w) return SAGE_ERR_INVALID_ARG;
+  return SAGE_OK;
+}
+
+SAGE_EXPORT sage_status_t sage_debug_qk_tile(const void* ws, int B, int Hq, int Hkv, int S, int D, sage_pv_t pv,
+                                             int smooth_q, int b, int h, int q_tile, int k_tile, int32_t* s_out,
+                                             void* stream) {
+  sage_status_t st;
+  if ((st = check_dense(B, Hq, Hkv, S, D, SAGE_HND)) != SAGE_OK) return st;
+  if (!ws || !s_out || !aligned(ws, 256) || !aligned(s_out, 16)) return SAGE_ERR_INVALID_ARG;
+  const int tps = cdiv(S, kTile);
+  if (b < 0 || b >= B || h < 0 || h >= Hq || q_tile < 0 || q_tile >= tps || k_tile < 0 || k_tile >= tps)
+    return SAGE_ERR_INVALID_ARG;
+  sage_ws_layout_t L;
+  if ((st = plan(B, B * S, B * S, S, Hq, Hkv, D, pv, smooth_q, 0, &L)) != SAGE_OK) return st;
+  if ((st = check_device()) != SAGE_OK) return st;
+  void* w = const_cast<void*>(ws);
+  const int hk = h / (Hq / Hkv);
+  const int8_t* qt = at<int8_t>(w, L.q_codes) + ((size_t)h * L.tiles_q + (size_t)b * tps + q_tile) * kTile * D;
+  const int8_t* kt = at<int8_t>(w, L.k_codes) + ((size_t)hk * L.tiles_k + (size_t)b * tps + k_tile) * kTile * D;
+  return cuda_status(debug_qk_tile(qt, kt, D, s_out, at<uint32_t>(w, L.err), static_cast<cudaStream_t>(stream)));
+}
+
+SAGE_EXPORT const char* sage_status_string(sage_status_t s) {
+  switch (s) {
+    case SAGE_OK: return "ok";
+    case SAGE_ERR_INVALID_ARG: return "invalid argument";
+    case SAGE_ERR_UNSUPPORTED: return "unsupported (device must be sm_100; D in {64,128}; Hq % Hkv == 0)";
+    case SAGE_ERR_WORKSPACE: return "workspace too small";
+    case SAGE_ERR_CUDA: return "CUDA error";
+    case SAGE_ERR_TIMEOUT: return "device pipeline wait timed out";
+  }
+  return "unknown status";
+}

@@ -1,0 +1,198 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle.
+
+Integer / byte work (INT8 codes, E4M3 codes, int32 scores) must match bit for
+bit; outputs within max-abs 2e-3 of the oracle (plus half an ulp of the
+output's 16-bit type, which the rounded output carries on top); accuracy
+against exact fp64 attention: cosine >= 0.999.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import quantized_attention_token_b200 as sage
+from tests import wsdecode
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-3
+
+
+def _dev(t):
+    return t.cuda()
+
+
+def _tol(ref: np.ndarray, dtype: str) -> np.ndarray:
+    ulp_bits = 10 if dtype == "fp16" else 7
+    return TOL + 0.5 * np.abs(ref) * 2.0 ** -ulp_bits + 2.0 ** -24
+
+
+def _assert_close(out: torch.Tensor, ref: np.ndarray, dtype: str, what=""):
+    o = out.float().cpu().numpy().astype(np.float64)
+    err = np.abs(o - ref)
+    bad = err > _tol(ref, dtype)
+    assert not bad.any(), f"{what}: {bad.sum()} of {bad.size} outside tolerance, max err {err.max():.3e}"
+
+
+def _ws_bytes(ws: torch.Tensor) -> np.ndarray:
+    torch.cuda.synchronize()
+    return ws.cpu().numpy()
+
+
+# ----------------------------------------------------------------------------- pre-pass
+@pytest.mark.parametrize("D,S,gran,dtype,layout", [
+    (128, 256, "per_block", "fp16", "HND"),
+    (128, 300, "per_warp", "bf16", "NHD"),
+    (64, 1000, "per_thread", "fp16", "HND"),
+    (64, 129, "per_block", "bf16", "HND"),
+    (128, 700, "per_thread", "bf16", "NHD"),
+])
+@pytest.mark.parametrize("smooth_k", [True, False])
+def test_prepass_codes_bit_exact(D, S, gran, dtype, layout, smooth_k):
+    sp = synth.Spec("t", Hq=4, Hkv=2, D=D, B=2, S=S, dtype=dtype, layout=layout, k_bias_std=3.0, seed=31)
+    q, k, v = synth.make(sp)
+    nb = sage.sage_workspace_bytes(2, 4, 2, S, D, 0, 0)
+    ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+    sage.quant_qk(_dev(q), _dev(k), ws, layout, gran, smooth_k=smooth_k)
+    sage.quant_v(_dev(v), ws, layout, "fp8")
+    assert sage.get_device_error(ws) == (0, 0)
+    L = sage.workspace_layout(2, 2 * S, 2 * S, S, 4, 2, D)
+    W = _ws_bytes(ws)
+    tps = (S + 127) // 128
+    qc = wsdecode.codes_int8(W, L, "q_codes", 4, L["tiles_q"], D)
+    kc = wsdecode.codes_int8(W, L, "k_codes", 2, L["tiles_k"], D)
+    qs = wsdecode.scales(W, L, "q_scale", 4, L["tiles_q"], 32)
+    ks = wsdecode.scales(W, L, "k_scale", 2, L["tiles_k"], 16)
+    v8 = wsdecode.v_fp8(W, L, 2, L["tiles_k"], D)
+    vs = wsdecode.f32(W, L, "v_scale", 2 * 2 * D).reshape(2, 2, D)
+    km = wsdecode.f32(W, L, "k_mean", 2 * 2 * D).reshape(2, 2, D)
+    pb = oracle.problem(q, k, v, layout)
+    for b in range(2):
+        for h in range(4):
+            r = oracle.quant_q(pb.q[b][h], gran, False)
+            g = qc[h, b * tps:(b + 1) * tps].reshape(-1, D)
+            assert np.array_equal(g[:S], r.codes), (b, h)
+            assert np.all(g[S:] == 0)
+            ng = oracle.q_groups_per_block(gran)
+            assert np.array_equal(qs[h, b * tps:(b + 1) * tps, :ng], r.scales)
+        for h in range(2):
+            r = oracle.quant_k(pb.k[b][h], gran, smooth_k, dtype == "fp16")
+            g = kc[h, b * tps:(b + 1) * tps].reshape(-1, D)
+            assert np.array_equal(g[:S], r.codes), (b, h)
+            assert np.all(g[S:] == 0)
+            ng = oracle.k_groups_per_block(gran)
+            assert np.array_equal(ks[h, b * tps:(b + 1) * tps, :ng], r.scales)
+            if smooth_k:
+                assert np.array_equal(km[b, h], r.mu)
+            rv = oracle.quant_v(pb.v[b][h])
+            g = v8[h, b * tps:(b + 1) * tps].reshape(-1, D)
+            assert np.array_equal(g[:S], rv.codes), (b, h)
+            assert np.all(g[S:] == 0)
+            assert np.array_equal(vs[b, h], rv.scales)
+
+
+def test_prepass_v16_layout():
+    sp = synth.Spec("t", Hq=2, Hkv=2, D=128, B=1, S=200, dtype="bf16", seed=32)
+    q, k, v = synth.make(sp)
+    ws = torch.zeros(sage.sage_workspace_bytes(1, 2, 2, 200, 128, 1, 0), dtype=torch.uint8, device="cuda")
+    sage.quant_v(_dev(v), ws, "HND", "fp16")
+    L = sage.workspace_layout(1, 200, 200, 200, 2, 2, 128, pv=1)
+    g = wsdecode.v_16(_ws_bytes(ws), L, 2, L["tiles_k"], 128).reshape(2, -1, 128)
+    ref = v[0].view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(g[:, :200], ref)
+    assert np.all(g[:, 200:] == 0)
+
+
+@pytest.mark.parametrize("D", [64, 128])
+def test_qk_tile_scores_bit_exact(D):
+    S = 384
+    sp = synth.Spec("t", Hq=2, Hkv=1, D=D, B=1, S=S, k_bias_std=3.0, seed=33)
+    q, k, v = synth.make(sp)
+    ws = torch.zeros(sage.sage_workspace_bytes(1, 2, 1, S, D, 0, 0), dtype=torch.uint8, device="cuda")
+    sage.quant_qk(_dev(q), _dev(k), ws, "HND", "per_thread")
+    pb = oracle.problem(q, k, v)
+    kc = oracle.quant_k(pb.k[0][0], "per_thread", True, True).codes
+    for h in range(2):
+        qc = oracle.quant_q(pb.q[0][h], "per_thread", False).codes
+        ref = oracle.scores_int32(qc, kc)
+        for qt, kt in [(0, 0), (1, 2), (2, 1)]:
+            s = sage.debug_qk_tile(ws, 1, 2, 1, S, D, 0, h, qt, kt).cpu().numpy()
+            assert np.array_equal(s, ref[qt * 128:(qt + 1) * 128, kt * 128:(kt + 1) * 128]), (h, qt, kt)
+    assert sage.get_device_error(ws) == (0, 0)
+
+
+# ----------------------------------------------------------------------------- attention
+CASES = [
+    # D, S, Hq, Hkv, causal, gran, pv, acc, dtype, layout
+    (64, 256, 2, 2, False, "per_block", "fp8", "fp32+fp32", "fp16", "HND"),
+    (64, 256, 2, 2, False, "per_block", "fp8", "fp32", "fp16", "HND"),
+    (128, 300, 4, 2, False, "per_warp", "fp8", "fp32", "fp16", "NHD"),
+    (128, 300, 4, 2, True, "per_thread", "fp8", "fp32+fp32", "fp16", "HND"),
+    (128, 520, 2, 1, True, "per_block", "fp8", "fp32", "bf16", "HND"),
+    (128, 640, 2, 2, False, "per_block", "fp16", "fp32", "fp16", "HND"),
+    (128, 333, 2, 2, True, "per_warp", "fp16", "fp32+fp32", "bf16", "NHD"),
+    (64, 700, 4, 1, True, "per_thread", "fp16", "fp32", "fp16", "HND"),
+    (64, 129, 2, 2, False, "per_thread", "fp8", "fp32+fp32", "bf16", "NHD"),
+    (128, 1, 2, 2, False, "per_block", "fp8", "fp32", "fp16", "HND"),
+    (128, 127, 2, 2, True, "per_block", "fp8", "fp32+fp32", "fp16", "HND"),
+]
+
+
+@pytest.mark.parametrize("D,S,Hq,Hkv,causal,gran,pv,acc,dtype,layout", CASES)
+def test_attention_matches_oracle(D, S, Hq, Hkv, causal, gran, pv, acc, dtype, layout):
+    sp = synth.Spec("t", Hq=Hq, Hkv=Hkv, D=D, B=2, S=S, dtype=dtype, layout=layout, causal=causal,
+                    k_bias_std=3.0, seed=40 + S)
+    q, k, v = synth.make(sp)
+    out = sage.sageattn(_dev(q), _dev(k), _dev(v), layout, causal, qk_quant_gran=gran, pv_dtype=pv,
+                        pv_accum_dtype=acc)
+    torch.cuda.synchronize()
+    ref = oracle.attention(q, k, v, layout, causal, gran=gran, pv=pv)
+    _assert_close(out, ref, dtype, "vs oracle")
+    ex = oracle.attention_exact(q, k, v, layout, causal)
+    o = out.double().cpu().numpy().ravel()
+    cos = o @ ex.ravel() / (np.linalg.norm(o) * np.linalg.norm(ex))
+    assert cos >= 0.999, cos
+
+
+def test_tiny_config():
+    sp = synth.CONFIGS["tiny"]
+    q, k, v = synth.make(sp)
+    out = sage.sageattn(_dev(q), _dev(k), _dev(v), "HND", False)
+    torch.cuda.synchronize()
+    _assert_close(out, oracle.attention(q, k, v), "fp16", "tiny")
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("pv,acc", [("fp8", "fp32+fp32"), ("fp16", "fp32")])
+def test_varlen_gqa_matches_oracle(causal, pv, acc):
+    sp = synth.Spec("t", Hq=4, Hkv=2, D=128, seqlens=[200, 1, 0, 129, 384, 77], causal=causal, seed=50)
+    q, k, v = synth.make(sp)
+    cu = sp.cu_seqlens()
+    cu_d = torch.from_numpy(cu).cuda()
+    out = sage.sageattn_varlen(_dev(q), _dev(k), _dev(v), cu_d, cu_d, max(sp.seqlens), causal, pv_dtype=pv,
+                               pv_accum_dtype=acc)
+    torch.cuda.synchronize()
+    ref = oracle.attention(q, k, v, causal=causal, pv=pv, cu_seqlens=cu)
+    _assert_close(out, ref, "fp16", "varlen")
+
+
+def test_varlen_single_sequence_equals_dense():
+    sp = synth.Spec("t", Hq=4, Hkv=2, D=128, B=1, S=300, layout="NHD", seed=51)
+    q, k, v = synth.make(sp)
+    dense = sage.sageattn(_dev(q), _dev(k), _dev(v), "NHD", True)
+    cu = torch.tensor([0, 300], dtype=torch.int32, device="cuda")
+    var = sage.sageattn_varlen(_dev(q[0]), _dev(k[0]), _dev(v[0]), cu, cu, 300, True)
+    torch.cuda.synchronize()
+    assert torch.equal(dense[0], var)
+
+
+def test_repeated_calls_are_deterministic():
+    sp = synth.Spec("t", Hq=4, Hkv=4, D=128, B=1, S=512, seed=52)
+    q, k, v = (_dev(t) for t in synth.make(sp))
+    a = sage.sageattn(q, k, v)
+    b = sage.sageattn(q, k, v)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
