@@ -42,6 +42,8 @@ def lib():
             "orc_e4m3_from_float_array": (None, [P, P, i64]),
             "orc_e4m3_to_float_array": (None, [P, P, i64]),
             "orc_round_f16": (f64, [f64]),
+            "orc_e4m3_alt_step": (f64, [f64]),
+            "orc_h16_alt_step": (f64, [f64, i32]),
             "orc_round_bf16": (f64, [f64]),
             "orc_q_groups_per_block": (i32, [i32]),
             "orc_k_groups_per_block": (i32, [i32]),
@@ -56,7 +58,7 @@ def lib():
             "orc_scores_int32": (None, [P, P, i64, i64, i32, P]),
             "orc_smooth_q_bias": (None, [P, i64, P, P, i64, i32, P]),
             "orc_attn_quant_head": (None, [P, P, P, P, P, P, P, i32, i32, P, i64, i64, i32,
-                                           i32, f32, i64, i64, P]),
+                                           i32, f32, i64, i64, P, P]),
             "orc_attn_tiled_fp64_head": (None, [P, P, P, i64, i64, i32, i32, f64, P]),
             "orc_attn_exact_head": (None, [P, P, P, i64, i64, i32, i32, f64, P]),
         }
@@ -229,7 +231,8 @@ def smooth_q_bias(qq: QuantQ, kq: QuantK) -> np.ndarray:
 
 def attn_head(qq: QuantQ, kq: QuantK, vq: Optional[QuantV], v16: Optional[np.ndarray],
               pv: str, v_is_bf16: bool, causal: bool, sm_scale: float,
-              rows: Optional[Tuple[int, int]] = None, bias: Optional[np.ndarray] = None) -> np.ndarray:
+              rows: Optional[Tuple[int, int]] = None, bias: Optional[np.ndarray] = None,
+              allow: Optional[np.ndarray] = None) -> np.ndarray:
     Lq, D = qq.codes.shape
     Lk = kq.codes.shape[0]
     r0, r1 = rows if rows is not None else (0, Lq)
@@ -238,7 +241,7 @@ def attn_head(qq: QuantQ, kq: QuantK, vq: Optional[QuantV], v16: Optional[np.nda
         _p(qq.codes), _p(qq.row_scales), _p(kq.codes), _p(kq.row_scales),
         _p(vq.codes) if vq is not None else None, _p(vq.scales) if vq is not None else None,
         _p(v16), PV[pv], int(v_is_bf16), _p(bias), Lq, Lk, D, int(causal),
-        ctypes.c_float(sm_scale), r0, r1, _p(out))
+        ctypes.c_float(sm_scale), r0, r1, _p(out), _p(allow))
     return out
 
 
@@ -295,22 +298,26 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout: str = "
               pv: str = "fp8", smooth_k: bool = True, smooth_q: bool = False,
               cu_seqlens: Optional[np.ndarray] = None,
               q_rows: Optional[Dict[Tuple[int, int], Tuple[int, int]]] = None,
-              heads: Optional[List[Tuple[int, int]]] = None) -> np.ndarray:
+              heads: Optional[List[Tuple[int, int]]] = None, with_allowance: bool = False):
     """The quantized forward pass; returns fp64 output shaped like q.
 
     q_rows optionally restricts (seq, head) -> [row0, row1); heads restricts
-    which (seq, head) pairs are computed (others stay zero).
+    which (seq, head) pairs are computed (others stay zero).  with_allowance:
+    return (out, allow), allow being the per-output bound on what ambiguous
+    roundings of P~ can change (see sage_oracle.c).
     """
     pb = problem(q, k, v, layout, cu_seqlens)
     scale = default_scale(pb.D, sm_scale)
     group = pb.Hq // pb.Hkv
-    outs = []
+    outs, allows = [], []
     for b in range(len(pb.q)):
         needed_kv = {h // group for h in range(pb.Hq) if heads is None or (b, h) in heads}
         kq = {hk: quant_k(pb.k[b][hk], gran, smooth_k, pb.is_fp16) for hk in needed_kv}
         vq = {hk: (quant_v(pb.v[b][hk]) if pv == "fp8" else None) for hk in needed_kv}
-        row = []
+        row, arow = [], []
         for h in range(pb.Hq):
+            al = np.zeros_like(pb.q[b][h])
+            arow.append(al)
             if heads is not None and (b, h) not in heads:
                 row.append(np.zeros_like(pb.q[b][h]))
                 continue
@@ -319,9 +326,14 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout: str = "
             bias = smooth_q_bias(qq, kq[hk]) if smooth_q else None
             rows = q_rows.get((b, h)) if q_rows else None
             row.append(attn_head(qq, kq[hk], vq[hk], pb.v[b][hk] if pv != "fp8" else None, pv,
-                                 not pb.is_fp16, causal, scale, rows, bias))
+                                 not pb.is_fp16, causal, scale, rows, bias,
+                                 al if with_allowance else None))
         outs.append(row)
-    return assemble(outs, q, layout, cu_seqlens)
+        allows.append(arow)
+    out = assemble(outs, q, layout, cu_seqlens)
+    if with_allowance:
+        return out, assemble(allows, q, layout, cu_seqlens)
+    return out
 
 
 def attention_exact(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout: str = "HND",

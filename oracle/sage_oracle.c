@@ -313,6 +313,42 @@ ORC_EXPORT void orc_smooth_q_bias(const float* mu_blk, int64_t nqblk, const int8
 }
 
 /* ------------------------------------------------------------------------ */
+/* Ambiguous roundings.  An implementation computes P~ with its own exp2, a  */
+/* few ulps away from the exact value.  Where the exact P~*448 (or P~) lies  */
+/* within a relative distance ORC_AMBIG of the midpoint between two          */
+/* neighbouring E4M3 (or 16-bit) values, both neighbours are correct         */
+/* roundings.  orc_alt_step returns |other - chosen| for such a value, else  */
+/* 0; the attention routine turns these into a per-output allowance.         */
+/* ------------------------------------------------------------------------ */
+#define ORC_AMBIG 0x1p-16
+
+static double e4m3_alt_step(double y) {
+    uint8_t c = orc_e4m3_from_float((float)y);
+    double v0 = (double)orc_e4m3_to_float(c);
+    double v1;
+    if (y >= v0) { if ((c & 0x7F) >= 0x7E) return 0.0; v1 = (double)orc_e4m3_to_float((uint8_t)(c + 1)); }
+    else { if ((c & 0x7F) == 0) return 0.0; v1 = (double)orc_e4m3_to_float((uint8_t)(c - 1)); }
+    double mid = 0.5 * (v0 + v1);
+    return fabs(y - mid) <= ORC_AMBIG * y ? fabs(v1 - v0) : 0.0;
+}
+static double h16_alt_step(double p, int bf16) {
+    double h0 = bf16 ? round_to_bf16(p) : round_to_f16((double)(float)p);
+    if (h0 <= 0.0) return 0.0;
+    int e;
+    frexp(h0, &e);                                       /* h0 in [2^(e-1), 2^e) */
+    int fb = bf16 ? 7 : 10;
+    double up = ldexp(1.0, (e - 1) - fb);
+    double down = (h0 == ldexp(1.0, e - 1)) ? up / 2 : up;
+    if (!bf16 && (e - 1) - fb < -24) up = down = ldexp(1.0, -24);
+    double h1 = p >= h0 ? h0 + up : h0 - down;
+    double mid = 0.5 * (h0 + h1);
+    return fabs(p - mid) <= ORC_AMBIG * p ? fabs(h1 - h0) : 0.0;
+}
+
+ORC_EXPORT double orc_e4m3_alt_step(double y) { return e4m3_alt_step(y); }
+ORC_EXPORT double orc_h16_alt_step(double p, int bf16) { return h16_alt_step(p, bf16); }
+
+/* ------------------------------------------------------------------------ */
 /* Quantized attention for one (sequence, head), following the FlashAttention */
 /* tiling the method is built on [SA2, 相关工作: SageAttention reuses the    */
 /* FlashAttention block decomposition]:                                     */
@@ -347,19 +383,24 @@ ORC_EXPORT void orc_smooth_q_bias(const float* mu_blk, int64_t nqblk, const int8
 /*              16-bit type P~ is rounded to;                               */
 /*   bias [ceil(Lq/128)][Lk] or NULL; rows [row0, row1) are computed.        */
 /*   out [Lq][D] (only the computed rows are written).                       */
+/*   allow [Lq][D] or NULL: the largest change of each output that ambiguous */
+/*   roundings of P~ (see above) can cause, carried through the same alpha   */
+/*   rescaling and normalization as O.                                       */
 /* ------------------------------------------------------------------------ */
 ORC_EXPORT void orc_attn_quant_head(const int8_t* qc, const float* q_rs, const int8_t* kc,
                                     const float* k_rs, const uint8_t* v8, const float* dv,
                                     const double* v16, int pv_mode, int v_is_bf16,
                                     const double* bias, int64_t Lq, int64_t Lk, int D,
                                     int causal, float sm_scale, int64_t row0, int64_t row1,
-                                    double* out) {
+                                    double* out, double* allow) {
     const float sl2 = sm_scale * 1.44269504f;             /* float(log2 e) */
     int64_t ntile = (Lk + 127) / 128;
     #pragma omp parallel
     {
         double* O = (double*)malloc(sizeof(double) * D);
         double* Op = (double*)malloc(sizeof(double) * D);
+        double* A = (double*)malloc(sizeof(double) * D);
+        double* Ap = (double*)malloc(sizeof(double) * D);
         float* s = (float*)malloc(sizeof(float) * 128);
         double* v8f = NULL;
         if (pv_mode == 0) v8f = (double*)malloc(sizeof(double) * 256);
@@ -368,7 +409,7 @@ ORC_EXPORT void orc_attn_quant_head(const int8_t* qc, const float* q_rs, const i
         for (int64_t i = row0; i < row1; ++i) {
             float m = -INFINITY;
             double l = 0.0;
-            for (int c = 0; c < D; ++c) O[c] = 0.0;
+            for (int c = 0; c < D; ++c) O[c] = A[c] = 0.0;
             for (int64_t t = 0; t < ntile; ++t) {
                 int64_t j0 = t * 128, j1 = j0 + 128 < Lk ? j0 + 128 : Lk;
                 if (causal && j1 > i + 1) j1 = i + 1;
@@ -386,7 +427,7 @@ ORC_EXPORT void orc_attn_quant_head(const int8_t* qc, const float* q_rs, const i
                 float mn = m > mt ? m : mt;
                 double alpha = (m == -INFINITY) ? 0.0 : exp2((double)m - (double)mn);
                 double lt = 0.0;
-                for (int c = 0; c < D; ++c) Op[c] = 0.0;
+                for (int c = 0; c < D; ++c) Op[c] = Ap[c] = 0.0;
                 for (int64_t j = j0; j < j1; ++j) {
                     double p = exp2((double)s[j - j0] - (double)mn);
                     lt += p;
@@ -394,14 +435,23 @@ ORC_EXPORT void orc_attn_quant_head(const int8_t* qc, const float* q_rs, const i
                         double p8 = v8f[orc_e4m3_from_float((float)(p * 448.0))];
                         const uint8_t* vr = v8 + j * D;
                         for (int c = 0; c < D; ++c) Op[c] += p8 * v8f[vr[c]];
+                        double st = allow ? e4m3_alt_step(p * 448.0) : 0.0;
+                        if (st > 0.0)
+                            for (int c = 0; c < D; ++c) Ap[c] += st * fabs(v8f[vr[c]]);
                     } else {
                         double ph = v_is_bf16 ? round_to_bf16(p) : round_to_f16((double)(float)p);
                         const double* vr = v16 + j * D;
                         for (int c = 0; c < D; ++c) Op[c] += ph * vr[c];
+                        double st = allow ? h16_alt_step(p, v_is_bf16) : 0.0;
+                        if (st > 0.0)
+                            for (int c = 0; c < D; ++c) Ap[c] += st * fabs(vr[c]);
                     }
                 }
                 l = alpha * l + lt;
-                for (int c = 0; c < D; ++c) O[c] = alpha * O[c] + Op[c];
+                for (int c = 0; c < D; ++c) {
+                    O[c] = alpha * O[c] + Op[c];
+                    A[c] = alpha * A[c] + Ap[c];
+                }
                 m = mn;
             }
             for (int c = 0; c < D; ++c) {
@@ -410,9 +460,12 @@ ORC_EXPORT void orc_attn_quant_head(const int8_t* qc, const float* q_rs, const i
                 else if (pv_mode == 0) o = O[c] * (double)dv[c] / (448.0 * l);
                 else o = O[c] / l;
                 out[i * D + c] = o;
+                if (allow)
+                    allow[i * D + c] = l <= 0.0 ? 0.0
+                                     : pv_mode == 0 ? A[c] * (double)dv[c] / (448.0 * l) : A[c] / l;
             }
         }
-        free(O); free(Op); free(s); free(v8f);
+        free(O); free(Op); free(A); free(Ap); free(s); free(v8f);
     }
 }
 

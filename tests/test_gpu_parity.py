@@ -25,15 +25,20 @@ def _dev(t):
     return t.cuda()
 
 
-def _tol(ref: np.ndarray, dtype: str) -> np.ndarray:
+def _tol(ref: np.ndarray, dtype: str, allow=None) -> np.ndarray:
+    """2e-3, plus half an ulp of the output's 16-bit type, plus the oracle's
+    allowance for P~ values whose rounding is ambiguous (within the exp2
+    error band of a rounding midpoint, both neighbours are correct)."""
     ulp_bits = 10 if dtype == "fp16" else 7
-    return TOL + 0.5 * np.abs(ref) * 2.0 ** -ulp_bits + 2.0 ** -24
+    t = TOL + 0.5 * np.abs(ref) * 2.0 ** -ulp_bits + 2.0 ** -24
+    return t if allow is None else t + allow
 
 
-def _assert_close(out: torch.Tensor, ref: np.ndarray, dtype: str, what=""):
+def _assert_close(out: torch.Tensor, ref, dtype: str, what=""):
+    ref, allow = ref if isinstance(ref, tuple) else (ref, None)
     o = out.float().cpu().numpy().astype(np.float64)
     err = np.abs(o - ref)
-    bad = err > _tol(ref, dtype)
+    bad = err > _tol(ref, dtype, allow)
     assert not bad.any(), f"{what}: {bad.sum()} of {bad.size} outside tolerance, max err {err.max():.3e}"
 
 
@@ -149,7 +154,7 @@ def test_attention_matches_oracle(D, S, Hq, Hkv, causal, gran, pv, acc, dtype, l
     out = sage.sageattn(_dev(q), _dev(k), _dev(v), layout, causal, qk_quant_gran=gran, pv_dtype=pv,
                         pv_accum_dtype=acc)
     torch.cuda.synchronize()
-    ref = oracle.attention(q, k, v, layout, causal, gran=gran, pv=pv)
+    ref = oracle.attention(q, k, v, layout, causal, gran=gran, pv=pv, with_allowance=True)
     _assert_close(out, ref, dtype, "vs oracle")
     ex = oracle.attention_exact(q, k, v, layout, causal)
     o = out.double().cpu().numpy().ravel()
@@ -162,7 +167,7 @@ def test_tiny_config():
     q, k, v = synth.make(sp)
     out = sage.sageattn(_dev(q), _dev(k), _dev(v), "HND", False)
     torch.cuda.synchronize()
-    _assert_close(out, oracle.attention(q, k, v), "fp16", "tiny")
+    _assert_close(out, oracle.attention(q, k, v, with_allowance=True), "fp16", "tiny")
 
 
 @pytest.mark.parametrize("causal", [True, False])
@@ -175,7 +180,7 @@ def test_varlen_gqa_matches_oracle(causal, pv, acc):
     out = sage.sageattn_varlen(_dev(q), _dev(k), _dev(v), cu_d, cu_d, max(sp.seqlens), causal, pv_dtype=pv,
                                pv_accum_dtype=acc)
     torch.cuda.synchronize()
-    ref = oracle.attention(q, k, v, causal=causal, pv=pv, cu_seqlens=cu)
+    ref = oracle.attention(q, k, v, causal=causal, pv=pv, cu_seqlens=cu, with_allowance=True)
     _assert_close(out, ref, "fp16", "varlen")
 
 

@@ -405,3 +405,49 @@ def test_row_subset_matches_full():
     part = oracle.attention(q, k, v, q_rows={(0, 0): (128, 256)})
     assert np.array_equal(part[0, 0, 128:256], full[0, 0, 128:256])
     assert np.all(part[0, 0, :128] == 0)
+
+
+# ----------------------------------------------------------------------------- ambiguity allowance
+def test_ambiguous_rounding_steps():
+    L = oracle.lib()
+    # E4M3 neighbours 416 and 448 have midpoint 432; 112 and 120 have 116
+    assert L.orc_e4m3_alt_step(432.0) == 32.0
+    assert L.orc_e4m3_alt_step(432.0 * (1 + 2 ** -18)) == 32.0
+    assert L.orc_e4m3_alt_step(116.0 * (1 - 2 ** -18)) == 8.0
+    assert L.orc_e4m3_alt_step(430.0) == 0.0
+    assert L.orc_e4m3_alt_step(448.0) == 0.0              # saturated: no neighbour above
+    assert L.orc_e4m3_alt_step(2.0 ** -10) == 2.0 ** -9   # subnormal tie 0 / 2^-9
+    # fp16: 1 and 1 + 2^-10 (midpoint 1 + 2^-11); below 1 the spacing halves
+    assert L.orc_h16_alt_step(1 + 2 ** -11, 0) == 2.0 ** -10
+    assert L.orc_h16_alt_step(1 - 2 ** -12, 0) == 2.0 ** -11
+    assert L.orc_h16_alt_step(0.7, 0) == 0.0
+    # bf16: 7 fraction bits
+    assert L.orc_h16_alt_step(1 + 2 ** -8, 1) == 2.0 ** -7
+
+
+def test_allowance_zero_when_no_rounding_is_ambiguous():
+    S, D = 256, 64
+    q = torch.zeros(1, 1, S, D, dtype=torch.float16)          # every P~ = 1 -> 448, exact
+    k = torch.randn(1, 1, S, D, generator=torch.Generator().manual_seed(0)).half()
+    v = torch.randn(1, 1, S, D, generator=torch.Generator().manual_seed(1)).half()
+    _, allow = oracle.attention(q, k, v, with_allowance=True)
+    assert np.all(allow == 0)
+
+
+@pytest.mark.parametrize("pv", ["fp8", "fp16"])
+def test_allowance_is_sparse_and_bounded(pv):
+    sp = synth.Spec("t", Hq=2, Hkv=2, D=64, B=1, S=512, causal=True, seed=23)
+    q, k, v = synth.make(sp)
+    out, allow = oracle.attention(q, k, v, causal=True, pv=pv, with_allowance=True)
+    assert np.all(allow >= 0)
+    # E4M3 steps are 2^-4..2^-3 relative, so few P~ fall in the ambiguity
+    # band; 16-bit steps are 2^-10 relative, so many do, each with a tiny step
+    if pv == "fp8":
+        assert np.mean(allow > 0) < 0.3
+    else:
+        assert np.max(allow) < 1e-3
+    # a single ambiguous P~ moves an output by at most one rounding step of
+    # that P~ times |v| / l; l >= 1 (the row maximum contributes P~ = 1)
+    step = 32.0 / 448 if pv == "fp8" else 2 ** -11
+    vmax = float(v.abs().max())
+    assert np.max(allow) <= 512 * step * vmax
