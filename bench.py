@@ -1,0 +1,346 @@
+#!/usr/bin/env python
+"""Throughput of the quantized attention forward pass on B200.
+
+One step = the whole hot path on one batch of synthetic input: the smooth +
+quantize pre-pass (K mean, INT8 Q/K, E4M3 V) followed by the attention kernel
+(INT8 QK^T, online softmax, E4M3 P~V).  Metric: attention TOPS =
+4*B*H*S^2*D / time (halved for causal), the figure the SageAttention pages
+quote for their kernels.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 runs under torch.distributed.run, one process per GPU; every rank runs
+the same workload on its own GPU (independent problems, no data-path
+collective: weak scaling) and the elapsed time is the maximum over ranks.
+Prints one JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+WORKLOAD = "b2_h32_s4096_d128"
+METRIC = "attention TOPS (4BHS²D/t) at D=128, S=4K–32K; % of B200 INT8/FP8 peak"
+FALLBACK_BF16_SUSTAINED = 1400.0   # TFLOP/s, used only without the measured peaks file
+FP8_OVER_BF16 = 2.0                # nominal dense ratio (4.5 / 2.25 PFLOP/s); INT8 = FP8 on B200
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--config", default=WORKLOAD)
+    ap.add_argument("--pv", default="fp8", choices=["fp8", "fp16"])
+    ap.add_argument("--pv-accum", default="fp32+fp32", choices=["fp32", "fp32+fp32"])
+    ap.add_argument("--gran", default="per_block", choices=["per_block", "per_warp", "per_thread"])
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- helpers
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        d = json.load(open(path))
+        return d, "measured"
+    except Exception:
+        return {"bf16_tflops_sustained": FALLBACK_BF16_SUSTAINED, "hbm_gbs": 6650.0}, "fallback"
+
+
+class Clocks:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.Q}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.idx)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("attn_fwd.cu", "sage_common.cuh", "sage_launch.cuh"):
+        h.update(open(os.path.join(ROOT, "quantized_attention_token_b200", "csrc", f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(workload: str):
+    """dram bytes per launch of the attention kernel from the committed ncu
+    summary, if it was taken on the current kernel source; else None."""
+    path = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
+    try:
+        d = json.load(open(path))
+    except Exception:
+        return None
+    e = d.get(workload)
+    if not e or e.get("source_hash") != kernel_source_hash():
+        return None
+    return e.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def cpu_baseline(spec: synth.Spec, q, k, v, pv: str, budget_s: float):
+    """The oracle as it stands, on a bounded sample of the workload: whole
+    query tiles (128 rows, all keys) of a few heads, pre-pass included."""
+    import oracle
+    oracle.lib()
+    tiles_per_head = (spec.S + 127) // 128
+    heads = [(b, h) for b in range(spec.B) for h in range(spec.Hq)]
+    rng = np.random.default_rng(0)
+    order = rng.permutation(len(heads))
+    done_rows, t0, sample = 0, time.perf_counter(), []
+    grp = spec.Hq // spec.Hkv
+    for i in order:
+        b, h = heads[i]
+        hk = h // grp
+        qt = int(rng.integers(0, tiles_per_head))
+        rows = (qt * 128, min(spec.S, qt * 128 + 128))
+        if spec.layout == "HND":
+            qs, ks, vs = q[b:b + 1, h:h + 1], k[b:b + 1, hk:hk + 1], v[b:b + 1, hk:hk + 1]
+        else:
+            qs, ks, vs = q[b:b + 1, :, h:h + 1], k[b:b + 1, :, hk:hk + 1], v[b:b + 1, :, hk:hk + 1]
+        oracle.attention(qs, ks, vs, spec.layout, spec.causal, pv=pv, q_rows={(0, 0): rows})
+        done_rows += rows[1] - rows[0]
+        sample.append(f"b{b}h{h}t{qt}")
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    ops = 4.0 * done_rows * spec.S * spec.D * (0.5 if spec.causal else 1.0)
+    cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
+    return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": cores, "kind": "oracle",
+            "sample": f"{len(sample)} query tiles x 128 rows x all {spec.S} keys (+ their K/V/Q pre-pass) of "
+                      f"{spec.name}, {dt:.1f} s, scaled by the ops of the rows computed"}
+
+
+# ----------------------------------------------------------------------------- main
+def main():
+    args = parse()
+    spec = synth.CONFIGS[args.config]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    ops = spec.attention_ops()
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        q, k, v = synth.make(spec)
+        per_step = []
+        for i in range(args.warmup + args.steps):
+            cb = cpu_baseline(spec, q, k, v, args.pv, max(1.0, args.cpu_seconds / max(1, args.steps)))
+            if i >= args.warmup:
+                per_step.append(cb["value"])
+        val = float(np.median(per_step))
+        cb["value"] = val
+        line = {"impl": "reference", "metric": METRIC, "value": val, "unit": "TOPS", "n_gpus": args.gpus,
+                "steps": args.steps, "warmup": args.warmup, "ms_per_step": ops / (val * 1e12) * 1e3,
+                "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8+e4m3 (f64 oracle)",
+                "data": "synthetic",
+                "config": {"workload": spec.name, "B": spec.B, "H": spec.Hq, "S": spec.S, "D": spec.D},
+                "cpu_baseline": cb,
+                "e2e": {"value": val, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+        print(json.dumps(line), flush=True)
+        return
+
+    import quantized_attention_token_b200 as sage
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+        from datetime import timedelta
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120), device_id=dev)
+
+    q_h, k_h, v_h = synth.make(spec)
+    q, k, v = (t.to(dev) for t in (q_h, k_h, v_h))
+    out = torch.empty_like(q)
+    B, H, S, D = spec.B, spec.Hq, spec.S, spec.D
+    layout = spec.layout
+    pv_code = sage.PV[args.pv]
+    ws = torch.empty(sage.sage_workspace_bytes(B, spec.Hq, spec.Hkv, S, D, pv_code, 0), dtype=torch.uint8,
+                     device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        if ev is not None:
+            ev[0].record(stream)
+        sage.quant_qk(q, k, ws, layout, args.gran)
+        sage.quant_v(v, ws, layout, args.pv)
+        if ev is not None:
+            ev[1].record(stream)
+        sage.attn_quantized(out, ws, B, spec.Hq, spec.Hkv, S, D, layout, spec.causal, None, args.gran, args.pv,
+                            args.pv_accum)
+        if ev is not None:
+            ev[2].record(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    st, bits = sage.get_device_error(ws)
+    if st != 0:
+        raise RuntimeError(f"device error word {bits:#x} after warm-up")
+
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    start, stop = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with Clocks(local) as clk:
+        start.record(stream)
+        for i in range(args.steps):
+            step(evs[i])
+        stop.record(stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    elapsed_ms = start.elapsed_time(stop)
+    attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    pre_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    if world > 1:
+        t = torch.tensor([elapsed_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        elapsed_ms = float(t.item())
+    st, bits = sage.get_device_error(ws)
+    if st != 0:
+        raise RuntimeError(f"device error word {bits:#x} after the timed region")
+
+    ms_per_step = elapsed_ms / args.steps
+    value = world * ops * args.steps / (elapsed_ms * 1e-3) / 1e12
+
+    # end to end through the public API with host buffers: pinned H2D of q,k,v,
+    # the forward pass, D2H of the output, every step
+    qp, kp, vp = (t.pin_memory() for t in (q_h, k_h, v_h))
+    op = torch.empty_like(q_h).pin_memory()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+    def e2e_step():
+        qd = qp.to(dev, non_blocking=True)
+        kd = kp.to(dev, non_blocking=True)
+        vd = vp.to(dev, non_blocking=True)
+        o = sage.sageattn(qd, kd, vd, layout, spec.causal, qk_quant_gran=args.gran, pv_dtype=args.pv,
+                          pv_accum_dtype=args.pv_accum, workspace=ws)
+        op.copy_(o, non_blocking=True)
+
+    for _ in range(2):
+        e2e_step()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    pk, pk_kind = peaks()
+    peak = FP8_OVER_BF16 * float(pk.get("bf16_tflops_sustained", FALLBACK_BF16_SUSTAINED))
+    attn_avg = float(np.mean(attn_ms))
+    achieved = ops / (attn_avg * 1e-3) / 1e12
+    pre_avg = float(np.mean(pre_ms))
+    elem = spec.total_tokens * D
+    pre_bytes = elem * (2 * spec.Hq + 4 * spec.Hkv) + elem * (spec.Hq + 2 * spec.Hkv)   # 9 B/elem at Hq=Hkv
+    line = {
+        "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "int8+e4m3" if args.pv == "fp8" else "int8+f16", "data": "synthetic",
+        "config": {"workload": spec.name, "B": B, "H": spec.Hq, "Hkv": spec.Hkv, "S": S, "D": D,
+                   "layout": layout, "causal": spec.causal, "input_dtype": spec.dtype, "qk_gran": args.gran,
+                   "pv": args.pv, "pv_accum": args.pv_accum,
+                   "l2": "inputs larger than L2: Q/K/V %s = %d MiB per GPU, L2 126 MB" % (
+                       spec.dtype, (spec.Hq + 2 * spec.Hkv) * elem * 2 >> 20)},
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": recorded_traffic(spec.name),
+                     "kernel": "attn_fwd_kernel", "kernel_ms": attn_avg,
+                     "peak_source": f"2 x bf16_tflops_sustained ({pk_kind}); burst figure "
+                                    f"{FP8_OVER_BF16 * float(pk.get('bf16_tflops', 0)):.0f}"},
+        "prepass": {"ms": pre_avg, "achieved_gbs": pre_bytes / (pre_avg * 1e-3) / 1e9,
+                    "peak_gbs": float(pk.get("hbm_gbs", 0)),
+                    "frac": pre_bytes / (pre_avg * 1e-3) / 1e9 / float(pk.get("hbm_gbs", 1))},
+        "e2e": {"value": ops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+                "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))),
+                "d2h_bytes_per_step": int(q_h.numel() * q_h.element_size())},
+        "gpu_launches": 6 * args.steps,
+        "clocks": clk.summary(),
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(spec, q_h, k_h, v_h, args.pv, args.cpu_seconds)
+    print(json.dumps(line), flush=True)
+
+
+if __name__ == "__main__":
+    main()

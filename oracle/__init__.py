@@ -60,7 +60,7 @@ def lib():
             "orc_attn_quant_head": (None, [P, P, P, P, P, P, P, i32, i32, P, i64, i64, i32,
                                            i32, f32, i64, i64, P, P]),
             "orc_attn_tiled_fp64_head": (None, [P, P, P, i64, i64, i32, i32, f64, P]),
-            "orc_attn_exact_head": (None, [P, P, P, i64, i64, i32, i32, f64, P]),
+            "orc_attn_exact_head": (None, [P, P, P, i64, i64, i32, i32, f64, i64, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -245,10 +245,11 @@ def attn_head(qq: QuantQ, kq: QuantK, vq: Optional[QuantV], v16: Optional[np.nda
     return out
 
 
-def attn_exact_head(q, k, v, causal, sm_scale) -> np.ndarray:
+def attn_exact_head(q, k, v, causal, sm_scale, row_offset: int = 0) -> np.ndarray:
+    q = np.ascontiguousarray(q)
     out = np.zeros(q.shape, dtype=np.float64)
     lib().orc_attn_exact_head(_p(q), _p(k), _p(v), q.shape[0], k.shape[0], q.shape[1],
-                              int(causal), float(sm_scale), _p(out))
+                              int(causal), float(sm_scale), int(row_offset), _p(out))
     return out
 
 

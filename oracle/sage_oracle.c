@@ -526,13 +526,15 @@ ORC_EXPORT void orc_attn_tiled_fp64_head(const double* q, const double* k, const
 /* ------------------------------------------------------------------------ */
 ORC_EXPORT void orc_attn_exact_head(const double* q, const double* k, const double* v,
                                     int64_t Lq, int64_t Lk, int D, int causal, double sm_scale,
-                                    double* out) {
+                                    int64_t row_offset, double* out) {
+    /* q holds rows row_offset .. row_offset+Lq-1 of the sequence (causal
+     * masking uses the sequence row index). */
     #pragma omp parallel
     {
         double* s = (double*)malloc(sizeof(double) * (Lk > 0 ? Lk : 1));
         #pragma omp for schedule(dynamic, 4)
         for (int64_t i = 0; i < Lq; ++i) {
-            int64_t n = causal ? (i + 1 < Lk ? i + 1 : Lk) : Lk;
+            int64_t n = causal ? (row_offset + i + 1 < Lk ? row_offset + i + 1 : Lk) : Lk;
             double mx = -INFINITY;
             for (int64_t j = 0; j < n; ++j) {
                 double d = 0.0;

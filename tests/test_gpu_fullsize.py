@@ -1,0 +1,98 @@
+"""Parity at the full sizes of the workloads, in the launch configuration the
+benchmark times: the GPU computes the whole problem, the oracle recomputes
+sampled query tiles (all keys) of sampled heads one by one."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+import quantized_attention_token_b200 as sage
+from tests.test_gpu_parity import _assert_close
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle_rows(spec, q, k, v, b, h, rows, gran, pv):
+    """Oracle output and allowance for rows [r0, r1) of (sequence b, head h),
+    computed on that sequence / head alone."""
+    grp = spec.Hq // spec.Hkv
+    hk = h // grp
+    if spec.varlen:
+        cu = spec.cu_seqlens()
+        s0, s1 = int(cu[b]), int(cu[b + 1])
+        qs, ks, vs = (t[s0:s1].transpose(0, 1).unsqueeze(0) for t in (q[:, h:h + 1], k[:, hk:hk + 1], v[:, hk:hk + 1]))
+        lay = "HND"
+    elif spec.layout == "HND":
+        qs, ks, vs = q[b:b + 1, h:h + 1], k[b:b + 1, hk:hk + 1], v[b:b + 1, hk:hk + 1]
+        lay = "HND"
+    else:
+        qs, ks, vs = q[b:b + 1, :, h:h + 1], k[b:b + 1, :, hk:hk + 1], v[b:b + 1, :, hk:hk + 1]
+        lay = "NHD"
+    out, allow = oracle.attention(qs, ks, vs, lay, spec.causal, gran=gran, pv=pv, q_rows={(0, 0): rows},
+                                  with_allowance=True)
+    sel = (slice(0, 1), slice(0, 1), slice(*rows)) if lay == "HND" else (slice(0, 1), slice(*rows), slice(0, 1))
+    pb = oracle.problem(qs, ks, vs, lay)
+    ex = oracle.attn_exact_head(pb.q[0][0][rows[0]:rows[1]], pb.k[0][0], pb.v[0][0], spec.causal,
+                                oracle.default_scale(spec.D, None), row_offset=rows[0])
+    return out[sel].reshape(-1, spec.D), allow[sel].reshape(-1, spec.D), ex
+
+
+def _gpu_rows(spec, out, b, h, rows):
+    if spec.varlen:
+        s0 = int(spec.cu_seqlens()[b])
+        return out[s0 + rows[0]:s0 + rows[1], h]
+    if spec.layout == "HND":
+        return out[b, h, rows[0]:rows[1]]
+    return out[b, rows[0]:rows[1], h]
+
+
+def _run(spec, gran="per_block", pv="fp8", acc="fp32+fp32"):
+    q, k, v = synth.make(spec)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    if spec.varlen:
+        cu = torch.from_numpy(spec.cu_seqlens()).cuda()
+        out = sage.sageattn_varlen(qd, kd, vd, cu, cu, max(spec.seqlens), spec.causal, qk_quant_gran=gran,
+                                   pv_dtype=pv, pv_accum_dtype=acc)
+    else:
+        out = sage.sageattn(qd, kd, vd, spec.layout, spec.causal, qk_quant_gran=gran, pv_dtype=pv,
+                            pv_accum_dtype=acc)
+    torch.cuda.synchronize()
+    ws = sage.Workspace._cache[0]
+    assert sage.get_device_error(ws) == (0, 0)
+    return q, k, v, out.cpu()
+
+
+def _check(spec, samples, gran="per_block", pv="fp8", acc="fp32+fp32"):
+    q, k, v, out = _run(spec, gran, pv, acc)
+    for b, h, rows in samples:
+        ref, allow, ex = _oracle_rows(spec, q, k, v, b, h, rows, gran, pv)
+        got = _gpu_rows(spec, out, b, h, rows)
+        _assert_close(got, (ref, allow), spec.dtype, f"{spec.name} b{b} h{h} rows{rows}")
+        o = got.double().numpy().ravel()
+        cos = o @ ex.ravel() / (np.linalg.norm(o) * np.linalg.norm(ex))
+        assert cos >= 0.999, (spec.name, b, h, rows, cos)
+
+
+@pytest.mark.parametrize("pv,acc", [("fp8", "fp32+fp32"), ("fp8", "fp32"), ("fp16", "fp32+fp32")])
+def test_b2_h32_s4096_d128(pv, acc):
+    spec = synth.CONFIGS["b2_h32_s4096_d128"]
+    _check(spec, [(0, 0, (0, 128)), (1, 31, (3968, 4096)), (0, 17, (1664, 1792))], pv=pv, acc=acc)
+
+
+def test_video_dit_bf16_nhd():
+    spec = synth.CONFIGS["video_dit"]
+    _check(spec, [(0, 0, (0, 128)), (0, 19, (32640, 32768)), (0, 7, (12800, 12928))])
+
+
+def test_varlen_gqa_causal():
+    spec = synth.CONFIGS["varlen_gqa"]
+    _check(spec, [(3, 0, (16256, 16384)), (3, 31, (0, 128)), (1, 9, (2944, 3072)), (0, 4, (512, 640))])
+
+
+@pytest.mark.parametrize("name,gran", [("sweep_S32768_D64_causal", "per_thread"), ("sweep_S1024_D128", "per_warp"),
+                                       ("sweep_S8192_D128_causal", "per_block")])
+def test_sweep_points(name, gran):
+    spec = synth.CONFIGS[name]
+    last = spec.S - 128
+    _check(spec, [(0, 0, (0, 128)), (spec.B - 1, 31, (last, spec.S))], gran=gran)
