@@ -33,14 +33,14 @@ struct AttnCfg {
   static constexpr int NQ = ACC2 ? 1 : 2;          // query tiles per CTA
   static constexpr int NSB = ACC2 ? 2 : 1;         // S buffers per query tile
   static constexpr int NST = 3;                    // K/V pipeline stages
-  static constexpr int NTHREADS = (NQ + 2) * 128;
+  static constexpr int NTHREADS = 384;             // 3 warpgroups (168 registers per thread)
   static constexpr int QT = kTile * D;             // bytes of a Q or K tile
   static constexpr int VT = D * kTile * (PV8 ? 1 : 2);
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NQ * QT;
   static constexpr int OFF_V = OFF_K + NST * QT;
-  static constexpr int OFF_ALPHA = OFF_V + NST * VT;          // float [NQ][2][128]
-  static constexpr int OFF_L = OFF_ALPHA + NQ * 2 * 128 * 4;  // float [NQ][128]
+  static constexpr int OFF_ALPHA = OFF_V + NST * VT;          // float [NQ][2][128]   (two-level)
+  static constexpr int OFF_L = OFF_ALPHA + NQ * 2 * 128 * 4;  // float [NQ][128]      (two-level)
   static constexpr int OFF_BAR = OFF_L + NQ * 128 * 4;
   enum {
     B_QFULL = 0,
@@ -49,12 +49,12 @@ struct AttnCfg {
     B_VFULL = B_KEMPTY + NST,
     B_VEMPTY = B_VFULL + NST,
     B_SFULL = B_VEMPTY + NST,
-    B_PFULL = B_SFULL + NQ * NSB,
-    B_OFULL = B_PFULL + NQ,
-    B_OREADY = B_OFULL + NQ,
-    B_AFULL = B_OREADY + NQ,
+    B_PFULL = B_SFULL + NQ * NSB,    // softmax -> MMA: P~ in TMEM (and O rescaled)
+    B_OFULL = B_PFULL + NQ,          // MMA -> consumer of O (every PV two-level, last PV one-level)
+    B_OREADY = B_OFULL + NQ,         // correction -> MMA: partial O consumed (two-level)
+    B_AFULL = B_OREADY + NQ,         // softmax -> correction: alpha (two-level)
     B_AEMPTY = B_AFULL + 2 * NQ,
-    B_LFULL = B_AEMPTY + 2 * NQ,
+    B_LFULL = B_AEMPTY + 2 * NQ,     // softmax -> correction: final row sum (two-level)
     B_DONE = B_LFULL + NQ,
     NBAR = B_DONE + 1
   };
@@ -71,91 +71,142 @@ struct AttnCfg {
 };
 
 // ---------------------------------------------------------------- softmax
-// One pass over the 128 scores of this thread's row in 32-column chunks.
-// KPT: per-thread K groups ((col/64)*8 + col%8) else per-64-key groups.
+// KPT: per-thread K groups ((col/64)*8 + col%8), else per-64-key groups.
 template <bool KPT>
-__device__ __forceinline__ int kgrp(int col) {
+__device__ __forceinline__ constexpr int kgrp(int col) {
   return KPT ? ((col >> 6) << 3) + (col & 7) : (col >> 6);
 }
 
-template <bool KPT, bool PV8>
-__device__ __forceinline__ void softmax_tile(uint32_t taddr, const float (&c)[16], bool masked, int col0,
-                                             int lim, float& m, float& l, float& alpha_out,
-                                             uint32_t alpha_bar_full, uint32_t alpha_bar_empty,
-                                             uint32_t alpha_parity, float* alpha_slot,
-                                             volatile int* abort_flag, uint32_t* err, bool out_bf16,
-                                             bool& ok) {
-  // pass 1: integer maximum per scale group (c > 0, so max(S*c) = c*max(S))
-  int mx[16];
+// One 128-key tile of one query row (this thread's TMEM lane):
+//   S (int32, TMEM) -> exact float (magic-number add) -> group maxima of the
+//   unscaled scores -> m_tile = max_g c_g * max_g(S) -> alpha -> exponent
+//   argument S*c - m (one packed FFMA), ex2, row sum -> P~ rounded to E4M3
+//   (448 folded into the exponent) or 16 bits, written over the S columns.
+// c[g] = dQ * dK_g * sm_scale * log2(e), positive or zero.
+template <bool PV8, bool KPT>
+__device__ __forceinline__ void softmax_tile(uint32_t taddr, const float (&c)[16], bool masked, int col0, int lim,
+                                             bool bf16p, float& m, float& l, float& alpha) {
+  uint32_t r[128];
+  tmem_ld128_sync(taddr, r);
+  float f[128];
 #pragma unroll
-  for (int g = 0; g < 16; ++g) mx[g] = INT_MIN;
+  for (int k = 0; k < 64; ++k)
+    add2(f[2 * k], f[2 * k + 1], __uint_as_float(r[2 * k] + 0x4B400000u), __uint_as_float(r[2 * k + 1] + 0x4B400000u),
+         -12582912.0f, -12582912.0f);
+  if (masked) {
 #pragma unroll
-  for (int ch = 0; ch < 4; ++ch) {
-    uint32_t r[32];
-    tmem_ld32(taddr + ch * 32, r);
-    tmem_wait_ld(r);
-#pragma unroll
-    for (int u = 0; u < 32; ++u) {
-      const int col = ch * 32 + u;
-      const bool valid = !masked || (col0 + col < lim);
-      if (valid) mx[kgrp<KPT>(col)] = max(mx[kgrp<KPT>(col)], (int)r[u]);
-    }
+    for (int i = 0; i < 128; ++i)
+      if (!(col0 + i < lim)) f[i] = -INFINITY;
   }
+  // maxima of the unscaled scores per scale group (c >= 0 keeps the order)
   float mt = -INFINITY;
+  if (KPT) {
 #pragma unroll
-  for (int g = 0; g < (KPT ? 16 : 2); ++g)
-    if (mx[g] != INT_MIN) mt = fmaxf(mt, c[g] * i2f_exact(mx[g]));
-  const float m_new = fmaxf(m, mt);
-  const float alpha = (m == -INFINITY) ? 0.f : ex2(m - m_new);
-  alpha_out = alpha;
-  // publish alpha for the correction warpgroup
-  if (!mbar_wait(alpha_bar_empty, alpha_parity ^ 1u, abort_flag, err, kErrTimeoutSoftmax)) { ok = false; return; }
-  *alpha_slot = alpha;
-  mbar_arrive(alpha_bar_full);
-
-  // pass 2: P~ = 2^(s - m_new) (times 448 in FP8 mode: the static scale is
-  // folded into the exponent), row sum, P~ packed over the S columns
-  const float bias = PV8 ? (m_new - kLog2Fp8Max) : m_new;
-  float lsum = 0.f;
-#pragma unroll
-  for (int ch = 0; ch < 4; ++ch) {
-    uint32_t r[32];
-    tmem_ld32(taddr + ch * 32, r);
-    tmem_wait_ld(r);
-    float pv[32];
-#pragma unroll
-    for (int u = 0; u < 32; ++u) {
-      const int col = ch * 32 + u;
-      const float s = fmaf(i2f_exact((int)r[u]), c[kgrp<KPT>(col)], -bias);
-      float p = ex2(s);
-      if (masked && !(col0 + col < lim)) p = 0.f;
-      pv[u] = p;
-      lsum += p;
+    for (int g = 0; g < 16; ++g) {
+      const int base = (g >> 3) * 64 + (g & 7);
+      float a = max3(f[base], f[base + 8], f[base + 16]);
+      float b = max3(f[base + 24], f[base + 32], f[base + 40]);
+      a = max3(a, b, fmaxf(f[base + 48], f[base + 56]));
+      if (a != -INFINITY) mt = fmaxf(mt, c[g] * a);
     }
-    if (PV8) {
-      uint32_t w[8];
+  } else {
 #pragma unroll
-      for (int k = 0; k < 8; ++k) w[k] = pack_e4m3x4(pv[4 * k], pv[4 * k + 1], pv[4 * k + 2], pv[4 * k + 3]);
-      tmem_st8(taddr + ch * 8, w);
-    } else {
-      uint32_t w[16];
-      if (out_bf16) {
+    for (int g = 0; g < 2; ++g) {
+      float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
-        for (int k = 0; k < 16; ++k) w[k] = pack_bf16x2(pv[2 * k], pv[2 * k + 1]);
-      } else {
-#pragma unroll
-        for (int k = 0; k < 16; ++k) w[k] = pack_f16x2(pv[2 * k], pv[2 * k + 1]);
+      for (int i = 0; i < 64; i += 8) {
+        a0 = max3(a0, f[64 * g + i], f[64 * g + i + 1]);
+        a1 = max3(a1, f[64 * g + i + 2], f[64 * g + i + 3]);
+        a2 = max3(a2, f[64 * g + i + 4], f[64 * g + i + 5]);
+        a3 = max3(a3, f[64 * g + i + 6], f[64 * g + i + 7]);
       }
-      tmem_st16(taddr + ch * 16, w);
+      const float a = max3(a0, a1, fmaxf(a2, a3));
+      if (a != -INFINITY) mt = fmaxf(mt, c[g] * a);
     }
   }
-  l = alpha * l + lsum;
+  const float m_new = fmaxf(m, mt);
+  alpha = (m == -INFINITY) ? 0.f : ex2(m - m_new);
+  const float nb = -(PV8 ? (m_new - kLog2Fp8Max) : m_new);
+  float ls0 = 0.f, ls1 = 0.f;
+#pragma unroll
+  for (int k = 0; k < 64; ++k) {
+    float a0, a1;
+    fma2(a0, a1, f[2 * k], f[2 * k + 1], c[kgrp<KPT>(2 * k)], c[kgrp<KPT>(2 * k + 1)], nb, nb);
+    float p0 = ex2(a0), p1 = ex2(a1);
+    if (masked) {
+      if (!(col0 + 2 * k < lim)) p0 = 0.f;
+      if (!(col0 + 2 * k + 1 < lim)) p1 = 0.f;
+    }
+    f[2 * k] = p0;
+    f[2 * k + 1] = p1;
+    add2(ls0, ls1, ls0, ls1, p0, p1);
+  }
+  l = alpha * l + (ls0 + ls1);
   m = m_new;
+  if (PV8) {
+    uint32_t w[32];
+#pragma unroll
+    for (int k = 0; k < 32; ++k) w[k] = pack_e4m3x4(f[4 * k], f[4 * k + 1], f[4 * k + 2], f[4 * k + 3]);
+    tmem_st32(taddr, w);
+  } else {
+    uint32_t w[32];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+#pragma unroll
+      for (int k = 0; k < 32; ++k)
+        w[k] = bf16p ? pack_bf16x2(f[64 * h + 2 * k], f[64 * h + 2 * k + 1])
+                     : pack_f16x2(f[64 * h + 2 * k], f[64 * h + 2 * k + 1]);
+      tmem_st32(taddr + 32 * h, w);
+    }
+  }
+}
+
+// Row epilogue: out[c] = O[c] * inv_l (* delta_V[c] in FP8 mode, where l sums
+// 448 * P~ and O sums P8 * V8, so the 448 cancels); 16-bit rounding, one row.
+template <int D, bool PV8, bool FROM_REGS>
+__device__ __forceinline__ void store_row(uint16_t* orow, uint32_t ob, const float* oacc, float inv_l,
+                                          const float* vsc, bool bf16, bool have_o, bool valid) {
+#pragma unroll
+  for (int ch = 0; ch < D / 32; ++ch) {
+    float o[32];
+    if (FROM_REGS) {
+#pragma unroll
+      for (int u = 0; u < 32; ++u) o[u] = oacc[ch * 32 + u];
+    } else {
+      uint32_t r[32];
+      if (have_o) {
+        tmem_ld32(ob + ch * 32, r);
+        tmem_wait_ld(r);
+      }
+#pragma unroll
+      for (int u = 0; u < 32; ++u) o[u] = have_o ? __uint_as_float(r[u]) : 0.f;
+    }
+    uint32_t w[16];
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      float a = o[2 * k] * inv_l, bb = o[2 * k + 1] * inv_l;
+      if (PV8) {
+        a *= __ldg(vsc + ch * 32 + 2 * k);
+        bb *= __ldg(vsc + ch * 32 + 2 * k + 1);
+      }
+      w[k] = bf16 ? pack_bf16x2(a, bb) : pack_f16x2(a, bb);
+    }
+    if (valid) {
+      uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
+#pragma unroll
+      for (int k = 0; k < 4; ++k) dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
+    }
+  }
 }
 
 // ---------------------------------------------------------------- kernel
+// Warp roles: 0 loader, 1 MMA issuer, 2 TMEM allocator, 3 idle; warpgroups
+// 1..NQ softmax (one query tile each).  One-level accumulation: the softmax
+// warpgroup also rescales O in TMEM (before releasing P~ to the MMA) and runs
+// the epilogue.  Two-level: warpgroup 2 is the correction warpgroup holding
+// the FP32 outer accumulator in registers.
 template <int D, bool PV8, bool ACC2>
-__global__ void __launch_bounds__(AttnCfg<D, PV8, ACC2>::NTHREADS, 1) attn_fwd_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
   using C = AttnCfg<D, PV8, ACC2>;
   constexpr int NQ = C::NQ, NSB = C::NSB, NST = C::NST;
   extern __shared__ uint8_t smem_raw[];
@@ -209,6 +260,7 @@ __global__ void __launch_bounds__(AttnCfg<D, PV8, ACC2>::NTHREADS, 1) attn_fwd_k
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc[0];
+  const float* vsc = p.v_scale + ((size_t)b * p.Hkv + hk) * D;
 
   if (warp == 0) {
     // ------------------------------------------------------------ loader
@@ -259,57 +311,68 @@ __global__ void __launch_bounds__(AttnCfg<D, PV8, ACC2>::NTHREADS, 1) attn_fwd_k
       for (int q = 0; q < NQ && ok; ++q)
         if (n[q] > 0) ok = mbar_wait(bar(C::B_QFULL + q), 0, abort_flag, p.err, kErrTimeoutMma);
       tc_fence_after();
-      auto issue_s = [&](int t) -> bool {
-        const int st = t % NST;
-        if (!mbar_wait(bar(C::B_KFULL + st), (t / NST) & 1, abort_flag, p.err, kErrTimeoutMma)) return false;
-        tc_fence_after();
-        for (int q = 0; q < NQ; ++q) {
-          if (t >= n[q]) continue;
-          const uint32_t d = tmem + C::TM_S + (q * NSB + t % NSB) * 128;
+      auto mma_s = [&](int q, int t, int st) {
+        const uint32_t d = tmem + C::TM_S + (q * NSB + t % NSB) * 128;
 #pragma unroll
-          for (int kk = 0; kk < D / 32; ++kk) {
-            const uint64_t a = smem_desc(sb + C::OFF_Q + q * C::QT + kk * 32, D);
-            const uint64_t bd = smem_desc(sb + C::OFF_K + st * C::QT + kk * 32, D);
-            mma_i8_ss(d, a, bd, ID_QK, kk > 0);
-          }
-          tc_commit(bar(C::B_SFULL + q * NSB + t % NSB));
+        for (int kk = 0; kk < D / 32; ++kk) {
+          const uint64_t a = smem_desc(sb + C::OFF_Q + q * C::QT + kk * 32, D);
+          const uint64_t bd = smem_desc(sb + C::OFF_K + st * C::QT + kk * 32, D);
+          mma_i8_ss(d, a, bd, ID_QK, kk > 0);
         }
-        tc_commit(bar(C::B_KEMPTY + st));
-        return true;
+        tc_commit(bar(C::B_SFULL + q * NSB + t % NSB));
       };
-      for (int t = 0; t < NSB && t < maxn && ok; ++t) ok = issue_s(t);
-      for (int j = 0; j < maxn && ok; ++j) {
-        const int st = j % NST;
-        if (!(ok = mbar_wait(bar(C::B_VFULL + st), (j / NST) & 1, abort_flag, p.err, kErrTimeoutMma))) break;
+      auto mma_pv = [&](int q, int j, int st) {
+        const uint32_t a0 = tmem + C::TM_S + (q * NSB + j % NSB) * 128;
+        const uint32_t d = tmem + C::TM_O + q * D;
+        if (PV8) {
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_f8_ts(d, a0 + kk * 8, smem_desc(sb + C::OFF_V + st * C::VT + kk * 32, 128), ID_PV,
+                      ACC2 ? (kk > 0) : (j > 0 || kk > 0));
+        } else {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk)
+            mma_f16_ts(d, a0 + kk * 8,
+                       smem_desc(sb + C::OFF_V + st * C::VT + (kk >> 2) * (D * 128) + (kk & 3) * 32, 128), ID_PV,
+                       ACC2 ? (kk > 0) : (j > 0 || kk > 0));
+        }
+      };
+      // S for the first NSB tiles
+      for (int t = 0; t < NSB && t < maxn && ok; ++t) {
+        ok = mbar_wait(bar(C::B_KFULL + t % NST), (t / NST) & 1, abort_flag, p.err, kErrTimeoutMma);
+        if (!ok) break;
         tc_fence_after();
+        for (int q = 0; q < NQ; ++q)
+          if (t < n[q]) mma_s(q, t, t % NST);
+        tc_commit(bar(C::B_KEMPTY + t % NST));
+      }
+      for (int j = 0; j < maxn && ok; ++j) {
+        const int st = j % NST, t = j + NSB;
+        if (!(ok = mbar_wait(bar(C::B_VFULL + st), (j / NST) & 1, abort_flag, p.err, kErrTimeoutMma))) break;
+        bool kready = false;
         for (int q = 0; q < NQ && ok; ++q) {
-          if (j >= n[q]) continue;
-          ok = mbar_wait(bar(C::B_PFULL + q), j & 1, abort_flag, p.err, kErrTimeoutMma);
-          if (ok && (!ACC2 || j > 0))
-            ok = mbar_wait(bar(C::B_OREADY + q), (ACC2 ? (j - 1) : j) & 1, abort_flag, p.err, kErrTimeoutMma);
-          if (!ok) break;
-          tc_fence_after();
-          const uint32_t a0 = tmem + C::TM_S + (q * NSB + j % NSB) * 128;
-          const uint32_t d = tmem + C::TM_O + q * D;
-          if (PV8) {
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-              const uint64_t bd = smem_desc(sb + C::OFF_V + st * C::VT + kk * 32, 128);
-              mma_f8_ts(d, a0 + kk * 8, bd, ID_PV, ACC2 ? (kk > 0) : (j > 0 || kk > 0));
-            }
-          } else {
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-              const uint64_t bd =
-                  smem_desc(sb + C::OFF_V + st * C::VT + (kk >> 2) * (D * 128) + (kk & 3) * 32, 128);
-              mma_f16_ts(d, a0 + kk * 8, bd, ID_PV, ACC2 ? (kk > 0) : (j > 0 || kk > 0));
-            }
+          if (j < n[q]) {
+            ok = mbar_wait(bar(C::B_PFULL + q), j & 1, abort_flag, p.err, kErrTimeoutMma);
+            if (ok && ACC2 && j > 0)
+              ok = mbar_wait(bar(C::B_OREADY + q), (j - 1) & 1, abort_flag, p.err, kErrTimeoutMma);
+            if (!ok) break;
+            tc_fence_after();
+            mma_pv(q, j, st);
+            if (ACC2 || j == n[q] - 1) tc_commit(bar(C::B_OFULL + q));
           }
-          tc_commit(bar(C::B_OFULL + q));
+          if (t < n[q]) {
+            if (!kready) {
+              if (!(ok = mbar_wait(bar(C::B_KFULL + t % NST), (t / NST) & 1, abort_flag, p.err, kErrTimeoutMma)))
+                break;
+              tc_fence_after();
+              kready = true;
+            }
+            mma_s(q, t, t % NST);
+          }
         }
         if (!ok) break;
         tc_commit(bar(C::B_VEMPTY + st));
-        if (j + NSB < maxn) ok = issue_s(j + NSB);
+        if (kready) tc_commit(bar(C::B_KEMPTY + t % NST));
       }
       // all MMAs issued by this thread complete before teardown
       tc_commit(bar(C::B_DONE));
@@ -322,15 +385,19 @@ __global__ void __launch_bounds__(AttnCfg<D, PV8, ACC2>::NTHREADS, 1) attn_fwd_k
     const int t = tid - 128 * (1 + q);
     const int qt = pair * NQ + q;
     const uint32_t lane_off = (uint32_t)((t & ~31)) << 16;
+    const int row = qt * kTile + t;
+    const bool bf16 = p.out_bf16 != 0;
     float m = -INFINITY, l = 0.f;
+    bool ok = true;
     if (n[q] > 0) {
       const float qsc = p.q_scale[((size_t)h * p.tiles_q + tq0 + qt) * kQGroupsMax + q_group(p.gran, t)];
       const float* ksb = p.k_scale + ((size_t)hk * p.tiles_k + tk0) * kKGroupsMax;
       const bool kpt = p.gran == 2;
-      const int row = qt * kTile + t;
+      const uint32_t ob = tmem + C::TM_O + q * D + lane_off;
       for (int j = 0; j < n[q]; ++j) {
         const int buf = j % NSB;
-        if (!mbar_wait(bar(C::B_SFULL + q * NSB + buf), (j / NSB) & 1, abort_flag, p.err, kErrTimeoutSoftmax)) break;
+        if (!(ok = mbar_wait(bar(C::B_SFULL + q * NSB + buf), (j / NSB) & 1, abort_flag, p.err, kErrTimeoutSoftmax)))
+          break;
         tc_fence_after();
         float c[16];
 #pragma unroll
@@ -340,120 +407,94 @@ __global__ void __launch_bounds__(AttnCfg<D, PV8, ACC2>::NTHREADS, 1) attn_fwd_k
         const bool masked = (col0 + kTile > Lk) || (p.causal && j == qt);
         const int lim = p.causal ? min(Lk, row + 1) : Lk;
         const uint32_t taddr = tmem + C::TM_S + (q * NSB + buf) * 128 + lane_off;
-        const int ab = j & 1;
         float alpha;
-        bool ok = true;
-        if (kpt)
-          softmax_tile<true, PV8>(taddr, c, masked, col0, lim, m, l, alpha, bar(C::B_AFULL + 2 * q + ab),
-                                  bar(C::B_AEMPTY + 2 * q + ab), (j >> 1) & 1, alpha_s + (q * 2 + ab) * 128 + t,
-                                  abort_flag, p.err, p.out_bf16 != 0, ok);
-        else
-          softmax_tile<false, PV8>(taddr, c, masked, col0, lim, m, l, alpha, bar(C::B_AFULL + 2 * q + ab),
-                                   bar(C::B_AEMPTY + 2 * q + ab), (j >> 1) & 1, alpha_s + (q * 2 + ab) * 128 + t,
-                                   abort_flag, p.err, p.out_bf16 != 0, ok);
-        if (!ok) break;
+        if (kpt) softmax_tile<PV8, true>(taddr, c, masked, col0, lim, bf16, m, l, alpha);
+        else softmax_tile<PV8, false>(taddr, c, masked, col0, lim, bf16, m, l, alpha);
+        if (ACC2) {
+          const int ab = j & 1;
+          if (!(ok = mbar_wait(bar(C::B_AEMPTY + 2 * q + ab), ((j >> 1) & 1) ^ 1, abort_flag, p.err,
+                               kErrTimeoutSoftmax)))
+            break;
+          alpha_s[(q * 2 + ab) * 128 + t] = alpha;
+          mbar_arrive(bar(C::B_AFULL + 2 * q + ab));
+        } else if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          // O(q) holds the sums of tiles < j (PV_{j-1} finished before S_j did)
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t r[32];
+            tmem_ld32(ob + ch * 32, r);
+            tmem_wait_ld(r);
+#pragma unroll
+            for (int u = 0; u < 32; u += 2) {
+              float x0, x1;
+              mul2(x0, x1, __uint_as_float(r[u]), __uint_as_float(r[u + 1]), alpha, alpha);
+              r[u] = __float_as_uint(x0);
+              r[u + 1] = __float_as_uint(x1);
+            }
+            tmem_st32(ob + ch * 32, r);
+          }
+        }
         tmem_wait_st();
         tc_fence_before();
         mbar_arrive(bar(C::B_PFULL + q));
       }
     }
-    l_s[q * 128 + t] = l;
-    mbar_arrive(bar(C::B_LFULL + q));
-  } else if (warp >= 4 + 4 * NQ) {
-    // ------------------------------------------------------------ correction + epilogue
-    const int t = tid - 128 * (1 + NQ);
-    const uint32_t lane_off = (uint32_t)((t & ~31)) << 16;
-    bool ok = true;
-    float oacc[ACC2 ? D : 1];
-#pragma unroll
-    for (int i = 0; i < (ACC2 ? D : 1); ++i) oacc[i] = 0.f;
-    for (int j = 0; j < maxn && ok; ++j) {
-      for (int q = 0; q < NQ && ok; ++q) {
-        if (j >= n[q]) continue;
-        const int ab = j & 1;
-        if (!(ok = mbar_wait(bar(C::B_AFULL + 2 * q + ab), (j >> 1) & 1, abort_flag, p.err, kErrTimeoutCorr))) break;
-        const float alpha = alpha_s[(q * 2 + ab) * 128 + t];
-        mbar_arrive(bar(C::B_AEMPTY + 2 * q + ab));
-        const uint32_t ob = tmem + C::TM_O + q * D + lane_off;
-        if (ACC2) {
-          if (!(ok = mbar_wait(bar(C::B_OFULL + q), j & 1, abort_flag, p.err, kErrTimeoutCorr))) break;
-          tc_fence_after();
-#pragma unroll
-          for (int ch = 0; ch < D / 16; ++ch) {
-            uint32_t r[16];
-            tmem_ld16(ob + ch * 16, r);
-            tmem_wait_ld(r);
-#pragma unroll
-            for (int u = 0; u < 16; ++u) oacc[ch * 16 + u] = fmaf(alpha, oacc[ch * 16 + u], __uint_as_float(r[u]));
-          }
-        } else if (j > 0) {
-          if (!(ok = mbar_wait(bar(C::B_OFULL + q), (j - 1) & 1, abort_flag, p.err, kErrTimeoutCorr))) break;
-          tc_fence_after();
-          if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-            for (int ch = 0; ch < D / 32; ++ch) {
-              uint32_t r[32];
-              tmem_ld32(ob + ch * 32, r);
-              tmem_wait_ld(r);
-#pragma unroll
-              for (int u = 0; u < 32; ++u) r[u] = __float_as_uint(__uint_as_float(r[u]) * alpha);
-              tmem_st32(ob + ch * 32, r);
-            }
-            tmem_wait_st();
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(bar(C::B_OREADY + q));
+    if (ACC2) {
+      l_s[q * 128 + t] = l;
+      mbar_arrive(bar(C::B_LFULL + q));
+    } else if (ok && qt * kTile < Lq) {
+      // epilogue of this query tile
+      if (n[q] > 0) {
+        ok = mbar_wait(bar(C::B_OFULL + q), 0, abort_flag, p.err, kErrTimeoutSoftmax);
+        tc_fence_after();
+      }
+      if (ok) {
+        uint16_t* orow = reinterpret_cast<uint16_t*>(p.out) + (long long)b * p.os.sb + (long long)h * p.os.sh +
+                         (long long)(qs + row) * p.os.ss;
+        store_row<D, PV8, false>(orow, tmem + C::TM_O + q * D + lane_off, nullptr, l > 0.f ? 1.0f / l : 0.f, vsc,
+                                 bf16, n[q] > 0, row < Lq);
       }
     }
-    // epilogue: out = O * (delta_V / l)   (FP8: l sums 448 * P~, O sums
-    // P8 * V8, so the 448 cancels) or O / l (16-bit)
-    const float* vsc = p.v_scale + ((size_t)b * p.Hkv + hk) * D;
-    for (int q = 0; q < NQ && ok; ++q) {
-      const int qt = pair * NQ + q;
-      const int row = qt * kTile + t;
-      if (qt * kTile >= Lq) continue;
-      float l = 0.f;
-      if (n[q] > 0) {
-        if (!ACC2 && !(ok = mbar_wait(bar(C::B_OFULL + q), (n[q] - 1) & 1, abort_flag, p.err, kErrTimeoutCorr))) break;
-        if (!(ok = mbar_wait(bar(C::B_LFULL + q), 0, abort_flag, p.err, kErrTimeoutCorr))) break;
-        tc_fence_after();
-        l = l_s[q * 128 + t];
+  } else if (ACC2 && warp >= 4 + 4 * NQ) {
+    // ------------------------------------------------------------ correction (two-level) + epilogue
+    const int t = tid - 128 * (1 + NQ);
+    const uint32_t lane_off = (uint32_t)((t & ~31)) << 16;
+    const uint32_t ob = tmem + C::TM_O + lane_off;
+    bool ok = true;
+    float oacc[D];
+#pragma unroll
+    for (int i = 0; i < D; ++i) oacc[i] = 0.f;
+    for (int j = 0; j < n[0] && ok; ++j) {
+      const int ab = j & 1;
+      if (!(ok = mbar_wait(bar(C::B_AFULL + ab), (j >> 1) & 1, abort_flag, p.err, kErrTimeoutCorr))) break;
+      const float alpha = alpha_s[ab * 128 + t];
+      mbar_arrive(bar(C::B_AEMPTY + ab));
+      if (!(ok = mbar_wait(bar(C::B_OFULL), j & 1, abort_flag, p.err, kErrTimeoutCorr))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int ch = 0; ch < D / 16; ++ch) {
+        uint32_t r[16];
+        tmem_ld16(ob + ch * 16, r);
+        tmem_wait_ld(r);
+#pragma unroll
+        for (int u = 0; u < 16; u += 2)
+          fma2(oacc[ch * 16 + u], oacc[ch * 16 + u + 1], alpha, alpha, oacc[ch * 16 + u], oacc[ch * 16 + u + 1],
+               __uint_as_float(r[u]), __uint_as_float(r[u + 1]));
       }
-      const float inv_l = l > 0.f ? 1.0f / l : 0.f;
-      uint16_t* orow = reinterpret_cast<uint16_t*>(p.out) + (long long)b * p.os.sb + (long long)h * p.os.sh +
-                       (long long)(qs + row) * p.os.ss;
-      const uint32_t ob = tmem + C::TM_O + q * D + lane_off;
-#pragma unroll
-      for (int ch = 0; ch < D / 32; ++ch) {
-        float o[32];
-        if (ACC2) {
-#pragma unroll
-          for (int u = 0; u < 32; ++u) o[u] = oacc[ch * 32 + u];
-        } else {
-          uint32_t r[32];
-          if (n[q] > 0) {
-            tmem_ld32(ob + ch * 32, r);
-            tmem_wait_ld(r);
-          }
-#pragma unroll
-          for (int u = 0; u < 32; ++u) o[u] = n[q] > 0 ? __uint_as_float(r[u]) : 0.f;
-        }
-        uint32_t w[16];
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          float a = o[2 * k] * inv_l, bb = o[2 * k + 1] * inv_l;
-          if (PV8) {
-            a *= __ldg(vsc + ch * 32 + 2 * k);
-            bb *= __ldg(vsc + ch * 32 + 2 * k + 1);
-          }
-          w[k] = p.out_bf16 ? pack_bf16x2(a, bb) : pack_f16x2(a, bb);
-        }
-        if (row < Lq) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + ch * 32);
-#pragma unroll
-          for (int k = 0; k < 4; ++k) dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
-        }
+      tc_fence_before();
+      mbar_arrive(bar(C::B_OREADY));
+    }
+    const int row = pair * kTile + t;
+    if (ok && pair * kTile < Lq) {
+      float l = 0.f;
+      if (n[0] > 0) {
+        ok = mbar_wait(bar(C::B_LFULL), 0, abort_flag, p.err, kErrTimeoutCorr);
+        l = l_s[t];
+      }
+      if (ok) {
+        uint16_t* orow = reinterpret_cast<uint16_t*>(p.out) + (long long)b * p.os.sb + (long long)h * p.os.sh +
+                         (long long)(qs + row) * p.os.ss;
+        store_row<D, PV8, true>(orow, ob, oacc, l > 0.f ? 1.0f / l : 0.f, vsc, p.out_bf16 != 0, true, row < Lq);
       }
     }
   }
