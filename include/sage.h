@@ -122,6 +122,7 @@ typedef struct {
   size_t err;       /* uint32 device error word */
   size_t tile_off_q, tile_off_k;   /* int32 [n_seqs+1] (varlen) */
   size_t k_stat, v_stat;           /* pre-pass accumulators */
+  size_t sched;                    /* pre-pass work counters and varlen item offsets */
   size_t k_mean, v_scale;
   size_t q_codes, q_scale, k_codes, k_scale, v_codes;
   size_t q_mean, q_bias;
@@ -147,6 +148,13 @@ sage_status_t sage_quant_qk(const void* q, const void* k, sage_dtype_t dtype, sa
                             int B, int Hq, int Hkv, int S, int D, sage_gran_t gran,
                             int smooth_k, int smooth_q, void* ws, size_t ws_bytes, void* stream);
 
+/* The whole pre-pass in one launch: sage_quant_qk and sage_quant_v together
+ * (Q, K and V read once from HBM; K and V are read a second time from L2). */
+sage_status_t sage_quant_qkv(const void* q, const void* k, const void* v, sage_dtype_t dtype,
+                             sage_layout_t layout, int B, int Hq, int Hkv, int S, int D,
+                             sage_gran_t gran, sage_pv_t pv, int smooth_k, int smooth_q, void* ws,
+                             size_t ws_bytes, void* stream);
+
 /* Quantize V per channel to E4M3 (pv == SAGE_PV_FP8) or re-lay it out in 16
  * bits (SAGE_PV_FP16), transposed to [D][keys] tiles.  [SageAttention2
  * summary, SageAttention2方法, FP8 quantization of P~V]  Writes v_stat,
@@ -157,8 +165,7 @@ sage_status_t sage_quant_v(const void* v, sage_dtype_t dtype, sage_layout_t layo
 /* ------------------------------------------------------------------------ */
 /* Attention.                                                               */
 /* ------------------------------------------------------------------------ */
-/* The whole forward pass: sage_quant_qk + sage_quant_v + the attention
- * kernel.  out has q's shape, layout and dtype.  [Install/tuning guide,
+/* The whole forward pass: sage_quant_qkv + the attention kernel.  out has q's shape, layout and dtype.  [Install/tuning guide,
  * 五分钟跑通 and 性能调优实战] */
 sage_status_t sage_attn_fwd(const void* q, const void* k, const void* v, void* out,
                             sage_dtype_t dtype, int B, int Hq, int Hkv, int S, int D,
@@ -188,6 +195,40 @@ sage_status_t sage_attn_varlen_fwd(const void* q, const void* k, const void* v, 
                                    float sm_scale, sage_gran_t gran, sage_pv_t pv,
                                    sage_acc_t pv_accum, int smooth_k, void* ws, size_t ws_bytes,
                                    void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* Allocation-free forward pass.                                            */
+/* ------------------------------------------------------------------------ */
+/* The pages have no counterpart to this call; it is a convenience of this
+ * library for callers that cannot allocate device memory where they run
+ * attention -- e.g. a plugin inside an engine that has already reserved the
+ * device's memory for its own pool, code held to a fixed memory budget after
+ * start-up, or latency-critical code that cannot accept cudaMalloc's implicit
+ * device synchronization.
+ *
+ * Same arguments and result as sage_attn_fwd (without smooth_q and without a
+ * workspace).  The workspace is a static device array of
+ * SAGE_NOALLOC_SCRATCH_BYTES inside the library: every GPU that loads the
+ * library holds it until the process exits.  Problems whose workspace
+ * (sage_workspace_bytes) exceeds that size are rejected with
+ * SAGE_ERR_WORKSPACE before anything is launched.
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture on the device.
+ *   - No device memory is allocated or freed, by this call or the library.
+ *   - All calls on a device share the one array: calls whose work overlaps on
+ *     the GPU (different streams, or different host threads) race and may
+ *     produce wrong results.  Serialize them (one stream, or events).
+ *   - Device-side timeouts are recorded in the shared array and cleared by
+ *     the next call; use sage_attn_fwd with your own workspace to read them
+ *     through sage_get_device_error. */
+#define SAGE_NOALLOC_SCRATCH_BYTES ((size_t)32 << 20)
+
+sage_status_t sage_attn_fwd_noalloc(const void* q, const void* k, const void* v, void* out,
+                                    sage_dtype_t dtype, int B, int Hq, int Hkv, int S, int D,
+                                    sage_layout_t layout, int is_causal, float sm_scale,
+                                    sage_gran_t gran, sage_pv_t pv, sage_acc_t pv_accum,
+                                    int smooth_k, void* stream);
 
 /* ------------------------------------------------------------------------ */
 /* Diagnostics.                                                             */

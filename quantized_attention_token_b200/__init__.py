@@ -18,7 +18,7 @@ import os
 from typing import Optional
 
 __all__ = [
-    "sageattn", "sageattn_varlen", "quant_qk", "quant_v", "attn_quantized", "workspace_layout",
+    "sageattn", "sageattn_varlen", "quant_qk", "quant_qkv", "quant_v", "attn_quantized", "workspace_layout",
     "get_device_error", "debug_qk_tile", "Workspace", "SageError", "lib", "LIB_PATH",
 ]
 
@@ -40,7 +40,7 @@ class SageError(RuntimeError):
 
 class WsLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
-        "err", "tile_off_q", "tile_off_k", "k_stat", "v_stat", "k_mean", "v_scale", "q_codes",
+        "err", "tile_off_q", "tile_off_k", "k_stat", "v_stat", "sched", "k_mean", "v_scale", "q_codes",
         "q_scale", "k_codes", "k_scale", "v_codes", "q_mean", "q_bias", "total")] + [
         ("tiles_q", ctypes.c_int), ("tiles_k", ctypes.c_int)]
 
@@ -64,6 +64,7 @@ def lib():
         "sage_workspace_layout": (I, [I, I, I, I, I, I, I, I, I, I, ctypes.POINTER(WsLayout)]),
         "sage_quant_qk": (I, [P, P, I, I, I, I, I, I, I, I, I, I, P, Z, P]),
         "sage_quant_v": (I, [P, I, I, I, I, I, I, I, P, Z, P]),
+        "sage_quant_qkv": (I, [P, P, P, I, I, I, I, I, I, I, I, I, I, I, P, Z, P]),
         "sage_attn_fwd": (I, [P, P, P, P, I, I, I, I, I, I, I, I, F, I, I, I, I, I, P, Z, P]),
         "sage_attn_quantized": (I, [P, I, I, I, I, I, I, I, I, F, I, I, I, I, P, Z, P]),
         "sage_attn_varlen_fwd": (I, [P, P, P, P, I, P, P, I, I, I, I, I, I, I, I, F, I, I, I, I, P, Z, P]),
@@ -225,6 +226,21 @@ def quant_qk(q, k, ws, tensor_layout="HND", qk_quant_gran="per_block", smooth_k=
                              GRAN[qk_quant_gran], int(smooth_k), int(smooth_q), ws.data_ptr(), ws.numel(),
                              _stream(q.device))
     _check("sage_quant_qk", st)
+
+
+def quant_qkv(q, k, v, ws, tensor_layout="HND", qk_quant_gran="per_block", pv_dtype="fp8", smooth_k=True,
+              smooth_q=False):
+    """The whole smooth + quantize pre-pass (Q, K and V) in one launch."""
+    if tensor_layout == "HND":
+        B, Hq, S, D = q.shape
+        Hkv = k.shape[1]
+    else:
+        B, S, Hq, D = q.shape
+        Hkv = k.shape[2]
+    st = lib().sage_quant_qkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), _dtype_code(q), LAYOUT[tensor_layout], B,
+                              Hq, Hkv, S, D, GRAN[qk_quant_gran], PV[pv_dtype], int(smooth_k), int(smooth_q),
+                              ws.data_ptr(), ws.numel(), _stream(q.device))
+    _check("sage_quant_qkv", st)
 
 
 def quant_v(v, ws, tensor_layout="HND", pv_dtype="fp8"):

@@ -60,8 +60,11 @@ sage_status_t plan(int nseq, int total_q, int total_k, int max_seqlen, int Hq, i
   L->err = take(256, 256);
   L->tile_off_q = take(varlen ? sizeof(int) * (nseq + 1) : 0, 256);
   L->tile_off_k = take(varlen ? sizeof(int) * (nseq + 1) : 0, 256);
+  // k_stat, v_stat and the pre-pass counters are contiguous: one memset
+  // zeroes them before each pre-pass launch
   L->k_stat = take(nd * 8, 256);
-  L->v_stat = take(nd * 4, 256);
+  L->v_stat = take(nd * 4, 4);
+  L->sched = take(4 * (1 + (size_t)nseq * Hkv) + 4 * (size_t)(nseq + 1), 4);
   L->k_mean = take(nd * 4, 256);
   L->v_scale = take(nd * 4, 256);
   L->k_codes = take((size_t)Hkv * tk * kTile * D, 1024);
@@ -96,58 +99,58 @@ sage_status_t check_common(sage_dtype_t dtype, int D, sage_gran_t gran, sage_pv_
   return SAGE_OK;
 }
 
-PrepassParams base_params(void* ws, const sage_ws_layout_t& L, const Seqs& seqs, int bf16) {
-  PrepassParams p{};
-  p.seqs = seqs;
-  p.bf16 = bf16;
-  p.err = at<uint32_t>(ws, L.err);
-  p.k_stat = at<unsigned long long>(ws, L.k_stat);
-  p.v_stat = at<uint32_t>(ws, L.v_stat);
-  p.k_mean = at<float>(ws, L.k_mean);
-  p.v_scale = at<float>(ws, L.v_scale);
-  return p;
+// Bytes from k_stat to the end of the pre-pass counters (zeroed per launch).
+size_t stats_zero_bytes(const sage_ws_layout_t& L, int nseq, int Hkv) {
+  return L.sched + 4 * (1 + (size_t)nseq * Hkv) - L.k_stat;
 }
 
-// Q/K pre-pass for dense or varlen problems (stats region zeroed here).
-sage_status_t run_quant_qk(const void* q, const void* k, int bf16, Strides sq, Strides sk, const Seqs& seqs,
-                           int nseq, int Hq, int Hkv, int D, int gran, int smooth_k, int smooth_q, void* ws,
-                           const sage_ws_layout_t& L, cudaStream_t s) {
-  if (cudaMemsetAsync(at<char>(ws, L.k_stat), 0, (size_t)nseq * Hkv * D * 8, s) != cudaSuccess)
+// The persistent pre-pass over any of Q, K, V (dense or varlen).
+sage_status_t run_prepass(const void* q, const void* k, const void* v, int bf16, Strides sq, Strides sk,
+                          Strides sv, const Seqs& seqs, int nseq, int Hq, int Hkv, int D, int gran, int pv,
+                          int smooth_k, int smooth_q, void* ws, const sage_ws_layout_t& L, cudaStream_t s) {
+  if (cudaMemsetAsync(at<char>(ws, L.k_stat), 0, stats_zero_bytes(L, nseq, Hkv), s) != cudaSuccess)
     return SAGE_ERR_CUDA;
-  PrepassParams pq = base_params(ws, L, seqs, bf16), pk = pq;
-  pq.x = static_cast<const uint16_t*>(q);
-  pq.st = sq;
-  pq.H = Hq;
-  pq.gran = gran;
-  pq.smooth = smooth_q;
-  pq.tiles = L.tiles_q;
-  pq.codes = at<int8_t>(ws, L.q_codes);
-  pq.scales = at<float>(ws, L.q_scale);
-  pq.q_mean = smooth_q ? at<float>(ws, L.q_mean) : nullptr;
-  pk.x = static_cast<const uint16_t*>(k);
-  pk.st = sk;
-  pk.H = Hkv;
-  pk.gran = gran;
-  pk.smooth = smooth_k;
-  pk.tiles = L.tiles_k;
-  pk.codes = at<int8_t>(ws, L.k_codes);
-  pk.scales = at<float>(ws, L.k_scale);
-  const int tps = cdiv(seqs.max_seqlen, kTile);
-  return cuda_status(prepass_qk(pq, pk, D, nseq, tps, tps, s));
-}
-
-sage_status_t run_quant_v(const void* v, int bf16, Strides sv, const Seqs& seqs, int nseq, int Hkv, int D,
-                          int pv, void* ws, const sage_ws_layout_t& L, cudaStream_t s) {
-  const bool pv8 = pv == SAGE_PV_FP8;
-  if (pv8 && cudaMemsetAsync(at<char>(ws, L.v_stat), 0, (size_t)nseq * Hkv * D * 4, s) != cudaSuccess)
+  PrepassJob j;
+  j.q = static_cast<const uint16_t*>(q);
+  j.k = static_cast<const uint16_t*>(k);
+  j.v = static_cast<const uint16_t*>(v);
+  j.sq = sq;
+  j.sk = sk;
+  j.sv = sv;
+  j.seqs = seqs;
+  j.nseq = nseq;
+  j.Hq = Hq;
+  j.Hkv = Hkv;
+  j.group = Hq / Hkv;
+  j.bf16 = bf16;
+  j.gran = gran;
+  j.smooth_k = smooth_k ? 1 : 0;
+  j.smooth_q = smooth_q ? 1 : 0;
+  j.pv8 = pv == SAGE_PV_FP8;
+  j.do_q = q != nullptr;
+  j.do_k = k != nullptr;
+  j.do_v = v != nullptr;
+  j.tiles_q = L.tiles_q;
+  j.tiles_k = L.tiles_k;
+  j.err = at<uint32_t>(ws, L.err);
+  j.k_stat = at<unsigned long long>(ws, L.k_stat);
+  j.v_stat = at<uint32_t>(ws, L.v_stat);
+  j.k_mean = at<float>(ws, L.k_mean);
+  j.v_scale = at<float>(ws, L.v_scale);
+  j.q_codes = at<int8_t>(ws, L.q_codes);
+  j.q_scale = at<float>(ws, L.q_scale);
+  j.k_codes = at<int8_t>(ws, L.k_codes);
+  j.k_scale = at<float>(ws, L.k_scale);
+  j.v_codes = at<uint8_t>(ws, L.v_codes);
+  j.q_mean = smooth_q ? at<float>(ws, L.q_mean) : nullptr;
+  j.ticket = at<uint32_t>(ws, L.sched);
+  j.stats_done = j.ticket + 1;
+  j.item_off = reinterpret_cast<int*>(j.stats_done + (size_t)nseq * Hkv);
+  if (seqs.cu_k &&
+      prepass_varlen_offsets(seqs.cu_q, seqs.cu_k, nseq, seqs.max_seqlen, L.tiles_q, L.tiles_k,
+                             const_cast<int*>(seqs.toff_q), const_cast<int*>(seqs.toff_k), j.err, j, s) != cudaSuccess)
     return SAGE_ERR_CUDA;
-  PrepassParams p = base_params(ws, L, seqs, bf16);
-  p.x = static_cast<const uint16_t*>(v);
-  p.st = sv;
-  p.H = Hkv;
-  p.tiles = L.tiles_k;
-  p.v_codes = at<uint8_t>(ws, L.v_codes);
-  return cuda_status(prepass_v(p, D, pv8, nseq, cdiv(seqs.max_seqlen, kTile), s));
+  return cuda_status(prepass_run(j, D, s));
 }
 
 sage_status_t run_attn(void* out, int bf16, Strides so, const Seqs& seqs, int nseq, int Hq, int Hkv, int D,
@@ -236,8 +239,9 @@ SAGE_EXPORT sage_status_t sage_quant_qk(const void* q, const void* k, sage_dtype
   if (ws_bytes < L.q_scale + (size_t)Hq * L.tiles_q * kQGroupsMax * 4) return SAGE_ERR_WORKSPACE;
   if ((st = check_device()) != SAGE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return run_quant_qk(q, k, dtype == SAGE_BF16, dense_strides(layout, Hq, S, D), dense_strides(layout, Hkv, S, D),
-                      dense_seqs(S), B, Hq, Hkv, D, gran, smooth_k, smooth_q, ws, L, s);
+  return run_prepass(q, k, nullptr, dtype == SAGE_BF16, dense_strides(layout, Hq, S, D),
+                     dense_strides(layout, Hkv, S, D), Strides{}, dense_seqs(S), B, Hq, Hkv, D, gran, SAGE_PV_FP8,
+                     smooth_k, smooth_q, ws, L, s);
 }
 
 SAGE_EXPORT sage_status_t sage_quant_v(const void* v, sage_dtype_t dtype, sage_layout_t layout, int B, int Hkv,
@@ -251,8 +255,27 @@ SAGE_EXPORT sage_status_t sage_quant_v(const void* v, sage_dtype_t dtype, sage_l
   if ((st = plan(B, B * S, B * S, S, Hkv, Hkv, D, pv, 0, 0, &L)) != SAGE_OK) return st;
   if (ws_bytes < L.q_codes) return SAGE_ERR_WORKSPACE;
   if ((st = check_device()) != SAGE_OK) return st;
-  return run_quant_v(v, dtype == SAGE_BF16, dense_strides(layout, Hkv, S, D), dense_seqs(S), B, Hkv, D, pv, ws, L,
-                     static_cast<cudaStream_t>(stream));
+  return run_prepass(nullptr, nullptr, v, dtype == SAGE_BF16, Strides{}, Strides{}, dense_strides(layout, Hkv, S, D),
+                     dense_seqs(S), B, Hkv, Hkv, D, SAGE_PER_BLOCK, pv, 0, 0, ws, L, static_cast<cudaStream_t>(stream));
+}
+
+SAGE_EXPORT sage_status_t sage_quant_qkv(const void* q, const void* k, const void* v, sage_dtype_t dtype,
+                                         sage_layout_t layout, int B, int Hq, int Hkv, int S, int D, sage_gran_t gran,
+                                         sage_pv_t pv, int smooth_k, int smooth_q, void* ws, size_t ws_bytes,
+                                         void* stream) {
+  sage_status_t st;
+  if ((st = check_dense(B, Hq, Hkv, S, D, layout)) != SAGE_OK) return st;
+  if ((st = check_common(dtype, D, gran, pv, SAGE_ACC_FP32)) != SAGE_OK) return st;
+  if (!q || !k || !v || !ws) return SAGE_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(ws, 256)) return SAGE_ERR_INVALID_ARG;
+  if (smooth_q) return SAGE_ERR_UNSUPPORTED;
+  sage_ws_layout_t L;
+  if ((st = plan(B, B * S, B * S, S, Hq, Hkv, D, pv, smooth_q, 0, &L)) != SAGE_OK) return st;
+  if (ws_bytes < L.total) return SAGE_ERR_WORKSPACE;
+  if ((st = check_device()) != SAGE_OK) return st;
+  return run_prepass(q, k, v, dtype == SAGE_BF16, dense_strides(layout, Hq, S, D), dense_strides(layout, Hkv, S, D),
+                     dense_strides(layout, Hkv, S, D), dense_seqs(S), B, Hq, Hkv, D, gran, pv, smooth_k, smooth_q,
+                     ws, L, static_cast<cudaStream_t>(stream));
 }
 
 SAGE_EXPORT sage_status_t sage_attn_quantized(void* out, sage_dtype_t dtype, int B, int Hq, int Hkv, int S, int D,
@@ -293,10 +316,9 @@ SAGE_EXPORT sage_status_t sage_attn_fwd(const void* q, const void* k, const void
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const int bf16 = dtype == SAGE_BF16;
   const Seqs seqs = dense_seqs(S);
-  if ((st = run_quant_qk(q, k, bf16, dense_strides(layout, Hq, S, D), dense_strides(layout, Hkv, S, D), seqs, B, Hq,
-                         Hkv, D, gran, smooth_k, smooth_q, ws, L, s)) != SAGE_OK)
-    return st;
-  if ((st = run_quant_v(v, bf16, dense_strides(layout, Hkv, S, D), seqs, B, Hkv, D, pv, ws, L, s)) != SAGE_OK)
+  if ((st = run_prepass(q, k, v, bf16, dense_strides(layout, Hq, S, D), dense_strides(layout, Hkv, S, D),
+                        dense_strides(layout, Hkv, S, D), seqs, B, Hq, Hkv, D, gran, pv, smooth_k, smooth_q, ws, L,
+                        s)) != SAGE_OK)
     return st;
   return run_attn(out, bf16, dense_strides(layout, Hq, S, D), seqs, B, Hq, Hkv, D, is_causal, sm_scale, gran, pv,
                   pv_accum, ws, L, s);
@@ -329,15 +351,11 @@ SAGE_EXPORT sage_status_t sage_attn_varlen_fwd(const void* q, const void* k, con
   seqs.toff_q = at<int>(ws, L.tile_off_q);
   seqs.toff_k = at<int>(ws, L.tile_off_k);
   seqs.max_seqlen = max_seqlen;
-  if (prepass_varlen_offsets(cu_seqlens_q, cu_seqlens_k, n_seqs, max_seqlen, L.tiles_q, L.tiles_k,
-                             at<int>(ws, L.tile_off_q), at<int>(ws, L.tile_off_k), at<uint32_t>(ws, L.err),
-                             s) != cudaSuccess)
-    return SAGE_ERR_CUDA;
   const int bf16 = dtype == SAGE_BF16;
   const Strides sq{0, (long long)D, (long long)Hq * D}, skv{0, (long long)D, (long long)Hkv * D};
-  if ((st = run_quant_qk(q, k, bf16, sq, skv, seqs, n_seqs, Hq, Hkv, D, gran, smooth_k, 0, ws, L, s)) != SAGE_OK)
+  if ((st = run_prepass(q, k, v, bf16, sq, skv, skv, seqs, n_seqs, Hq, Hkv, D, gran, pv, smooth_k, 0, ws, L, s)) !=
+      SAGE_OK)
     return st;
-  if ((st = run_quant_v(v, bf16, skv, seqs, n_seqs, Hkv, D, pv, ws, L, s)) != SAGE_OK) return st;
   return run_attn(out, bf16, sq, seqs, n_seqs, Hq, Hkv, D, is_causal, sm_scale, gran, pv, pv_accum, ws, L, s);
 }
 

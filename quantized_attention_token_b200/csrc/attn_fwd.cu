@@ -82,32 +82,38 @@ __device__ __forceinline__ constexpr int kgrp(int col) {
 //   unscaled scores -> m_tile = max_g c_g * max_g(S) -> alpha -> exponent
 //   argument S*c - m (one packed FFMA), ex2, row sum -> P~ rounded to E4M3
 //   (448 folded into the exponent) or 16 bits, written over the S columns.
-// c[g] = dQ * dK_g * sm_scale * log2(e), positive or zero.
-template <bool PV8, bool KPT>
+// c[g] = dQ * dK_g * sm_scale * log2(e), kept >= 1e-30 so that a masked
+// score (-inf) always yields P~ = 0 (a group whose scale is 0 has S = 0 and
+// s = S * 1e-30 rounds every P~ exactly as s = 0 does).
+template <bool PV8, bool KPT, bool BF16P>
 __device__ __forceinline__ void softmax_tile(uint32_t taddr, const float (&c)[16], bool masked, int col0, int lim,
-                                             bool bf16p, float& m, float& l, float& alpha) {
+                                             float& m, float& l, float& alpha) {
   uint32_t r[128];
   tmem_ld128_sync(taddr, r);
-  float f[128];
 #pragma unroll
-  for (int k = 0; k < 64; ++k)
-    add2(f[2 * k], f[2 * k + 1], __uint_as_float(r[2 * k] + 0x4B400000u), __uint_as_float(r[2 * k + 1] + 0x4B400000u),
+  for (int k = 0; k < 64; ++k) {
+    float x0, x1;
+    add2(x0, x1, __uint_as_float(r[2 * k] + 0x4B400000u), __uint_as_float(r[2 * k + 1] + 0x4B400000u),
          -12582912.0f, -12582912.0f);
+    r[2 * k] = __float_as_uint(x0);
+    r[2 * k + 1] = __float_as_uint(x1);
+  }
   if (masked) {
 #pragma unroll
     for (int i = 0; i < 128; ++i)
-      if (!(col0 + i < lim)) f[i] = -INFINITY;
+      if (!(col0 + i < lim)) r[i] = 0xFF800000u;   // -inf
   }
-  // maxima of the unscaled scores per scale group (c >= 0 keeps the order)
+  auto F = [&](int i) { return __uint_as_float(r[i]); };
+  // maxima of the unscaled scores per scale group (c > 0 keeps the order)
   float mt = -INFINITY;
   if (KPT) {
 #pragma unroll
     for (int g = 0; g < 16; ++g) {
       const int base = (g >> 3) * 64 + (g & 7);
-      float a = max3(f[base], f[base + 8], f[base + 16]);
-      float b = max3(f[base + 24], f[base + 32], f[base + 40]);
-      a = max3(a, b, fmaxf(f[base + 48], f[base + 56]));
-      if (a != -INFINITY) mt = fmaxf(mt, c[g] * a);
+      float a = max3(F(base), F(base + 8), F(base + 16));
+      float bb = max3(F(base + 24), F(base + 32), F(base + 40));
+      a = max3(a, bb, fmaxf(F(base + 48), F(base + 56)));
+      mt = fmaxf(mt, c[g] * a);
     }
   } else {
 #pragma unroll
@@ -115,49 +121,39 @@ __device__ __forceinline__ void softmax_tile(uint32_t taddr, const float (&c)[16
       float a0 = -INFINITY, a1 = -INFINITY, a2 = -INFINITY, a3 = -INFINITY;
 #pragma unroll
       for (int i = 0; i < 64; i += 8) {
-        a0 = max3(a0, f[64 * g + i], f[64 * g + i + 1]);
-        a1 = max3(a1, f[64 * g + i + 2], f[64 * g + i + 3]);
-        a2 = max3(a2, f[64 * g + i + 4], f[64 * g + i + 5]);
-        a3 = max3(a3, f[64 * g + i + 6], f[64 * g + i + 7]);
+        a0 = max3(a0, F(64 * g + i), F(64 * g + i + 1));
+        a1 = max3(a1, F(64 * g + i + 2), F(64 * g + i + 3));
+        a2 = max3(a2, F(64 * g + i + 4), F(64 * g + i + 5));
+        a3 = max3(a3, F(64 * g + i + 6), F(64 * g + i + 7));
       }
-      const float a = max3(a0, a1, fmaxf(a2, a3));
-      if (a != -INFINITY) mt = fmaxf(mt, c[g] * a);
+      mt = fmaxf(mt, c[g] * max3(a0, a1, fmaxf(a2, a3)));
     }
   }
   const float m_new = fmaxf(m, mt);
   alpha = (m == -INFINITY) ? 0.f : ex2(m - m_new);
   const float nb = -(PV8 ? (m_new - kLog2Fp8Max) : m_new);
-  float ls0 = 0.f, ls1 = 0.f;
+  float ls0 = 0.f, ls1 = 0.f, h0 = 0.f, h1 = 0.f;
+  uint32_t w[PV8 ? 32 : 64];
 #pragma unroll
   for (int k = 0; k < 64; ++k) {
     float a0, a1;
-    fma2(a0, a1, f[2 * k], f[2 * k + 1], c[kgrp<KPT>(2 * k)], c[kgrp<KPT>(2 * k + 1)], nb, nb);
-    float p0 = ex2(a0), p1 = ex2(a1);
-    if (masked) {
-      if (!(col0 + 2 * k < lim)) p0 = 0.f;
-      if (!(col0 + 2 * k + 1 < lim)) p1 = 0.f;
-    }
-    f[2 * k] = p0;
-    f[2 * k + 1] = p1;
+    fma2(a0, a1, F(2 * k), F(2 * k + 1), c[kgrp<KPT>(2 * k)], c[kgrp<KPT>(2 * k + 1)], nb, nb);
+    const float p0 = ex2(a0), p1 = ex2(a1);
     add2(ls0, ls1, ls0, ls1, p0, p1);
+    if (PV8) {
+      if (k & 1) w[k >> 1] = pack_e4m3x4(h0, h1, p0, p1);
+      else { h0 = p0; h1 = p1; }
+    } else {
+      w[k] = BF16P ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
+    }
   }
   l = alpha * l + (ls0 + ls1);
   m = m_new;
   if (PV8) {
-    uint32_t w[32];
-#pragma unroll
-    for (int k = 0; k < 32; ++k) w[k] = pack_e4m3x4(f[4 * k], f[4 * k + 1], f[4 * k + 2], f[4 * k + 3]);
-    tmem_st32(taddr, w);
+    tmem_st32(taddr, reinterpret_cast<const uint32_t(&)[32]>(w[0]));
   } else {
-    uint32_t w[32];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-#pragma unroll
-      for (int k = 0; k < 32; ++k)
-        w[k] = bf16p ? pack_bf16x2(f[64 * h + 2 * k], f[64 * h + 2 * k + 1])
-                     : pack_f16x2(f[64 * h + 2 * k], f[64 * h + 2 * k + 1]);
-      tmem_st32(taddr + 32 * h, w);
-    }
+    tmem_st32(taddr, reinterpret_cast<const uint32_t(&)[32]>(w[0]));
+    tmem_st32(taddr + 32, reinterpret_cast<const uint32_t(&)[32]>(w[PV8 ? 0 : 32]));
   }
 }
 
@@ -197,6 +193,115 @@ __device__ __forceinline__ void store_row(uint16_t* orow, uint32_t ob, const flo
       for (int k = 0; k < 4; ++k) dst[k] = make_uint4(w[4 * k], w[4 * k + 1], w[4 * k + 2], w[4 * k + 3]);
     }
   }
+}
+
+// One softmax warpgroup: the online softmax of query tile q over its KV
+// tiles; in one-level mode also the O rescale and the epilogue.
+template <int D, bool PV8, bool ACC2, bool KPT, bool BF16P>
+__device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, uint32_t tmem, int warp, int tid,
+                                             int pair, int b, int h, int hk, int qs, int Lq, int Lk, int tq0,
+                                             int tk0, const int* n, const float* vsc) {
+  using C = AttnCfg<D, PV8, ACC2>;
+  constexpr int NQ = C::NQ, NSB = C::NSB;
+  auto bar = [&](int i) -> uint32_t { return sb + C::OFF_BAR + 8 * i; };
+  uint8_t* smem = reinterpret_cast<uint8_t*>(__cvta_shared_to_generic(sb));
+  uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
+  float* alpha_s = reinterpret_cast<float*>(smem + C::OFF_ALPHA);
+  float* l_s = reinterpret_cast<float*>(smem + C::OFF_L);
+    const int q = (warp - 4) >> 2;
+    const int t = tid - 128 * (1 + q);
+    const int qt = pair * NQ + q;
+    const uint32_t lane_off = (uint32_t)((t & ~31)) << 16;
+    const int row = qt * kTile + t;
+    const bool bf16 = BF16P || (PV8 && p.out_bf16 != 0);
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    if (n[q] > 0) {
+      const float qsc = p.q_scale[((size_t)h * p.tiles_q + tq0 + qt) * kQGroupsMax + q_group(p.gran, t)];
+      const float* ksb = p.k_scale + ((size_t)hk * p.tiles_k + tk0) * kKGroupsMax;
+      const uint32_t ob = tmem + C::TM_O + q * D + lane_off;
+      // K group scales of the next tile are fetched one tile ahead
+      float ksn[KPT ? 16 : 2];
+#pragma unroll
+      for (int g = 0; g < (KPT ? 16 : 2); ++g) ksn[g] = __ldg(ksb + g);
+      for (int j = 0; j < n[q]; ++j) {
+        const int buf = j % NSB;
+        float c[16];
+#pragma unroll
+        for (int g = 0; g < 16; ++g) c[g] = g < (KPT ? 16 : 2) ? fmaxf((qsc * ksn[g]) * p.sl2, 1e-30f) : 1e-30f;
+        if (j + 1 < n[q]) {
+#pragma unroll
+          for (int g = 0; g < (KPT ? 16 : 2); ++g) ksn[g] = __ldg(ksb + (j + 1) * kKGroupsMax + g);
+        }
+        if (!(ok = mbar_wait(bar(C::B_SFULL + q * NSB + buf), (j / NSB) & 1, abort_flag, p.err, kErrTimeoutSoftmax)))
+          break;
+        tc_fence_after();
+        // keys past the sequence, or (causal) past this row, are masked
+        const int col0 = j * kTile;
+        const bool masked = (col0 + kTile > Lk) || (p.causal && j == qt);
+        const int lim = p.causal ? min(Lk, row + 1) : Lk;
+        const uint32_t taddr = tmem + C::TM_S + (q * NSB + buf) * 128 + lane_off;
+        float alpha;
+        softmax_tile<PV8, KPT, BF16P>(taddr, c, masked, col0, lim, m, l, alpha);
+        if (ACC2) {
+          const int ab = j & 1;
+          if (!(ok = mbar_wait(bar(C::B_AEMPTY + 2 * q + ab), ((j >> 1) & 1) ^ 1, abort_flag, p.err,
+                               kErrTimeoutSoftmax)))
+            break;
+          alpha_s[(q * 2 + ab) * 128 + t] = alpha;
+          mbar_arrive(bar(C::B_AFULL + 2 * q + ab));
+        } else if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          // O(q) holds the sums of tiles < j (PV_{j-1} finished before S_j did)
+          if (D == 128) {
+            uint32_t r[128];
+            tmem_ld128_sync(ob, r);
+#pragma unroll
+            for (int u = 0; u < 128; u += 2) {
+              float x0, x1;
+              mul2(x0, x1, __uint_as_float(r[u]), __uint_as_float(r[u + 1]), alpha, alpha);
+              r[u] = __float_as_uint(x0);
+              r[u + 1] = __float_as_uint(x1);
+            }
+            tmem_st128(ob, r);
+          } else {
+#pragma unroll
+            for (int ch = 0; ch < D / 32; ++ch) {
+              uint32_t r[32];
+              tmem_ld32(ob + ch * 32, r);
+              tmem_wait_ld(r);
+#pragma unroll
+              for (int u = 0; u < 32; u += 2) {
+                float x0, x1;
+                mul2(x0, x1, __uint_as_float(r[u]), __uint_as_float(r[u + 1]), alpha, alpha);
+                r[u] = __float_as_uint(x0);
+                r[u + 1] = __float_as_uint(x1);
+              }
+              tmem_st32(ob + ch * 32, r);
+            }
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(C::B_PFULL + q));
+      }
+    }
+    if (ACC2) {
+      l_s[q * 128 + t] = l;
+      mbar_arrive(bar(C::B_LFULL + q));
+    } else if (ok && qt * kTile < Lq) {
+      // epilogue of this query tile
+      if (n[q] > 0) {
+        ok = mbar_wait(bar(C::B_OFULL + q), 0, abort_flag, p.err, kErrTimeoutSoftmax);
+        tc_fence_after();
+      }
+      if (ok) {
+        uint16_t* orow = reinterpret_cast<uint16_t*>(p.out) + (long long)b * p.os.sb + (long long)h * p.os.sh +
+                         (long long)(qs + row) * p.os.ss;
+        store_row<D, PV8, false>(orow, tmem + C::TM_O + q * D + lane_off, nullptr, l > 0.f ? 1.0f / l : 0.f, vsc,
+                                 bf16, n[q] > 0, row < Lq);
+      }
+    }
 }
 
 // ---------------------------------------------------------------- kernel
@@ -381,79 +486,13 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
     }
   } else if (warp >= 4 && warp < 4 + 4 * NQ) {
     // ------------------------------------------------------------ softmax
-    const int q = (warp - 4) >> 2;
-    const int t = tid - 128 * (1 + q);
-    const int qt = pair * NQ + q;
-    const uint32_t lane_off = (uint32_t)((t & ~31)) << 16;
-    const int row = qt * kTile + t;
-    const bool bf16 = p.out_bf16 != 0;
-    float m = -INFINITY, l = 0.f;
-    bool ok = true;
-    if (n[q] > 0) {
-      const float qsc = p.q_scale[((size_t)h * p.tiles_q + tq0 + qt) * kQGroupsMax + q_group(p.gran, t)];
-      const float* ksb = p.k_scale + ((size_t)hk * p.tiles_k + tk0) * kKGroupsMax;
-      const bool kpt = p.gran == 2;
-      const uint32_t ob = tmem + C::TM_O + q * D + lane_off;
-      for (int j = 0; j < n[q]; ++j) {
-        const int buf = j % NSB;
-        if (!(ok = mbar_wait(bar(C::B_SFULL + q * NSB + buf), (j / NSB) & 1, abort_flag, p.err, kErrTimeoutSoftmax)))
-          break;
-        tc_fence_after();
-        float c[16];
-#pragma unroll
-        for (int g = 0; g < 16; ++g) c[g] = (kpt || g < 2) ? (qsc * __ldg(ksb + j * kKGroupsMax + g)) * p.sl2 : 0.f;
-        // keys past the sequence, or (causal) past this row, are masked
-        const int col0 = j * kTile;
-        const bool masked = (col0 + kTile > Lk) || (p.causal && j == qt);
-        const int lim = p.causal ? min(Lk, row + 1) : Lk;
-        const uint32_t taddr = tmem + C::TM_S + (q * NSB + buf) * 128 + lane_off;
-        float alpha;
-        if (kpt) softmax_tile<PV8, true>(taddr, c, masked, col0, lim, bf16, m, l, alpha);
-        else softmax_tile<PV8, false>(taddr, c, masked, col0, lim, bf16, m, l, alpha);
-        if (ACC2) {
-          const int ab = j & 1;
-          if (!(ok = mbar_wait(bar(C::B_AEMPTY + 2 * q + ab), ((j >> 1) & 1) ^ 1, abort_flag, p.err,
-                               kErrTimeoutSoftmax)))
-            break;
-          alpha_s[(q * 2 + ab) * 128 + t] = alpha;
-          mbar_arrive(bar(C::B_AFULL + 2 * q + ab));
-        } else if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-          // O(q) holds the sums of tiles < j (PV_{j-1} finished before S_j did)
-#pragma unroll
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t r[32];
-            tmem_ld32(ob + ch * 32, r);
-            tmem_wait_ld(r);
-#pragma unroll
-            for (int u = 0; u < 32; u += 2) {
-              float x0, x1;
-              mul2(x0, x1, __uint_as_float(r[u]), __uint_as_float(r[u + 1]), alpha, alpha);
-              r[u] = __float_as_uint(x0);
-              r[u + 1] = __float_as_uint(x1);
-            }
-            tmem_st32(ob + ch * 32, r);
-          }
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(C::B_PFULL + q));
-      }
-    }
-    if (ACC2) {
-      l_s[q * 128 + t] = l;
-      mbar_arrive(bar(C::B_LFULL + q));
-    } else if (ok && qt * kTile < Lq) {
-      // epilogue of this query tile
-      if (n[q] > 0) {
-        ok = mbar_wait(bar(C::B_OFULL + q), 0, abort_flag, p.err, kErrTimeoutSoftmax);
-        tc_fence_after();
-      }
-      if (ok) {
-        uint16_t* orow = reinterpret_cast<uint16_t*>(p.out) + (long long)b * p.os.sb + (long long)h * p.os.sh +
-                         (long long)(qs + row) * p.os.ss;
-        store_row<D, PV8, false>(orow, tmem + C::TM_O + q * D + lane_off, nullptr, l > 0.f ? 1.0f / l : 0.f, vsc,
-                                 bf16, n[q] > 0, row < Lq);
-      }
+    const bool bf16p = !PV8 && p.out_bf16;
+    if (p.gran == 2) {
+      if (bf16p) softmax_role<D, PV8, ACC2, true, true>(p, sb, tmem, warp, tid, pair, b, h, hk, qs, Lq, Lk, tq0, tk0, n, vsc);
+      else softmax_role<D, PV8, ACC2, true, false>(p, sb, tmem, warp, tid, pair, b, h, hk, qs, Lq, Lk, tq0, tk0, n, vsc);
+    } else {
+      if (bf16p) softmax_role<D, PV8, ACC2, false, true>(p, sb, tmem, warp, tid, pair, b, h, hk, qs, Lq, Lk, tq0, tk0, n, vsc);
+      else softmax_role<D, PV8, ACC2, false, false>(p, sb, tmem, warp, tid, pair, b, h, hk, qs, Lq, Lk, tq0, tk0, n, vsc);
     }
   } else if (ACC2 && warp >= 4 + 4 * NQ) {
     // ------------------------------------------------------------ correction (two-level) + epilogue

@@ -6,24 +6,32 @@
 
 namespace sage {
 
-struct PrepassParams {
-  const uint16_t* x;          // input tensor (fp16 / bf16 bits)
-  Strides st;
+// One launch of the persistent pre-pass: which tensors to quantize, where
+// they are, and the workspace regions it fills.
+struct PrepassJob {
+  const uint16_t* q = nullptr;
+  const uint16_t* k = nullptr;
+  const uint16_t* v = nullptr;
+  Strides sq{}, sk{}, sv{};
   Seqs seqs;
-  int H;                      // heads of this tensor
-  int bf16;
-  int gran;
-  int smooth;                 // K: subtract channel mean; Q: subtract block mean
-  int tiles;                  // workspace tiles per head
-  uint32_t* err;
-  unsigned long long* k_stat; // [nseq][H][D] int64 (fp16) / fp64 bits (bf16) channel sums
-  uint32_t* v_stat;           // [nseq][H][D] float bits of channel |max|
-  float* k_mean;              // [nseq][H][D]
-  float* v_scale;             // [nseq][H][D]
-  int8_t* codes;              // Q or K tiles
-  float* scales;              // [H][tiles][32 or 16]
-  uint8_t* v_codes;           // V tiles
-  float* q_mean;              // [H][tiles][D] (smooth Q)
+  int nseq = 0, Hq = 0, Hkv = 0, group = 1;
+  int bf16 = 0, gran = 0, smooth_k = 0, smooth_q = 0, pv8 = 1;
+  int do_q = 0, do_k = 0, do_v = 0;
+  int tiles_q = 0, tiles_k = 0;    // workspace tiles per head
+  uint32_t* err = nullptr;
+  unsigned long long* k_stat = nullptr;   // [nseq][Hkv][D] int64 (fp16) / fp64 bits (bf16) channel sums
+  uint32_t* v_stat = nullptr;             // [nseq][Hkv][D] float bits of channel |max|
+  float* k_mean = nullptr;                // [nseq][Hkv][D]
+  float* v_scale = nullptr;               // [nseq][Hkv][D]
+  int8_t* q_codes = nullptr;
+  float* q_scale = nullptr;               // [Hq][tiles_q][32]
+  int8_t* k_codes = nullptr;
+  float* k_scale = nullptr;               // [Hkv][tiles_k][16]
+  uint8_t* v_codes = nullptr;
+  float* q_mean = nullptr;                // [Hq][tiles_q][D] (smooth Q)
+  uint32_t* ticket = nullptr;             // work-item counter, zero at launch
+  uint32_t* stats_done = nullptr;         // [nseq][Hkv] finished statistics items, zero at launch
+  int* item_off = nullptr;                // varlen: first work item of each sequence [nseq+1]
 };
 
 struct AttnParams {
@@ -46,11 +54,10 @@ struct AttnParams {
 };
 
 // prepass.cu
-cudaError_t prepass_qk(const PrepassParams& pq, const PrepassParams& pk, int D, int nseq, int tps_q,
-                       int tps_k, cudaStream_t s);
-cudaError_t prepass_v(const PrepassParams& pv, int D, bool pv8, int nseq, int tps, cudaStream_t s);
-cudaError_t prepass_varlen_offsets(const int* cu_q, const int* cu_k, int n, int max_seqlen, int cap_q,
-                                   int cap_k, int* toff_q, int* toff_k, uint32_t* err, cudaStream_t s);
+cudaError_t prepass_run(const PrepassJob& j, int D, cudaStream_t s);
+cudaError_t prepass_varlen_offsets(const int* cu_q, const int* cu_k, int n, int max_seqlen, int cap_q, int cap_k,
+                                   int* toff_q, int* toff_k, uint32_t* err, const PrepassJob& job,
+                                   cudaStream_t s);
 
 // attn_fwd.cu
 int attn_tiles_per_cta(int D, bool pv8, bool acc2);

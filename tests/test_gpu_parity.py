@@ -201,3 +201,32 @@ def test_repeated_calls_are_deterministic():
     b = sage.sageattn(q, k, v)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("pv", ["fp8", "fp16"])
+def test_one_level_accumulation_as_accurate_as_two_level(pv):
+    """The two accumulation modes see the same P~ and V codes; they differ in
+    where each tile's partial sums are added: inside the tensor core's
+    accumulator (fp32) or into a separate FP32 register buffer (fp32+fp32).
+    The oracle adds the same products in fp64.  Over 256 key tiles, an inner
+    accumulator narrower than FP32 (the "FP22" of the pages' Hopper kernels,
+    SageAttention2 summary) would make the one-level mode measurably worse;
+    on B200 both must be equally close to the oracle."""
+    S = 32768
+    sp = synth.Spec("t", Hq=2, Hkv=2, D=128, B=1, S=S, k_bias_std=4.0, seed=61)
+    q, k, v = synth.make(sp)
+    qd, kd, vd = (t.cuda() for t in (q, k, v))
+    a = sage.sageattn(qd, kd, vd, "HND", False, pv_dtype=pv, pv_accum_dtype="fp32").double().cpu().numpy()
+    b = sage.sageattn(qd, kd, vd, "HND", False, pv_dtype=pv, pv_accum_dtype="fp32+fp32").double().cpu().numpy()
+    torch.cuda.synchronize()
+    errs = {"fp32": [], "fp32+fp32": []}
+    for h in range(2):
+        for r0 in (0, S - 128):
+            ref = oracle.attention(q[:, h:h + 1], k[:, h:h + 1], v[:, h:h + 1], pv=pv,
+                                   q_rows={(0, 0): (r0, r0 + 128)})[0, 0, r0:r0 + 128]
+            errs["fp32"].append(np.abs(a[0, h, r0:r0 + 128] - ref))
+            errs["fp32+fp32"].append(np.abs(b[0, h, r0:r0 + 128] - ref))
+    e1 = float(np.mean(np.concatenate(errs["fp32"])))
+    e2 = float(np.mean(np.concatenate(errs["fp32+fp32"])))
+    print(f"mean |gpu - oracle|: fp32 {e1:.3e}, fp32+fp32 {e2:.3e}")
+    assert e1 <= 1.1 * e2 + 1e-7, (e1, e2)
