@@ -144,6 +144,23 @@ def recorded_traffic(workload: str):
     return e.get("dram_bytes_per_launch")
 
 
+def max_over_ranks(x: float, device) -> float:
+    """The maximum of x over the ranks of the default process group (x itself
+    without one): a multi-GPU time is the slowest rank's."""
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return x
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tops(world: int, ops_per_step: float, steps: int, elapsed_ms: float) -> float:
+    """Whole-job TOPS: each of `world` ranks ran `steps` steps of
+    `ops_per_step` ops in `elapsed_ms` (the slowest rank's time)."""
+    return world * ops_per_step * steps / (elapsed_ms * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------------------- CPU oracle
 def cpu_baseline(spec: synth.Spec, q, k, v, pv: str, budget_s: float):
     """The oracle as it stands, on a bounded sample of the workload: whole
@@ -260,16 +277,13 @@ def main():
     elapsed_ms = start.elapsed_time(stop)
     attn_ms = [e[1].elapsed_time(e[2]) for e in evs]
     pre_ms = [e[0].elapsed_time(e[1]) for e in evs]
-    if world > 1:
-        t = torch.tensor([elapsed_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        elapsed_ms = float(t.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dev)
     st, bits = sage.get_device_error(ws)
     if st != 0:
         raise RuntimeError(f"device error word {bits:#x} after the timed region")
 
     ms_per_step = elapsed_ms / args.steps
-    value = world * ops * args.steps / (elapsed_ms * 1e-3) / 1e12
+    value = job_tops(world, ops, args.steps, elapsed_ms)
 
     # end to end through the public API with host buffers: pinned H2D of q,k,v,
     # the forward pass, D2H of the output, every step
@@ -293,11 +307,7 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dev)
 
     if world > 1:
         import torch.distributed as dist
@@ -330,10 +340,10 @@ def main():
         "prepass": {"ms": pre_avg, "achieved_gbs": pre_bytes / (pre_avg * 1e-3) / 1e9,
                     "peak_gbs": float(pk.get("hbm_gbs", 0)),
                     "frac": pre_bytes / (pre_avg * 1e-3) / 1e9 / float(pk.get("hbm_gbs", 1))},
-        "e2e": {"value": ops * world / (e2e_ms * 1e-3) / 1e12, "unit": "TOPS",
+        "e2e": {"value": job_tops(world, ops, 1, e2e_ms), "unit": "TOPS",
                 "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))),
                 "d2h_bytes_per_step": int(q_h.numel() * q_h.element_size())},
-        "gpu_launches": 2 * args.steps,     # the persistent pre-pass + the attention kernel
+        "gpu_launches": 3 * args.steps,     # pre-pass launches A and B + the attention kernel
         "clocks": clk.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:

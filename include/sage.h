@@ -122,7 +122,6 @@ typedef struct {
   size_t err;       /* uint32 device error word */
   size_t tile_off_q, tile_off_k;   /* int32 [n_seqs+1] (varlen) */
   size_t k_stat, v_stat;           /* pre-pass accumulators */
-  size_t sched;                    /* pre-pass work counters and varlen item offsets */
   size_t k_mean, v_scale;
   size_t q_codes, q_scale, k_codes, k_scale, v_codes;
   size_t q_mean, q_bias;

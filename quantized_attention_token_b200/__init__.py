@@ -40,7 +40,7 @@ class SageError(RuntimeError):
 
 class WsLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
-        "err", "tile_off_q", "tile_off_k", "k_stat", "v_stat", "sched", "k_mean", "v_scale", "q_codes",
+        "err", "tile_off_q", "tile_off_k", "k_stat", "v_stat", "k_mean", "v_scale", "q_codes",
         "q_scale", "k_codes", "k_scale", "v_codes", "q_mean", "q_bias", "total")] + [
         ("tiles_q", ctypes.c_int), ("tiles_k", ctypes.c_int)]
 
@@ -254,11 +254,13 @@ def quant_v(v, ws, tensor_layout="HND", pv_dtype="fp8"):
 
 
 def attn_quantized(out, ws, B, Hq, Hkv, S, D, tensor_layout="HND", is_causal=False, sm_scale=None,
-                   qk_quant_gran="per_block", pv_dtype="fp8", pv_accum_dtype="fp32+fp32"):
-    """The attention kernel alone on a workspace filled by quant_qk + quant_v."""
+                   qk_quant_gran="per_block", pv_dtype="fp8", pv_accum_dtype="fp32+fp32", smooth_q=False):
+    """The attention kernel alone on a workspace filled by quant_qk + quant_v
+    (smooth_q as given to quant_qk)."""
     st = lib().sage_attn_quantized(out.data_ptr(), _dtype_code(out), B, Hq, Hkv, S, D, LAYOUT[tensor_layout],
                                    int(is_causal), float(sm_scale or 0.0), GRAN[qk_quant_gran], PV[pv_dtype],
-                                   ACC[pv_accum_dtype], 0, ws.data_ptr(), ws.numel(), _stream(out.device))
+                                   ACC[pv_accum_dtype], int(smooth_q), ws.data_ptr(), ws.numel(),
+                                   _stream(out.device))
     _check("sage_attn_quantized", st)
 
 

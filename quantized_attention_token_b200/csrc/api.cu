@@ -60,11 +60,10 @@ sage_status_t plan(int nseq, int total_q, int total_k, int max_seqlen, int Hq, i
   L->err = take(256, 256);
   L->tile_off_q = take(varlen ? sizeof(int) * (nseq + 1) : 0, 256);
   L->tile_off_k = take(varlen ? sizeof(int) * (nseq + 1) : 0, 256);
-  // k_stat, v_stat and the pre-pass counters are contiguous: one memset
-  // zeroes them before each pre-pass launch
+  // k_stat and v_stat are contiguous: one memset zeroes them before each
+  // pre-pass
   L->k_stat = take(nd * 8, 256);
   L->v_stat = take(nd * 4, 4);
-  L->sched = take(4 * (1 + (size_t)nseq * Hkv) + 4 * (size_t)(nseq + 1), 4);
   L->k_mean = take(nd * 4, 256);
   L->v_scale = take(nd * 4, 256);
   L->k_codes = take((size_t)Hkv * tk * kTile * D, 1024);
@@ -99,16 +98,16 @@ sage_status_t check_common(sage_dtype_t dtype, int D, sage_gran_t gran, sage_pv_
   return SAGE_OK;
 }
 
-// Bytes from k_stat to the end of the pre-pass counters (zeroed per launch).
-size_t stats_zero_bytes(const sage_ws_layout_t& L, int nseq, int Hkv) {
-  return L.sched + 4 * (1 + (size_t)nseq * Hkv) - L.k_stat;
+// Bytes of the pre-pass accumulators k_stat .. v_stat (zeroed per pre-pass).
+size_t stats_zero_bytes(const sage_ws_layout_t& L, int nseq, int Hkv, int D) {
+  return L.v_stat + 4 * (size_t)nseq * Hkv * D - L.k_stat;
 }
 
-// The persistent pre-pass over any of Q, K, V (dense or varlen).
+// The pre-pass over any of Q, K, V (dense or varlen).
 sage_status_t run_prepass(const void* q, const void* k, const void* v, int bf16, Strides sq, Strides sk,
                           Strides sv, const Seqs& seqs, int nseq, int Hq, int Hkv, int D, int gran, int pv,
                           int smooth_k, int smooth_q, void* ws, const sage_ws_layout_t& L, cudaStream_t s) {
-  if (cudaMemsetAsync(at<char>(ws, L.k_stat), 0, stats_zero_bytes(L, nseq, Hkv), s) != cudaSuccess)
+  if (cudaMemsetAsync(at<char>(ws, L.k_stat), 0, stats_zero_bytes(L, nseq, Hkv, D), s) != cudaSuccess)
     return SAGE_ERR_CUDA;
   PrepassJob j;
   j.q = static_cast<const uint16_t*>(q);
@@ -143,18 +142,16 @@ sage_status_t run_prepass(const void* q, const void* k, const void* v, int bf16,
   j.k_scale = at<float>(ws, L.k_scale);
   j.v_codes = at<uint8_t>(ws, L.v_codes);
   j.q_mean = smooth_q ? at<float>(ws, L.q_mean) : nullptr;
-  j.ticket = at<uint32_t>(ws, L.sched);
-  j.stats_done = j.ticket + 1;
-  j.item_off = reinterpret_cast<int*>(j.stats_done + (size_t)nseq * Hkv);
+  j.q_bias = smooth_q ? at<float>(ws, L.q_bias) : nullptr;
   if (seqs.cu_k &&
       prepass_varlen_offsets(seqs.cu_q, seqs.cu_k, nseq, seqs.max_seqlen, L.tiles_q, L.tiles_k,
-                             const_cast<int*>(seqs.toff_q), const_cast<int*>(seqs.toff_k), j.err, j, s) != cudaSuccess)
+                             const_cast<int*>(seqs.toff_q), const_cast<int*>(seqs.toff_k), j.err, s) != cudaSuccess)
     return SAGE_ERR_CUDA;
   return cuda_status(prepass_run(j, D, s));
 }
 
 sage_status_t run_attn(void* out, int bf16, Strides so, const Seqs& seqs, int nseq, int Hq, int Hkv, int D,
-                       int causal, float sm_scale, int gran, int pv, int acc, const void* ws,
+                       int causal, float sm_scale, int gran, int pv, int acc, int smooth_q, const void* ws,
                        const sage_ws_layout_t& L, cudaStream_t s) {
   void* w = const_cast<void*>(ws);
   AttnParams p{};
@@ -175,6 +172,8 @@ sage_status_t run_attn(void* out, int bf16, Strides so, const Seqs& seqs, int ns
   p.os = so;
   const float scale = sm_scale > 0.f ? sm_scale : 1.0f / sqrtf((float)D);
   p.sl2 = scale * kLog2e;
+  p.q_bias = smooth_q ? at<float>(w, L.q_bias) : nullptr;
+  p.bias_ld = seqs.tps * kTile;
   p.gran = gran;
   p.causal = causal ? 1 : 0;
   p.out_bf16 = bf16;
@@ -233,10 +232,9 @@ SAGE_EXPORT sage_status_t sage_quant_qk(const void* q, const void* k, sage_dtype
   if ((st = check_common(dtype, D, gran, SAGE_PV_FP8, SAGE_ACC_FP32)) != SAGE_OK) return st;
   if (!q || !k || !ws) return SAGE_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(ws, 256)) return SAGE_ERR_INVALID_ARG;
-  if (smooth_q) return SAGE_ERR_UNSUPPORTED;
   sage_ws_layout_t L;
   if ((st = plan(B, B * S, B * S, S, Hq, Hkv, D, SAGE_PV_FP8, smooth_q, 0, &L)) != SAGE_OK) return st;
-  if (ws_bytes < L.q_scale + (size_t)Hq * L.tiles_q * kQGroupsMax * 4) return SAGE_ERR_WORKSPACE;
+  if (ws_bytes < (smooth_q ? L.total : L.q_scale + (size_t)Hq * L.tiles_q * kQGroupsMax * 4)) return SAGE_ERR_WORKSPACE;
   if ((st = check_device()) != SAGE_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return run_prepass(q, k, nullptr, dtype == SAGE_BF16, dense_strides(layout, Hq, S, D),
@@ -268,7 +266,6 @@ SAGE_EXPORT sage_status_t sage_quant_qkv(const void* q, const void* k, const voi
   if ((st = check_common(dtype, D, gran, pv, SAGE_ACC_FP32)) != SAGE_OK) return st;
   if (!q || !k || !v || !ws) return SAGE_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(ws, 256)) return SAGE_ERR_INVALID_ARG;
-  if (smooth_q) return SAGE_ERR_UNSUPPORTED;
   sage_ws_layout_t L;
   if ((st = plan(B, B * S, B * S, S, Hq, Hkv, D, pv, smooth_q, 0, &L)) != SAGE_OK) return st;
   if (ws_bytes < L.total) return SAGE_ERR_WORKSPACE;
@@ -287,13 +284,12 @@ SAGE_EXPORT sage_status_t sage_attn_quantized(void* out, sage_dtype_t dtype, int
   if ((st = check_common(dtype, D, gran, pv, pv_accum)) != SAGE_OK) return st;
   if (!out || !ws || !aligned(out, 16) || !aligned(ws, 256)) return SAGE_ERR_INVALID_ARG;
   if (!std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
-  if (smooth_q) return SAGE_ERR_UNSUPPORTED;
   sage_ws_layout_t L;
   if ((st = plan(B, B * S, B * S, S, Hq, Hkv, D, pv, smooth_q, 0, &L)) != SAGE_OK) return st;
   if (ws_bytes < L.total) return SAGE_ERR_WORKSPACE;
   if ((st = check_device()) != SAGE_OK) return st;
   return run_attn(out, dtype == SAGE_BF16, dense_strides(layout, Hq, S, D), dense_seqs(S), B, Hq, Hkv, D,
-                  is_causal, sm_scale, gran, pv, pv_accum, ws, L, static_cast<cudaStream_t>(stream));
+                  is_causal, sm_scale, gran, pv, pv_accum, smooth_q, ws, L, static_cast<cudaStream_t>(stream));
 }
 
 SAGE_EXPORT sage_status_t sage_attn_fwd(const void* q, const void* k, const void* v, void* out,
@@ -308,7 +304,6 @@ SAGE_EXPORT sage_status_t sage_attn_fwd(const void* q, const void* k, const void
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(out, 16) || !aligned(ws, 256))
     return SAGE_ERR_INVALID_ARG;
   if (!std::isfinite(sm_scale)) return SAGE_ERR_INVALID_ARG;
-  if (smooth_q) return SAGE_ERR_UNSUPPORTED;
   sage_ws_layout_t L;
   if ((st = plan(B, B * S, B * S, S, Hq, Hkv, D, pv, smooth_q, 0, &L)) != SAGE_OK) return st;
   if (ws_bytes < L.total) return SAGE_ERR_WORKSPACE;
@@ -321,7 +316,7 @@ SAGE_EXPORT sage_status_t sage_attn_fwd(const void* q, const void* k, const void
                         s)) != SAGE_OK)
     return st;
   return run_attn(out, bf16, dense_strides(layout, Hq, S, D), seqs, B, Hq, Hkv, D, is_causal, sm_scale, gran, pv,
-                  pv_accum, ws, L, s);
+                  pv_accum, smooth_q, ws, L, s);
 }
 
 SAGE_EXPORT sage_status_t sage_attn_varlen_fwd(const void* q, const void* k, const void* v, void* out,
@@ -356,7 +351,7 @@ SAGE_EXPORT sage_status_t sage_attn_varlen_fwd(const void* q, const void* k, con
   if ((st = run_prepass(q, k, v, bf16, sq, skv, skv, seqs, n_seqs, Hq, Hkv, D, gran, pv, smooth_k, 0, ws, L, s)) !=
       SAGE_OK)
     return st;
-  return run_attn(out, bf16, sq, seqs, n_seqs, Hq, Hkv, D, is_causal, sm_scale, gran, pv, pv_accum, ws, L, s);
+  return run_attn(out, bf16, sq, seqs, n_seqs, Hq, Hkv, D, is_causal, sm_scale, gran, pv, pv_accum, 0, ws, L, s);
 }
 
 SAGE_EXPORT sage_status_t sage_get_device_error(void* ws, void* stream, uint32_t* bits) {

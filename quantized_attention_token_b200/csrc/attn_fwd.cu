@@ -10,18 +10,21 @@
 // FP32 tensor-memory accumulator (fp32) or, per tile, into a separate FP32
 // register accumulator (fp32+fp32, the two-level scheme).
 //
-// B200 design.  One CTA owns NQ query tiles of 128 rows of one (sequence,
-// head) and runs four roles:
+// B200 design.  One CTA (384 threads) owns NQ query tiles of 128 rows of one
+// (sequence, head):
 //   warp 0        loader: one bulk copy per MMA-ready tile (the pre-pass wrote
 //                 tiles already in the swizzled operand layout), NST stages;
-//   warp 1        MMA issuer: tcgen05.mma kind::i8 (S, SMEM x SMEM -> TMEM s32)
-//                 and kind::f8f6f4 / kind::f16 (O, P~ from TMEM x V from SMEM);
+//   warp 1        MMA issuer: tcgen05.mma kind::i8 (S = Q K^T, SMEM x SMEM ->
+//                 TMEM s32) and kind::f8f6f4 / kind::f16 (O += P~ V, SMEM x
+//                 SMEM -> TMEM f32);
 //   warp 2        tensor-memory allocation;
-//   WG 1..NQ      softmax, one thread per query row (TMEM lane): integer row
-//                 max per scale group, one FFMA + ex2 per score, P~ packed and
-//                 written back into TMEM over the S it came from;
-//   last WG       correction: rescales O in TMEM (fp32) or adds the per-tile
-//                 partial O into FP32 registers (fp32+fp32); epilogue.
+//   WG 1..NQ      softmax, one thread per query row (TMEM lane).  It loads its
+//                 row of S and at once releases the S columns, so the next
+//                 tile's QK^T runs while it works; P~ goes to shared memory in
+//                 the swizzled K-major operand layout; in one-level mode it
+//                 also rescales O in TMEM and writes the epilogue;
+//   WG 2 (two-level mode, NQ = 1) correction: adds each tile's fresh FP32
+//                 partial O into an FP32 register accumulator; epilogue.
 // Every mbarrier wait is bounded (sage_common.cuh): a wait that never ends sets
 // the device error word and the CTA tears down instead of hanging.
 #include "sage_launch.cuh"
@@ -31,40 +34,44 @@ namespace sage {
 template <int D, bool PV8, bool ACC2>
 struct AttnCfg {
   static constexpr int NQ = ACC2 ? 1 : 2;          // query tiles per CTA
-  static constexpr int NSB = ACC2 ? 2 : 1;         // S buffers per query tile
-  static constexpr int NST = 3;                    // K/V pipeline stages
+  static constexpr int NST = PV8 ? 3 : 2;          // K/V pipeline stages
   static constexpr int NTHREADS = 384;             // 3 warpgroups (168 registers per thread)
   static constexpr int QT = kTile * D;             // bytes of a Q or K tile
   static constexpr int VT = D * kTile * (PV8 ? 1 : 2);
+  static constexpr int PT = kTile * kTile * (PV8 ? 1 : 2);   // P~ tile in shared memory
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NQ * QT;
   static constexpr int OFF_V = OFF_K + NST * QT;
-  static constexpr int OFF_ALPHA = OFF_V + NST * VT;          // float [NQ][2][128]   (two-level)
+  static constexpr int OFF_P = OFF_V + NST * VT;
+  static constexpr int OFF_ALPHA = OFF_P + NQ * PT;           // float [NQ][2][128]   (two-level)
   static constexpr int OFF_L = OFF_ALPHA + NQ * 2 * 128 * 4;  // float [NQ][128]      (two-level)
-  static constexpr int OFF_BAR = OFF_L + NQ * 128 * 4;
+  static constexpr int OFF_BIAS = OFF_L + NQ * 128 * 4;       // float [NST][NQ][128]  (smooth Q)
+  static constexpr int OFF_BAR = OFF_BIAS + NST * NQ * 128 * 4;
   enum {
     B_QFULL = 0,
     B_KFULL = B_QFULL + NQ,
     B_KEMPTY = B_KFULL + NST,
     B_VFULL = B_KEMPTY + NST,
     B_VEMPTY = B_VFULL + NST,
-    B_SFULL = B_VEMPTY + NST,
-    B_PFULL = B_SFULL + NQ * NSB,    // softmax -> MMA: P~ in TMEM (and O rescaled)
-    B_OFULL = B_PFULL + NQ,          // MMA -> consumer of O (every PV two-level, last PV one-level)
+    B_SFULL = B_VEMPTY + NST,        // MMA -> softmax: S_j in TMEM
+    B_SCONS = B_SFULL + NQ,          // softmax -> MMA: S_j read, its columns are free
+    B_PFULL = B_SCONS + NQ,          // softmax -> MMA: P~_j in shared memory (and O rescaled)
+    B_OFULL = B_PFULL + NQ,          // MMA -> softmax / correction: PV_j done
     B_OREADY = B_OFULL + NQ,         // correction -> MMA: partial O consumed (two-level)
     B_AFULL = B_OREADY + NQ,         // softmax -> correction: alpha (two-level)
     B_AEMPTY = B_AFULL + 2 * NQ,
     B_LFULL = B_AEMPTY + 2 * NQ,     // softmax -> correction: final row sum (two-level)
     B_DONE = B_LFULL + NQ,
-    NBAR = B_DONE + 1
+    B_GO = B_DONE + 1,               // softmax 0 -> softmax 1: start half a tile later
+    NBAR = B_GO + 1
   };
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // [0] tmem base, [1] abort flag
   static constexpr int SMEM_USED = OFF_MISC + 16;
   // At least 116 KB so that a single CTA holds an SM: the CTA allocates all
   // 512 TMEM columns, a second resident CTA would only wait for them.
   static constexpr int SMEM_BYTES = (SMEM_USED > 116 * 1024 ? SMEM_USED : 116 * 1024) + 1024;
-  static constexpr int TM_S = 0;                   // S[q][b] at (q*NSB + b) * 128
-  static constexpr int TM_O = NQ * NSB * 128;      // O[q] at TM_O + q * D
+  static constexpr int TM_S = 0;                   // S[q] at q * 128
+  static constexpr int TM_O = NQ * 128;            // O[q] at TM_O + q * D
   static constexpr uint32_t TM_COLS = 512;
   static_assert(TM_O + NQ * D <= 512, "TMEM budget");
   static_assert(SMEM_USED + 1024 <= 227 * 1024, "shared memory budget");
@@ -77,34 +84,19 @@ __device__ __forceinline__ constexpr int kgrp(int col) {
   return KPT ? ((col >> 6) << 3) + (col & 7) : (col >> 6);
 }
 
-// One 128-key tile of one query row (this thread's TMEM lane):
-//   S (int32, TMEM) -> exact float (magic-number add) -> group maxima of the
-//   unscaled scores -> m_tile = max_g c_g * max_g(S) -> alpha -> exponent
-//   argument S*c - m (one packed FFMA), ex2, row sum -> P~ rounded to E4M3
-//   (448 folded into the exponent) or 16 bits, written over the S columns.
-// c[g] = dQ * dK_g * sm_scale * log2(e), kept >= 1e-30 so that a masked
-// score (-inf) always yields P~ = 0 (a group whose scale is 0 has S = 0 and
-// s = S * 1e-30 rounds every P~ exactly as s = 0 does).
-template <bool PV8, bool KPT, bool BF16P>
-__device__ __forceinline__ void softmax_tile(uint32_t taddr, const float (&c)[16], bool masked, int col0, int lim,
-                                             float& m, float& l, float& alpha) {
-  uint32_t r[128];
-  tmem_ld128_sync(taddr, r);
-#pragma unroll
-  for (int k = 0; k < 64; ++k) {
-    float x0, x1;
-    add2(x0, x1, __uint_as_float(r[2 * k] + 0x4B400000u), __uint_as_float(r[2 * k + 1] + 0x4B400000u),
-         -12582912.0f, -12582912.0f);
-    r[2 * k] = __float_as_uint(x0);
-    r[2 * k + 1] = __float_as_uint(x1);
-  }
+// Phase 1 of a tile for one query row.  The S accumulator was seeded with
+// the bit pattern of 1.5 * 2^23 before the MMA added the int32 products, so
+// each column holds the float t = 1.5 * 2^23 + S exactly (|S| < 2^22).
+// Masked keys -> -inf; returns the tile maximum m_tile = max_g c_g *
+// max_g(S) (c > 0 keeps the order; t is monotonic in S).
+template <bool KPT>
+__device__ __forceinline__ float tile_max(uint32_t (&r)[128], const float (&c)[16], bool masked, int col0, int lim) {
   if (masked) {
 #pragma unroll
     for (int i = 0; i < 128; ++i)
       if (!(col0 + i < lim)) r[i] = 0xFF800000u;   // -inf
   }
   auto F = [&](int i) { return __uint_as_float(r[i]); };
-  // maxima of the unscaled scores per scale group (c > 0 keeps the order)
   float mt = -INFINITY;
   if (KPT) {
 #pragma unroll
@@ -113,7 +105,7 @@ __device__ __forceinline__ void softmax_tile(uint32_t taddr, const float (&c)[16
       float a = max3(F(base), F(base + 8), F(base + 16));
       float bb = max3(F(base + 24), F(base + 32), F(base + 40));
       a = max3(a, bb, fmaxf(F(base + 48), F(base + 56)));
-      mt = fmaxf(mt, c[g] * a);
+      mt = fmaxf(mt, c[g] * (a - 12582912.0f));
     }
   } else {
 #pragma unroll
@@ -126,35 +118,106 @@ __device__ __forceinline__ void softmax_tile(uint32_t taddr, const float (&c)[16
         a2 = max3(a2, F(64 * g + i + 4), F(64 * g + i + 5));
         a3 = max3(a3, F(64 * g + i + 6), F(64 * g + i + 7));
       }
-      mt = fmaxf(mt, c[g] * max3(a0, a1, fmaxf(a2, a3)));
+      mt = fmaxf(mt, c[g] * (max3(a0, a1, fmaxf(a2, a3)) - 12582912.0f));
     }
   }
-  const float m_new = fmaxf(m, mt);
-  alpha = (m == -INFINITY) ? 0.f : ex2(m - m_new);
-  const float nb = -(PV8 ? (m_new - kLog2Fp8Max) : m_new);
-  float ls0 = 0.f, ls1 = 0.f, h0 = 0.f, h1 = 0.f;
-  uint32_t w[PV8 ? 32 : 64];
+  return mt;
+}
+
+// Smooth-Q phase 1: the score of key j is s_j = S_j * c_g(j) + b_j * sl2,
+// b_j the tile's per-key correction (shared memory, the same for every row).
+// Each column of r is rewritten to s_j (float bits; masked keys -inf) and the
+// row maximum is returned.
+template <bool KPT>
+__device__ __forceinline__ float tile_max_bias(uint32_t (&r)[128], const float (&c)[16], const float* bias,
+                                               float sl2, bool masked, int col0, int lim) {
+  float m0 = -INFINITY, m1 = -INFINITY;
 #pragma unroll
-  for (int k = 0; k < 64; ++k) {
-    float a0, a1;
-    fma2(a0, a1, F(2 * k), F(2 * k + 1), c[kgrp<KPT>(2 * k)], c[kgrp<KPT>(2 * k + 1)], nb, nb);
-    const float p0 = ex2(a0), p1 = ex2(a1);
-    add2(ls0, ls1, ls0, ls1, p0, p1);
-    if (PV8) {
-      if (k & 1) w[k >> 1] = pack_e4m3x4(h0, h1, p0, p1);
-      else { h0 = p0; h1 = p1; }
-    } else {
-      w[k] = BF16P ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
+  for (int k0 = 0; k0 < 128; k0 += 4) {
+    const float4 bb = *reinterpret_cast<const float4*>(bias + k0);
+    float b0, b1, b2, b3, s0, s1, s2, s3;
+    mul2(b0, b1, bb.x, bb.y, sl2, sl2);
+    mul2(b2, b3, bb.z, bb.w, sl2, sl2);
+    add2(s0, s1, __uint_as_float(r[k0]), __uint_as_float(r[k0 + 1]), -12582912.0f, -12582912.0f);
+    add2(s2, s3, __uint_as_float(r[k0 + 2]), __uint_as_float(r[k0 + 3]), -12582912.0f, -12582912.0f);
+    fma2(s0, s1, s0, s1, c[kgrp<KPT>(k0)], c[kgrp<KPT>(k0 + 1)], b0, b1);
+    fma2(s2, s3, s2, s3, c[kgrp<KPT>(k0 + 2)], c[kgrp<KPT>(k0 + 3)], b2, b3);
+    if (masked) {
+      if (!(col0 + k0 < lim)) s0 = -INFINITY;
+      if (!(col0 + k0 + 1 < lim)) s1 = -INFINITY;
+      if (!(col0 + k0 + 2 < lim)) s2 = -INFINITY;
+      if (!(col0 + k0 + 3 < lim)) s3 = -INFINITY;
+    }
+    r[k0] = __float_as_uint(s0);
+    r[k0 + 1] = __float_as_uint(s1);
+    r[k0 + 2] = __float_as_uint(s2);
+    r[k0 + 3] = __float_as_uint(s3);
+    m0 = max3(m0, s0, s1);
+    m1 = max3(m1, s2, s3);
+  }
+  return fmaxf(m0, m1);
+}
+
+// Phase 2: P~ = 2^(S*c - m) (times 448 in FP8 mode: the static scale is
+// folded into the exponent), the row sum, and P~ rounded to E4M3 / 16 bits
+// and stored to row `row` of the shared-memory P~ tile (swizzled K-major,
+// 128-byte rows: FP8 one block of 128 keys, 16-bit two blocks of 64 keys).
+// Returns the row sum of this tile.
+
+
+template <bool PV8, bool KPT, bool BF16P, bool BIAS>
+__device__ __forceinline__ float tile_exp_store(const uint32_t (&r)[128], const float (&c)[16], float nb,
+                                                uint32_t p_smem, int row) {
+  auto F = [&](int i) { return __uint_as_float(r[i]); };
+  float ls[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};   // independent partial sums
+  const uint32_t rbase = p_smem + row * 128;
+  const int sw = row & 7;
+  if (PV8) {
+#pragma unroll
+    for (int ch = 0; ch < 8; ++ch) {          // 16 keys = one 16-byte chunk
+      uint32_t w[4];
+#pragma unroll
+      for (int q4 = 0; q4 < 4; ++q4) {
+        const int k0 = 16 * ch + 4 * q4;
+        float a0, a1, a2, a3;
+        if (BIAS) {                                   // r holds the scores
+          add2(a0, a1, F(k0), F(k0 + 1), nb, nb);
+          add2(a2, a3, F(k0 + 2), F(k0 + 3), nb, nb);
+        } else {
+          add2(a0, a1, F(k0), F(k0 + 1), -12582912.0f, -12582912.0f);        // exact S
+          add2(a2, a3, F(k0 + 2), F(k0 + 3), -12582912.0f, -12582912.0f);
+          fma2(a0, a1, a0, a1, c[kgrp<KPT>(k0)], c[kgrp<KPT>(k0 + 1)], nb, nb);
+          fma2(a2, a3, a2, a3, c[kgrp<KPT>(k0 + 2)], c[kgrp<KPT>(k0 + 3)], nb, nb);
+        }
+        const float p0 = ex2(a0), p1 = ex2(a1), p2 = ex2(a2), p3 = ex2(a3);
+        add2(ls[2 * (q4 & 1)], ls[2 * (q4 & 1) + 1], ls[2 * (q4 & 1)], ls[2 * (q4 & 1) + 1], p0, p1);
+        add2(ls[4 + 2 * (q4 & 1)], ls[5 + 2 * (q4 & 1)], ls[4 + 2 * (q4 & 1)], ls[5 + 2 * (q4 & 1)], p2, p3);
+        w[q4] = pack_e4m3x4(p0, p1, p2, p3);
+      }
+      st_shared_v4(rbase + ((ch ^ sw) << 4), w[0], w[1], w[2], w[3]);
+    }
+  } else {
+#pragma unroll
+    for (int ch = 0; ch < 16; ++ch) {         // 8 keys = one 16-byte chunk
+      uint32_t w[4];
+#pragma unroll
+      for (int q2 = 0; q2 < 4; ++q2) {
+        const int k0 = 8 * ch + 2 * q2;
+        float a0, a1;
+        if (BIAS) {
+          add2(a0, a1, F(k0), F(k0 + 1), nb, nb);
+        } else {
+          add2(a0, a1, F(k0), F(k0 + 1), -12582912.0f, -12582912.0f);        // exact S
+          fma2(a0, a1, a0, a1, c[kgrp<KPT>(k0)], c[kgrp<KPT>(k0 + 1)], nb, nb);
+        }
+        const float p0 = ex2(a0), p1 = ex2(a1);
+        add2(ls[2 * q2], ls[2 * q2 + 1], ls[2 * q2], ls[2 * q2 + 1], p0, p1);
+        w[q2] = BF16P ? pack_bf16x2(p0, p1) : pack_f16x2(p0, p1);
+      }
+      st_shared_v4(rbase + (ch >> 3) * (kTile * 128) + (((ch & 7) ^ sw) << 4), w[0], w[1], w[2], w[3]);
     }
   }
-  l = alpha * l + (ls0 + ls1);
-  m = m_new;
-  if (PV8) {
-    tmem_st32(taddr, reinterpret_cast<const uint32_t(&)[32]>(w[0]));
-  } else {
-    tmem_st32(taddr, reinterpret_cast<const uint32_t(&)[32]>(w[0]));
-    tmem_st32(taddr + 32, reinterpret_cast<const uint32_t(&)[32]>(w[PV8 ? 0 : 32]));
-  }
+  return ((ls[0] + ls[1]) + (ls[2] + ls[3])) + ((ls[4] + ls[5]) + (ls[6] + ls[7]));
 }
 
 // Row epilogue: out[c] = O[c] * inv_l (* delta_V[c] in FP8 mode, where l sums
@@ -197,123 +260,159 @@ __device__ __forceinline__ void store_row(uint16_t* orow, uint32_t ob, const flo
 
 // One softmax warpgroup: the online softmax of query tile q over its KV
 // tiles; in one-level mode also the O rescale and the epilogue.
-template <int D, bool PV8, bool ACC2, bool KPT, bool BF16P>
+template <int D, bool PV8, bool ACC2, bool KPT, bool BF16P, bool SMQ>
 __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, uint32_t tmem, int warp, int tid,
                                              int pair, int b, int h, int hk, int qs, int Lq, int Lk, int tq0,
                                              int tk0, const int* n, const float* vsc) {
   using C = AttnCfg<D, PV8, ACC2>;
-  constexpr int NQ = C::NQ, NSB = C::NSB;
+  constexpr int NQ = C::NQ;
   auto bar = [&](int i) -> uint32_t { return sb + C::OFF_BAR + 8 * i; };
   uint8_t* smem = reinterpret_cast<uint8_t*>(__cvta_shared_to_generic(sb));
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(misc + 1);
   float* alpha_s = reinterpret_cast<float*>(smem + C::OFF_ALPHA);
   float* l_s = reinterpret_cast<float*>(smem + C::OFF_L);
-    const int q = (warp - 4) >> 2;
-    const int t = tid - 128 * (1 + q);
-    const int qt = pair * NQ + q;
-    const uint32_t lane_off = (uint32_t)((t & ~31)) << 16;
-    const int row = qt * kTile + t;
-    const bool bf16 = BF16P || (PV8 && p.out_bf16 != 0);
-    float m = -INFINITY, l = 0.f;
-    bool ok = true;
-    if (n[q] > 0) {
-      const float qsc = p.q_scale[((size_t)h * p.tiles_q + tq0 + qt) * kQGroupsMax + q_group(p.gran, t)];
-      const float* ksb = p.k_scale + ((size_t)hk * p.tiles_k + tk0) * kKGroupsMax;
-      const uint32_t ob = tmem + C::TM_O + q * D + lane_off;
-      // K group scales of the next tile are fetched one tile ahead
-      float ksn[KPT ? 16 : 2];
+
+  const int q = (warp - 4) >> 2;
+  const int t = tid - 128 * (1 + q);
+  const int qt = pair * NQ + q;
+  const uint32_t lane_off = (uint32_t)((t & ~31)) << 16;
+  const int row = qt * kTile + t;
+  const bool bf16 = BF16P || (PV8 && p.out_bf16 != 0);
+  const uint32_t p_smem = sb + C::OFF_P + q * C::PT;
+  const uint32_t taddr = tmem + C::TM_S + q * 128 + lane_off;
+  const uint32_t ob = tmem + C::TM_O + q * D + lane_off;
+  float m = -INFINITY, l = 0.f;
+  bool ok = true;
+  int n_stop = n[q];
+  if (n[q] > 0) {
+    const float qsc = p.q_scale[((size_t)h * p.tiles_q + tq0 + qt) * kQGroupsMax + q_group(p.gran, t)];
+    const float* ksb = p.k_scale + ((size_t)hk * p.tiles_k + tk0) * kKGroupsMax;
+    // K group scales of the next tile are fetched one tile ahead
+    float ksn[KPT ? 16 : 2];
 #pragma unroll
-      for (int g = 0; g < (KPT ? 16 : 2); ++g) ksn[g] = __ldg(ksb + g);
-      for (int j = 0; j < n[q]; ++j) {
-        const int buf = j % NSB;
-        float c[16];
+    for (int g = 0; g < (KPT ? 16 : 2); ++g) ksn[g] = __ldg(ksb + g);
+    // seed the S columns for the first QK^T (see tile_max)
+    tmem_fill128(taddr, 0x4B400000u);
+    tmem_wait_st();
+    tc_fence_before();
+    mbar_arrive(bar(C::B_SCONS + q));
+    if (NQ == 2 && q == 1 && n[0] > 0) {
+      if (!(ok = mbar_wait(bar(C::B_GO), 0, abort_flag, p.err, kErrTimeoutSoftmax))) n_stop = 0;
+    }
+    for (int j = 0; j < n_stop; ++j) {
+      float c[16];
 #pragma unroll
-        for (int g = 0; g < 16; ++g) c[g] = g < (KPT ? 16 : 2) ? fmaxf((qsc * ksn[g]) * p.sl2, 1e-30f) : 1e-30f;
-        if (j + 1 < n[q]) {
+      for (int g = 0; g < 16; ++g) c[g] = g < (KPT ? 16 : 2) ? fmaxf((qsc * ksn[g]) * p.sl2, 1e-30f) : 1e-30f;
+      if (j + 1 < n[q]) {
 #pragma unroll
-          for (int g = 0; g < (KPT ? 16 : 2); ++g) ksn[g] = __ldg(ksb + (j + 1) * kKGroupsMax + g);
-        }
-        if (!(ok = mbar_wait(bar(C::B_SFULL + q * NSB + buf), (j / NSB) & 1, abort_flag, p.err, kErrTimeoutSoftmax)))
+        for (int g = 0; g < (KPT ? 16 : 2); ++g) ksn[g] = __ldg(ksb + (j + 1) * kKGroupsMax + g);
+      }
+      if (!(ok = mbar_wait(bar(C::B_SFULL + q), j & 1, abort_flag, p.err, kErrTimeoutSoftmax))) break;
+      tc_fence_after();
+      uint32_t r[128];
+      tmem_ld128_sync(taddr, r);
+      // the S columns are read: re-seed them (the stores complete during the
+      // max below) and then let the next QK^T in
+      tmem_fill128(taddr, 0x4B400000u);
+      // keys past the sequence, or (causal) past this row, are masked
+      const int col0 = j * kTile;
+      const bool masked = (col0 + kTile > Lk) || (p.causal && j == qt);
+      const int lim = p.causal ? min(Lk, row + 1) : Lk;
+      float mt;
+      if (SMQ) {
+        // the tile's key corrections arrive with its V tile
+        if (!(ok = mbar_wait(bar(C::B_VFULL + j % C::NST), (j / C::NST) & 1, abort_flag, p.err,
+                             kErrTimeoutSoftmax)))
           break;
+        const float* bias = reinterpret_cast<const float*>(smem + C::OFF_BIAS + ((j % C::NST) * NQ + q) * 512);
+        mt = tile_max_bias<KPT>(r, c, bias, p.sl2, masked, col0, lim);
+      } else {
+        mt = tile_max<KPT>(r, c, masked, col0, lim);
+      }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_SCONS + q));
+      const float m_new = fmaxf(m, mt);
+      const float alpha = (m == -INFINITY) ? 0.f : ex2(m - m_new);
+      // the two softmax warpgroups run half a tile apart, so that one's
+      // exponentials (MUFU) overlap the other's integer / max work
+      if (NQ == 2 && q == 0 && j == 0) mbar_arrive(bar(C::B_GO));
+      // PV_{j-1} must be done before O is rescaled and the P~ buffer rewritten
+      if (j > 0) {
+        if (!(ok = mbar_wait(bar(C::B_OFULL + q), (j - 1) & 1, abort_flag, p.err, kErrTimeoutSoftmax))) break;
         tc_fence_after();
-        // keys past the sequence, or (causal) past this row, are masked
-        const int col0 = j * kTile;
-        const bool masked = (col0 + kTile > Lk) || (p.causal && j == qt);
-        const int lim = p.causal ? min(Lk, row + 1) : Lk;
-        const uint32_t taddr = tmem + C::TM_S + (q * NSB + buf) * 128 + lane_off;
-        float alpha;
-        softmax_tile<PV8, KPT, BF16P>(taddr, c, masked, col0, lim, m, l, alpha);
-        if (ACC2) {
-          const int ab = j & 1;
-          if (!(ok = mbar_wait(bar(C::B_AEMPTY + 2 * q + ab), ((j >> 1) & 1) ^ 1, abort_flag, p.err,
-                               kErrTimeoutSoftmax)))
-            break;
-          alpha_s[(q * 2 + ab) * 128 + t] = alpha;
-          mbar_arrive(bar(C::B_AFULL + 2 * q + ab));
-        } else if (j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-          // O(q) holds the sums of tiles < j (PV_{j-1} finished before S_j did)
-          if (D == 128) {
-            uint32_t r[128];
-            tmem_ld128_sync(ob, r);
+      }
+      if (ACC2) {
+        const int ab = j & 1;
+        if (!(ok = mbar_wait(bar(C::B_AEMPTY + 2 * q + ab), ((j >> 1) & 1) ^ 1, abort_flag, p.err,
+                             kErrTimeoutSoftmax)))
+          break;
+        alpha_s[(q * 2 + ab) * 128 + t] = alpha;
+        mbar_arrive(bar(C::B_AFULL + 2 * q + ab));
+      }
+      const float nb = -(PV8 ? (m_new - kLog2Fp8Max) : m_new);
+      const float lt = tile_exp_store<PV8, KPT, BF16P, SMQ>(r, c, nb, p_smem, t);
+      l = alpha * l + lt;
+      m = m_new;
+      if (!ACC2 && j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+        // O(q) holds the sums of tiles < j
+        if (D == 128) {
+          uint32_t o[128];
+          tmem_ld128_sync(ob, o);
 #pragma unroll
-            for (int u = 0; u < 128; u += 2) {
+          for (int u = 0; u < 128; u += 2) {
+            float x0, x1;
+            mul2(x0, x1, __uint_as_float(o[u]), __uint_as_float(o[u + 1]), alpha, alpha);
+            o[u] = __float_as_uint(x0);
+            o[u + 1] = __float_as_uint(x1);
+          }
+          tmem_st128(ob, o);
+        } else {
+#pragma unroll
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t o[32];
+            tmem_ld32(ob + ch * 32, o);
+            tmem_wait_ld(o);
+#pragma unroll
+            for (int u = 0; u < 32; u += 2) {
               float x0, x1;
-              mul2(x0, x1, __uint_as_float(r[u]), __uint_as_float(r[u + 1]), alpha, alpha);
-              r[u] = __float_as_uint(x0);
-              r[u + 1] = __float_as_uint(x1);
+              mul2(x0, x1, __uint_as_float(o[u]), __uint_as_float(o[u + 1]), alpha, alpha);
+              o[u] = __float_as_uint(x0);
+              o[u + 1] = __float_as_uint(x1);
             }
-            tmem_st128(ob, r);
-          } else {
-#pragma unroll
-            for (int ch = 0; ch < D / 32; ++ch) {
-              uint32_t r[32];
-              tmem_ld32(ob + ch * 32, r);
-              tmem_wait_ld(r);
-#pragma unroll
-              for (int u = 0; u < 32; u += 2) {
-                float x0, x1;
-                mul2(x0, x1, __uint_as_float(r[u]), __uint_as_float(r[u + 1]), alpha, alpha);
-                r[u] = __float_as_uint(x0);
-                r[u + 1] = __float_as_uint(x1);
-              }
-              tmem_st32(ob + ch * 32, r);
-            }
+            tmem_st32(ob + ch * 32, o);
           }
         }
-        tmem_wait_st();
-        tc_fence_before();
-        mbar_arrive(bar(C::B_PFULL + q));
       }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(C::B_PFULL + q));
     }
-    if (ACC2) {
-      l_s[q * 128 + t] = l;
-      mbar_arrive(bar(C::B_LFULL + q));
-    } else if (ok && qt * kTile < Lq) {
-      // epilogue of this query tile
-      if (n[q] > 0) {
-        ok = mbar_wait(bar(C::B_OFULL + q), 0, abort_flag, p.err, kErrTimeoutSoftmax);
-        tc_fence_after();
-      }
-      if (ok) {
-        uint16_t* orow = reinterpret_cast<uint16_t*>(p.out) + (long long)b * p.os.sb + (long long)h * p.os.sh +
-                         (long long)(qs + row) * p.os.ss;
-        store_row<D, PV8, false>(orow, tmem + C::TM_O + q * D + lane_off, nullptr, l > 0.f ? 1.0f / l : 0.f, vsc,
-                                 bf16, n[q] > 0, row < Lq);
-      }
+  }
+  if (ACC2) {
+    l_s[q * 128 + t] = l;
+    mbar_arrive(bar(C::B_LFULL + q));
+  } else if (ok && qt * kTile < Lq) {
+    // epilogue of this query tile
+    if (n[q] > 0) {
+      ok = mbar_wait(bar(C::B_OFULL + q), (n[q] - 1) & 1, abort_flag, p.err, kErrTimeoutSoftmax);
+      tc_fence_after();
     }
+    if (ok) {
+      uint16_t* orow = reinterpret_cast<uint16_t*>(p.out) + (long long)b * p.os.sb + (long long)h * p.os.sh +
+                       (long long)(qs + row) * p.os.ss;
+      store_row<D, PV8, false>(orow, ob, nullptr, l > 0.f ? 1.0f / l : 0.f, vsc, bf16, n[q] > 0, row < Lq);
+    }
+  }
 }
 
 // ---------------------------------------------------------------- kernel
-// Warp roles: 0 loader, 1 MMA issuer, 2 TMEM allocator, 3 idle; warpgroups
-// 1..NQ softmax (one query tile each).  One-level accumulation: the softmax
-// warpgroup also rescales O in TMEM (before releasing P~ to the MMA) and runs
-// the epilogue.  Two-level: warpgroup 2 is the correction warpgroup holding
-// the FP32 outer accumulator in registers.
 template <int D, bool PV8, bool ACC2>
 __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
   using C = AttnCfg<D, PV8, ACC2>;
-  constexpr int NQ = C::NQ, NSB = C::NSB, NST = C::NST;
+  constexpr int NQ = C::NQ, NST = C::NST;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024 - (smem_u32(smem_raw) & 1023)) & 1023);
   const uint32_t sb = smem_u32(smem);
@@ -349,8 +448,9 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
   if (tid == 0) {
     for (int i = 0; i < C::NBAR; ++i) {
       uint32_t cnt = 1;
-      if ((i >= C::B_PFULL && i < C::B_PFULL + NQ) || (i >= C::B_OREADY && i < C::B_OREADY + NQ) ||
-          (i >= C::B_AFULL && i < C::B_AFULL + 4 * NQ) || (i >= C::B_LFULL && i < C::B_LFULL + NQ))
+      if ((i >= C::B_SCONS && i < C::B_SCONS + NQ) || (i >= C::B_PFULL && i < C::B_PFULL + NQ) ||
+          (i >= C::B_OREADY && i < C::B_OREADY + NQ) || (i >= C::B_AFULL && i < C::B_AFULL + 4 * NQ) ||
+          (i >= C::B_LFULL && i < C::B_LFULL + NQ) || i == C::B_GO)
         cnt = 128;
       mbar_init(bar(i), cnt);
     }
@@ -378,16 +478,24 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
         }
       const int8_t* kb = p.k_codes + ((size_t)hk * p.tiles_k + tk0) * C::QT;
       const uint8_t* vb = p.v_codes + ((size_t)hk * p.tiles_k + tk0) * (size_t)C::VT;
+      // smooth Q: bias rows of the valid query tiles (n[q] > 0 for a prefix of q)
+      int nbias = 0;
+      if (p.q_bias)
+        for (int q = 0; q < NQ; ++q) nbias += n[q] > 0;
+      const float* bias_b = p.q_bias ? p.q_bias + ((size_t)h * p.tiles_q + tq0 + pair * NQ) * p.bias_ld : nullptr;
       int issued_k = 0, issued_v = 0;
       for (int t = 0; t < maxn; ++t) {
         const int st = t % NST, u = t / NST;
-        if (u > 0 && !mbar_wait(bar(C::B_KEMPTY + st), (u - 1) & 1, abort_flag, p.err, kErrTimeoutLoad)) break;
+        if (u > 0 && !mbar_wait_poll(bar(C::B_KEMPTY + st), (u - 1) & 1, abort_flag, p.err, kErrTimeoutLoad)) break;
         mbar_expect_tx(bar(C::B_KFULL + st), C::QT);
         bulk_g2s(sb + C::OFF_K + st * C::QT, kb + (size_t)t * C::QT, C::QT, bar(C::B_KFULL + st));
         issued_k = t + 1;
-        if (u > 0 && !mbar_wait(bar(C::B_VEMPTY + st), (u - 1) & 1, abort_flag, p.err, kErrTimeoutLoad)) break;
-        mbar_expect_tx(bar(C::B_VFULL + st), C::VT);
+        if (u > 0 && !mbar_wait_poll(bar(C::B_VEMPTY + st), (u - 1) & 1, abort_flag, p.err, kErrTimeoutLoad)) break;
+        mbar_expect_tx(bar(C::B_VFULL + st), C::VT + nbias * 512);
         bulk_g2s(sb + C::OFF_V + st * C::VT, vb + (size_t)t * C::VT, C::VT, bar(C::B_VFULL + st));
+        for (int q = 0; q < nbias; ++q)     // smooth Q: the query tiles' corrections for key tile t
+          bulk_g2s(sb + C::OFF_BIAS + (st * NQ + q) * 512, bias_b + (size_t)q * p.bias_ld + (size_t)t * kTile, 512,
+                   bar(C::B_VFULL + st));
         issued_v = t + 1;
       }
       if (*abort_flag) {
@@ -409,75 +517,78 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
+    // Per KV tile j: for each query tile, once the softmax has read S_j,
+    // S_{j+1} = Q K_{j+1}^T; then for each query tile, once P~_j is in shared
+    // memory (and, two-level, the last partial O was consumed), O (+)= P~_j V_j.
     if (lane == 0 && maxn > 0) {
       constexpr uint32_t ID_QK = idesc_i8(128, 128);
       const uint32_t ID_PV = PV8 ? idesc_e4m3(128, D) : idesc_f16(128, D, p.out_bf16 != 0);
       bool ok = true;
       for (int q = 0; q < NQ && ok; ++q)
-        if (n[q] > 0) ok = mbar_wait(bar(C::B_QFULL + q), 0, abort_flag, p.err, kErrTimeoutMma);
-      tc_fence_after();
-      auto mma_s = [&](int q, int t, int st) {
-        const uint32_t d = tmem + C::TM_S + (q * NSB + t % NSB) * 128;
+        if (n[q] > 0) ok = mbar_wait_poll(bar(C::B_QFULL + q), 0, abort_flag, p.err, kErrTimeoutMma);
+      auto mma_s = [&](int q, int st) {
+        const uint32_t d = tmem + C::TM_S + q * 128;
 #pragma unroll
         for (int kk = 0; kk < D / 32; ++kk) {
           const uint64_t a = smem_desc(sb + C::OFF_Q + q * C::QT + kk * 32, D);
           const uint64_t bd = smem_desc(sb + C::OFF_K + st * C::QT + kk * 32, D);
-          mma_i8_ss(d, a, bd, ID_QK, kk > 0);
+          mma_i8_ss(d, a, bd, ID_QK, 1);        // onto the 1.5 * 2^23 seed
         }
-        tc_commit(bar(C::B_SFULL + q * NSB + t % NSB));
+        tc_commit(bar(C::B_SFULL + q));
       };
       auto mma_pv = [&](int q, int j, int st) {
-        const uint32_t a0 = tmem + C::TM_S + (q * NSB + j % NSB) * 128;
         const uint32_t d = tmem + C::TM_O + q * D;
+        const uint32_t pa = sb + C::OFF_P + q * C::PT;
+        const uint32_t va = sb + C::OFF_V + st * C::VT;
         if (PV8) {
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            mma_f8_ts(d, a0 + kk * 8, smem_desc(sb + C::OFF_V + st * C::VT + kk * 32, 128), ID_PV,
+            mma_f8_ss(d, smem_desc(pa + kk * 32, 128), smem_desc(va + kk * 32, 128), ID_PV,
                       ACC2 ? (kk > 0) : (j > 0 || kk > 0));
         } else {
 #pragma unroll
           for (int kk = 0; kk < 8; ++kk)
-            mma_f16_ts(d, a0 + kk * 8,
-                       smem_desc(sb + C::OFF_V + st * C::VT + (kk >> 2) * (D * 128) + (kk & 3) * 32, 128), ID_PV,
+            mma_f16_ss(d, smem_desc(pa + (kk >> 2) * (kTile * 128) + (kk & 3) * 32, 128),
+                       smem_desc(va + (kk >> 2) * (D * 128) + (kk & 3) * 32, 128), ID_PV,
                        ACC2 ? (kk > 0) : (j > 0 || kk > 0));
         }
+        tc_commit(bar(C::B_OFULL + q));
       };
-      // S for the first NSB tiles
-      for (int t = 0; t < NSB && t < maxn && ok; ++t) {
-        ok = mbar_wait(bar(C::B_KFULL + t % NST), (t / NST) & 1, abort_flag, p.err, kErrTimeoutMma);
-        if (!ok) break;
-        tc_fence_after();
-        for (int q = 0; q < NQ; ++q)
-          if (t < n[q]) mma_s(q, t, t % NST);
-        tc_commit(bar(C::B_KEMPTY + t % NST));
+      // S_0 (once the softmax warpgroups have seeded the S columns)
+      if (ok && (ok = mbar_wait_poll(bar(C::B_KFULL), 0, abort_flag, p.err, kErrTimeoutMma))) {
+        for (int q = 0; q < NQ && ok; ++q)
+          if (n[q] > 0 && (ok = mbar_wait_poll(bar(C::B_SCONS + q), 0, abort_flag, p.err, kErrTimeoutMma))) {
+            tc_fence_after();
+            mma_s(q, 0);
+          }
+        tc_commit(bar(C::B_KEMPTY));
       }
       for (int j = 0; j < maxn && ok; ++j) {
-        const int st = j % NST, t = j + NSB;
-        if (!(ok = mbar_wait(bar(C::B_VFULL + st), (j / NST) & 1, abort_flag, p.err, kErrTimeoutMma))) break;
-        bool kready = false;
-        for (int q = 0; q < NQ && ok; ++q) {
-          if (j < n[q]) {
-            ok = mbar_wait(bar(C::B_PFULL + q), j & 1, abort_flag, p.err, kErrTimeoutMma);
-            if (ok && ACC2 && j > 0)
-              ok = mbar_wait(bar(C::B_OREADY + q), (j - 1) & 1, abort_flag, p.err, kErrTimeoutMma);
-            if (!ok) break;
+        const int st = j % NST, t = j + 1;
+        // next QK^T as soon as each softmax has read S_j
+        if (t < maxn) {
+          if (!(ok = mbar_wait_poll(bar(C::B_KFULL + t % NST), (t / NST) & 1, abort_flag, p.err, kErrTimeoutMma))) break;
+          for (int q = 0; q < NQ && ok; ++q) {
+            if (t >= n[q]) continue;
+            if (!(ok = mbar_wait_poll(bar(C::B_SCONS + q), t & 1, abort_flag, p.err, kErrTimeoutMma))) break;
             tc_fence_after();
-            mma_pv(q, j, st);
-            if (ACC2 || j == n[q] - 1) tc_commit(bar(C::B_OFULL + q));
+            mma_s(q, t % NST);
           }
-          if (t < n[q]) {
-            if (!kready) {
-              if (!(ok = mbar_wait(bar(C::B_KFULL + t % NST), (t / NST) & 1, abort_flag, p.err, kErrTimeoutMma)))
-                break;
-              tc_fence_after();
-              kready = true;
-            }
-            mma_s(q, t, t % NST);
-          }
+          if (!ok) break;
+          tc_commit(bar(C::B_KEMPTY + t % NST));
+        }
+        if (!(ok = mbar_wait_poll(bar(C::B_VFULL + st), (j / NST) & 1, abort_flag, p.err, kErrTimeoutMma))) break;
+        for (int q = 0; q < NQ && ok; ++q) {
+          if (j >= n[q]) continue;
+          ok = mbar_wait_poll(bar(C::B_PFULL + q), j & 1, abort_flag, p.err, kErrTimeoutMma);
+          if (ok && ACC2 && j > 0)
+            ok = mbar_wait_poll(bar(C::B_OREADY + q), (j - 1) & 1, abort_flag, p.err, kErrTimeoutMma);
+          if (!ok) break;
+          tc_fence_after();
+          mma_pv(q, j, st);
         }
         if (!ok) break;
         tc_commit(bar(C::B_VEMPTY + st));
-        if (kready) tc_commit(bar(C::B_KEMPTY + t % NST));
       }
       // all MMAs issued by this thread complete before teardown
       tc_commit(bar(C::B_DONE));
@@ -487,13 +598,20 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
   } else if (warp >= 4 && warp < 4 + 4 * NQ) {
     // ------------------------------------------------------------ softmax
     const bool bf16p = !PV8 && p.out_bf16;
-    if (p.gran == 2) {
-      if (bf16p) softmax_role<D, PV8, ACC2, true, true>(p, sb, tmem, warp, tid, pair, b, h, hk, qs, Lq, Lk, tq0, tk0, n, vsc);
-      else softmax_role<D, PV8, ACC2, true, false>(p, sb, tmem, warp, tid, pair, b, h, hk, qs, Lq, Lk, tq0, tk0, n, vsc);
-    } else {
-      if (bf16p) softmax_role<D, PV8, ACC2, false, true>(p, sb, tmem, warp, tid, pair, b, h, hk, qs, Lq, Lk, tq0, tk0, n, vsc);
-      else softmax_role<D, PV8, ACC2, false, false>(p, sb, tmem, warp, tid, pair, b, h, hk, qs, Lq, Lk, tq0, tk0, n, vsc);
+    const int variant = (p.gran == 2 ? 4 : 0) + (bf16p ? 2 : 0) + (p.q_bias ? 1 : 0);
+#define SAGE_SOFTMAX(KPT, BF16P, SMQ) \
+  softmax_role<D, PV8, ACC2, KPT, BF16P, SMQ>(p, sb, tmem, warp, tid, pair, b, h, hk, qs, Lq, Lk, tq0, tk0, n, vsc)
+    switch (variant) {
+      case 0: SAGE_SOFTMAX(false, false, false); break;
+      case 1: SAGE_SOFTMAX(false, false, true); break;
+      case 2: SAGE_SOFTMAX(false, true, false); break;
+      case 3: SAGE_SOFTMAX(false, true, true); break;
+      case 4: SAGE_SOFTMAX(true, false, false); break;
+      case 5: SAGE_SOFTMAX(true, false, true); break;
+      case 6: SAGE_SOFTMAX(true, true, false); break;
+      default: SAGE_SOFTMAX(true, true, true); break;
     }
+#undef SAGE_SOFTMAX
   } else if (ACC2 && warp >= 4 + 4 * NQ) {
     // ------------------------------------------------------------ correction (two-level) + epilogue
     const int t = tid - 128 * (1 + NQ);
@@ -544,6 +662,8 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TM_COLS);
   }
+  (void)alpha_s;
+  (void)l_s;
 }
 
 // ---------------------------------------------------------------- debug S tile
@@ -604,6 +724,7 @@ __global__ void __launch_bounds__(128, 1) qk_tile_kernel(const int8_t* qt, const
     tmem_dealloc(tmem, 128);
   }
 }
+
 
 // ---------------------------------------------------------------- launchers
 template <int D, bool PV8, bool ACC2>

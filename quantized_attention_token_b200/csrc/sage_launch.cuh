@@ -29,9 +29,7 @@ struct PrepassJob {
   float* k_scale = nullptr;               // [Hkv][tiles_k][16]
   uint8_t* v_codes = nullptr;
   float* q_mean = nullptr;                // [Hq][tiles_q][D] (smooth Q)
-  uint32_t* ticket = nullptr;             // work-item counter, zero at launch
-  uint32_t* stats_done = nullptr;         // [nseq][Hkv] finished statistics items, zero at launch
-  int* item_off = nullptr;                // varlen: first work item of each sequence [nseq+1]
+  float* q_bias = nullptr;                // [Hq][tiles_q][tps*128] smooth-Q score correction (dense)
 };
 
 struct AttnParams {
@@ -48,6 +46,8 @@ struct AttnParams {
   void* out;
   Strides os;
   float sl2;                 // sm_scale * log2(e)
+  const float* q_bias;       // smooth Q: [Hq][tiles_q][bias_ld] per-key score corrections, else null
+  int bias_ld;
   int gran;
   int causal;
   int out_bf16;
@@ -56,8 +56,7 @@ struct AttnParams {
 // prepass.cu
 cudaError_t prepass_run(const PrepassJob& j, int D, cudaStream_t s);
 cudaError_t prepass_varlen_offsets(const int* cu_q, const int* cu_k, int n, int max_seqlen, int cap_q, int cap_k,
-                                   int* toff_q, int* toff_k, uint32_t* err, const PrepassJob& job,
-                                   cudaStream_t s);
+                                   int* toff_q, int* toff_k, uint32_t* err, cudaStream_t s);
 
 // attn_fwd.cu
 int attn_tiles_per_cta(int D, bool pv8, bool acc2);

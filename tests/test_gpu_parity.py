@@ -99,6 +99,42 @@ def test_prepass_codes_bit_exact(D, S, gran, dtype, layout, smooth_k):
             assert np.array_equal(vs[b, h], rv.scales)
 
 
+@pytest.mark.parametrize("D,S,gran,dtype,layout", [
+    (128, 300, "per_block", "fp16", "HND"),
+    (64, 257, "per_thread", "bf16", "NHD"),
+])
+def test_prepass_smooth_q_bit_exact(D, S, gran, dtype, layout):
+    """Smooth Q: block means, INT8 codes of Q - mean, and the per-key score
+    corrections (fp64 sum in channel order, rounded to float once)."""
+    Hq, Hkv, B = 4, 2, 2
+    sp = synth.Spec("t", Hq=Hq, Hkv=Hkv, D=D, B=B, S=S, dtype=dtype, layout=layout, k_bias_std=3.0,
+                    q_block_offset_std=1.0, seed=35)
+    q, k, v = synth.make(sp)
+    ws = torch.zeros(sage.sage_workspace_bytes(B, Hq, Hkv, S, D, 0, 1), dtype=torch.uint8, device="cuda")
+    sage.quant_qk(_dev(q), _dev(k), ws, layout, gran, smooth_k=True, smooth_q=True)
+    assert sage.get_device_error(ws) == (0, 0)
+    L = sage.workspace_layout(B, B * S, B * S, S, Hq, Hkv, D, smooth_q=1)
+    W = _ws_bytes(ws)
+    tps = (S + 127) // 128
+    tq = L["tiles_q"]
+    qc = wsdecode.codes_int8(W, L, "q_codes", Hq, tq, D)
+    qs = wsdecode.scales(W, L, "q_scale", Hq, tq, 32)
+    qm = wsdecode.f32(W, L, "q_mean", Hq * tq * D).reshape(Hq, tq, D)
+    qb = wsdecode.f32(W, L, "q_bias", Hq * tq * tps * 128).reshape(Hq, tq, tps * 128)
+    pb = oracle.problem(q, k, v, layout)
+    ng = oracle.q_groups_per_block(gran)
+    for b in range(B):
+        for h in range(Hq):
+            r = oracle.quant_q(pb.q[b][h], gran, True)
+            sl = slice(b * tps, (b + 1) * tps)
+            assert np.array_equal(qm[h, sl], r.mu_blk), (b, h)
+            assert np.array_equal(qc[h, sl].reshape(-1, D)[:S], r.codes), (b, h)
+            assert np.array_equal(qs[h, sl, :ng], r.scales), (b, h)
+            kq = oracle.quant_k(pb.k[b][h // (Hq // Hkv)], gran, True, dtype == "fp16")
+            ref = oracle.smooth_q_bias(r, kq).astype(np.float32)
+            assert np.array_equal(qb[h, sl, :S], ref), (b, h)
+
+
 def test_prepass_v16_layout():
     sp = synth.Spec("t", Hq=2, Hkv=2, D=128, B=1, S=200, dtype="bf16", seed=32)
     q, k, v = synth.make(sp)
@@ -156,6 +192,29 @@ def test_attention_matches_oracle(D, S, Hq, Hkv, causal, gran, pv, acc, dtype, l
     torch.cuda.synchronize()
     ref = oracle.attention(q, k, v, layout, causal, gran=gran, pv=pv, with_allowance=True)
     _assert_close(out, ref, dtype, "vs oracle")
+    ex = oracle.attention_exact(q, k, v, layout, causal)
+    o = out.double().cpu().numpy().ravel()
+    cos = o @ ex.ravel() / (np.linalg.norm(o) * np.linalg.norm(ex))
+    assert cos >= 0.999, cos
+
+
+@pytest.mark.parametrize("D,S,causal,gran,pv,acc,dtype,layout", [
+    (128, 384, False, "per_block", "fp8", "fp32", "fp16", "HND"),
+    (128, 300, True, "per_thread", "fp8", "fp32+fp32", "bf16", "NHD"),
+    (64, 257, False, "per_warp", "fp16", "fp32", "fp16", "HND"),
+    (64, 200, True, "per_block", "fp16", "fp32+fp32", "bf16", "HND"),
+])
+def test_attention_smooth_q_matches_oracle(D, S, causal, gran, pv, acc, dtype, layout):
+    """Smooth Q (Q less its block mean, the lost scores restored per key) on
+    inputs whose Q carries per-block offsets, as in the video-DiT workload."""
+    sp = synth.Spec("t", Hq=4, Hkv=2, D=D, B=2, S=S, dtype=dtype, layout=layout, causal=causal, k_bias_std=3.0,
+                    q_block_offset_std=1.0, seed=60 + S)
+    q, k, v = synth.make(sp)
+    out = sage.sageattn(_dev(q), _dev(k), _dev(v), layout, causal, qk_quant_gran=gran, pv_dtype=pv,
+                        pv_accum_dtype=acc, smooth_q=True)
+    torch.cuda.synchronize()
+    ref = oracle.attention(q, k, v, layout, causal, gran=gran, pv=pv, smooth_q=True, with_allowance=True)
+    _assert_close(out, ref, dtype, "smooth Q vs oracle")
     ex = oracle.attention_exact(q, k, v, layout, causal)
     o = out.double().cpu().numpy().ravel()
     cos = o @ ex.ravel() / (np.linalg.norm(o) * np.linalg.norm(ex))
