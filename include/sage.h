@@ -147,8 +147,9 @@ sage_status_t sage_quant_qk(const void* q, const void* k, sage_dtype_t dtype, sa
                             int B, int Hq, int Hkv, int S, int D, sage_gran_t gran,
                             int smooth_k, int smooth_q, void* ws, size_t ws_bytes, void* stream);
 
-/* The whole pre-pass in one launch: sage_quant_qk and sage_quant_v together
- * (Q, K and V read once from HBM; K and V are read a second time from L2). */
+/* The whole pre-pass: sage_quant_qk and sage_quant_v together, in two
+ * launches (Q tiles and the K / V statistics, then the K and V tiles) plus,
+ * with smooth_q, the launch of the per-key smooth-Q corrections. */
 sage_status_t sage_quant_qkv(const void* q, const void* k, const void* v, sage_dtype_t dtype,
                              sage_layout_t layout, int B, int Hq, int Hkv, int S, int D,
                              sage_gran_t gran, sage_pv_t pv, int smooth_k, int smooth_q, void* ws,
