@@ -39,11 +39,14 @@ struct AttnCfg {
   static constexpr int QT = kTile * D;             // bytes of a Q or K tile
   static constexpr int VT = D * kTile * (PV8 ? 1 : 2);
   static constexpr int PT = kTile * kTile * (PV8 ? 1 : 2);   // P~ tile in shared memory
+  // P~ buffers per query tile: two in FP8 one-level mode, so that P~_j is
+  // written while P~V_{j-1} still reads P~_{j-1} (16-bit tiles do not fit twice)
+  static constexpr int NPB = (PV8 && !ACC2) ? 2 : 1;
   static constexpr int OFF_Q = 0;
   static constexpr int OFF_K = OFF_Q + NQ * QT;
   static constexpr int OFF_V = OFF_K + NST * QT;
   static constexpr int OFF_P = OFF_V + NST * VT;
-  static constexpr int OFF_ALPHA = OFF_P + NQ * PT;           // float [NQ][2][128]   (two-level)
+  static constexpr int OFF_ALPHA = OFF_P + NPB * NQ * PT;     // float [NQ][2][128]   (two-level)
   static constexpr int OFF_L = OFF_ALPHA + NQ * 2 * 128 * 4;  // float [NQ][128]      (two-level)
   static constexpr int OFF_BIAS = OFF_L + NQ * 128 * 4;       // float [NST][NQ][128]  (smooth Q)
   static constexpr int OFF_BAR = OFF_BIAS + NST * NQ * 128 * 4;
@@ -279,7 +282,6 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
   const uint32_t lane_off = (uint32_t)((t & ~31)) << 16;
   const int row = qt * kTile + t;
   const bool bf16 = BF16P || (PV8 && p.out_bf16 != 0);
-  const uint32_t p_smem = sb + C::OFF_P + q * C::PT;
   const uint32_t taddr = tmem + C::TM_S + q * 128 + lane_off;
   const uint32_t ob = tmem + C::TM_O + q * D + lane_off;
   float m = -INFINITY, l = 0.f;
@@ -338,11 +340,13 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
       // the two softmax warpgroups run half a tile apart, so that one's
       // exponentials (MUFU) overlap the other's integer / max work
       if (NQ == 2 && q == 0 && j == 0) mbar_arrive(bar(C::B_GO));
-      // PV_{j-1} must be done before O is rescaled and the P~ buffer rewritten
-      if (j > 0) {
+      // PV_{j-1} must be done before the P~ buffer it reads is rewritten (one
+      // buffer) and before O is rescaled (both cases)
+      if (C::NPB == 1 && j > 0) {
         if (!(ok = mbar_wait(bar(C::B_OFULL + q), (j - 1) & 1, abort_flag, p.err, kErrTimeoutSoftmax))) break;
         tc_fence_after();
       }
+      const uint32_t p_smem = sb + C::OFF_P + ((j % C::NPB) * NQ + q) * C::PT;
       if (ACC2) {
         const int ab = j & 1;
         if (!(ok = mbar_wait(bar(C::B_AEMPTY + 2 * q + ab), ((j >> 1) & 1) ^ 1, abort_flag, p.err,
@@ -355,6 +359,10 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
       const float lt = tile_exp_store<PV8, KPT, BF16P, SMQ>(r, c, nb, p_smem, t);
       l = alpha * l + lt;
       m = m_new;
+      if (C::NPB == 2 && j > 0) {
+        if (!(ok = mbar_wait(bar(C::B_OFULL + q), (j - 1) & 1, abort_flag, p.err, kErrTimeoutSoftmax))) break;
+        tc_fence_after();
+      }
       if (!ACC2 && j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
         // O(q) holds the sums of tiles < j
         if (D == 128) {
@@ -538,7 +546,7 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
       };
       auto mma_pv = [&](int q, int j, int st) {
         const uint32_t d = tmem + C::TM_O + q * D;
-        const uint32_t pa = sb + C::OFF_P + q * C::PT;
+        const uint32_t pa = sb + C::OFF_P + ((j % C::NPB) * NQ + q) * C::PT;
         const uint32_t va = sb + C::OFF_V + st * C::VT;
         if (PV8) {
 #pragma unroll
