@@ -65,7 +65,8 @@ struct AttnCfg {
     B_AEMPTY = B_AFULL + 2 * NQ,
     B_LFULL = B_AEMPTY + 2 * NQ,     // softmax -> correction: final row sum (two-level)
     B_DONE = B_LFULL + NQ,
-    B_GO = B_DONE + 1,               // softmax 0 -> softmax 1: start half a tile later
+    B_TOK = B_DONE + 1,              // FP8: exponential-phase token, [0] query tile 0 may run, [1] tile 1 may
+    B_GO = B_TOK + 2,                // 16-bit: softmax 0 -> softmax 1, start after tile 0's maximum
     NBAR = B_GO + 1
   };
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;  // [0] tmem base, [1] abort flag
@@ -299,7 +300,7 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
     tmem_wait_st();
     tc_fence_before();
     mbar_arrive(bar(C::B_SCONS + q));
-    if (NQ == 2 && q == 1 && n[0] > 0) {
+    if (!PV8 && NQ == 2 && q == 1 && n[0] > 0) {
       if (!(ok = mbar_wait(bar(C::B_GO), 0, abort_flag, p.err, kErrTimeoutSoftmax))) n_stop = 0;
     }
     for (int j = 0; j < n_stop; ++j) {
@@ -337,9 +338,7 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
       mbar_arrive(bar(C::B_SCONS + q));
       const float m_new = fmaxf(m, mt);
       const float alpha = (m == -INFINITY) ? 0.f : ex2(m - m_new);
-      // the two softmax warpgroups run half a tile apart, so that one's
-      // exponentials (MUFU) overlap the other's integer / max work
-      if (NQ == 2 && q == 0 && j == 0) mbar_arrive(bar(C::B_GO));
+      if (!PV8 && NQ == 2 && q == 0 && j == 0) mbar_arrive(bar(C::B_GO));
       // PV_{j-1} must be done before the P~ buffer it reads is rewritten (one
       // buffer) and before O is rescaled (both cases)
       if (C::NPB == 1 && j > 0) {
@@ -356,7 +355,20 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
         mbar_arrive(bar(C::B_AFULL + 2 * q + ab));
       }
       const float nb = -(PV8 ? (m_new - kLog2Fp8Max) : m_new);
+      // Two query tiles: their exponential phases take turns (tile 0's of KV
+      // tile j, then tile 1's, then tile 0's of j+1, ...), so that each runs
+      // at the MUFU's full rate while the other warpgroup does its maximum and
+      // O rescale.  A tile waits only for turns its partner has (causal: the
+      // second query tile can have one KV tile more than the first).
+      if (PV8 && NQ == 2) {
+        const bool wait_turn = q == 0 ? (j > 0 && j - 1 < n[1]) : (j < n[0]);
+        if (wait_turn &&
+            !(ok = mbar_wait(bar(C::B_TOK + q), q == 0 ? ((j - 1) & 1) : (j & 1), abort_flag, p.err,
+                             kErrTimeoutSoftmax)))
+          break;
+      }
       const float lt = tile_exp_store<PV8, KPT, BF16P, SMQ>(r, c, nb, p_smem, t);
+      if (PV8 && NQ == 2 && (q == 0 ? j < n[1] : j + 1 < n[0])) mbar_arrive(bar(C::B_TOK + (q ^ 1)));
       l = alpha * l + lt;
       m = m_new;
       if (C::NPB == 2 && j > 0) {
@@ -458,7 +470,7 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
       uint32_t cnt = 1;
       if ((i >= C::B_SCONS && i < C::B_SCONS + NQ) || (i >= C::B_PFULL && i < C::B_PFULL + NQ) ||
           (i >= C::B_OREADY && i < C::B_OREADY + NQ) || (i >= C::B_AFULL && i < C::B_AFULL + 4 * NQ) ||
-          (i >= C::B_LFULL && i < C::B_LFULL + NQ) || i == C::B_GO)
+          (i >= C::B_LFULL && i < C::B_LFULL + NQ) || i == C::B_TOK || i == C::B_TOK + 1 || i == C::B_GO)
         cnt = 128;
       mbar_init(bar(i), cnt);
     }
