@@ -76,8 +76,11 @@ typedef enum { SAGE_F16 = 0, SAGE_BF16 = 1 } sage_dtype_t;
  *   PER_WARP  : Q four groups of 32 rows; K two groups of 64 rows.
  *   PER_THREAD: Q rows of each 32-row slice with equal (row mod 8) share a
  *               scale (32 groups); K rows of each 64-row half with equal
- *               (row mod 8) share a scale (16 groups).                        */
-typedef enum { SAGE_PER_BLOCK = 0, SAGE_PER_WARP = 1, SAGE_PER_THREAD = 2 } sage_gran_t;
+ *               (row mod 8) share a scale (16 groups).
+ *   PER_TOKEN : Q one group per row (128 groups) [repo summary, Tinh nang
+ *               chinh: per-token granularity]; K two groups of 64 rows.
+ * q_scale holds 128 slots per tile, k_scale 16 (unused slots are unwritten). */
+typedef enum { SAGE_PER_BLOCK = 0, SAGE_PER_WARP = 1, SAGE_PER_THREAD = 2, SAGE_PER_TOKEN = 3 } sage_gran_t;
 
 /* P~V precision: FP8 E4M3 (P~ scale 1/448 static, V scale per channel) or
  * 16-bit (P~ rounded to the input's 16-bit type, V unquantized). */
@@ -104,7 +107,7 @@ size_t sage_varlen_workspace_bytes(int n_seqs, int total_q, int total_k, int max
  * tensors, e.g. to cache K/V).  Quantized tiles hold 128 tokens; tile t of
  * sequence b is global tile tile_off(b) + t (dense: b*ceil(S/128) + t).
  *   q_codes : int8  [Hq ][tiles_q][128 rows][D]   swizzled, see below
- *   q_scale : float [Hq ][tiles_q][32]            group g of the tile at [g]
+ *   q_scale : float [Hq ][tiles_q][128]           group g of the tile at [g]
  *   k_codes : int8  [Hkv][tiles_k][128 rows][D]   swizzled
  *   k_scale : float [Hkv][tiles_k][16]
  *   k_mean  : float [n_seqs][Hkv][D]              (0 when smooth_k is off)

@@ -23,7 +23,7 @@ import torch
 
 from . import build as _build
 
-GRAN = {"per_block": 0, "per_warp": 1, "per_thread": 2}
+GRAN = {"per_block": 0, "per_warp": 1, "per_thread": 2, "per_token": 3}
 PV = {"fp8": 0, "fp16": 1}
 
 _lib = None

@@ -122,14 +122,16 @@ ORC_EXPORT double orc_round_bf16(double x) { return round_to_bf16(x); }
 /*               per slice, 32 per block;                                   */
 /*               K rows of a 64-row half with equal (row mod 8) -> 8 groups  */
 /*               per half, 16 per block.                                    */
+/*   per_token : Q one group per row [REPO, Tinh nang chinh: per-token      */
+/*               granularity];                K two groups of 64 rows.     */
 /* (per_thread mirrors the thread-to-row map of the m16n8k32 MMA fragments  */
 /* the pages' kernels were written for: a thread owns rows r and r+8 of     */
 /* each 16-row slab, hence one scale per residue mod 8.)                    */
 /* ------------------------------------------------------------------------ */
-enum { ORC_PER_BLOCK = 0, ORC_PER_WARP = 1, ORC_PER_THREAD = 2 };
+enum { ORC_PER_BLOCK = 0, ORC_PER_WARP = 1, ORC_PER_THREAD = 2, ORC_PER_TOKEN = 3 };
 
 ORC_EXPORT int orc_q_groups_per_block(int gran) {
-    return gran == ORC_PER_BLOCK ? 1 : gran == ORC_PER_WARP ? 4 : 32;
+    return gran == ORC_PER_BLOCK ? 1 : gran == ORC_PER_WARP ? 4 : gran == ORC_PER_TOKEN ? 128 : 32;
 }
 ORC_EXPORT int orc_k_groups_per_block(int gran) {
     return gran == ORC_PER_THREAD ? 16 : 2;
@@ -137,6 +139,7 @@ ORC_EXPORT int orc_k_groups_per_block(int gran) {
 ORC_EXPORT int orc_q_group(int gran, int r) {           /* r: row within its 128-block */
     if (gran == ORC_PER_BLOCK) return 0;
     if (gran == ORC_PER_WARP) return r / 32;
+    if (gran == ORC_PER_TOKEN) return r;
     return (r / 32) * 8 + (r % 8);
 }
 ORC_EXPORT int orc_k_group(int gran, int r) {

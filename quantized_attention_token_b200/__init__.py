@@ -27,7 +27,7 @@ LIB_PATH = os.path.join(HERE, "libsage.so")
 
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
 LAYOUT = {"HND": 0, "NHD": 1}
-GRAN = {"per_block": 0, "per_warp": 1, "per_thread": 2}
+GRAN = {"per_block": 0, "per_warp": 1, "per_thread": 2, "per_token": 3}
 PV = {"fp8": 0, "fp16": 1}
 ACC = {"fp32": 0, "fp32+fp32": 1, "fp32fp32": 1}
 

@@ -91,7 +91,8 @@ sage_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? SAGE_OK : S
 
 sage_status_t check_common(sage_dtype_t dtype, int D, sage_gran_t gran, sage_pv_t pv, sage_acc_t acc) {
   if (dtype != SAGE_F16 && dtype != SAGE_BF16) return SAGE_ERR_INVALID_ARG;
-  if (gran != SAGE_PER_BLOCK && gran != SAGE_PER_WARP && gran != SAGE_PER_THREAD) return SAGE_ERR_INVALID_ARG;
+  if (gran != SAGE_PER_BLOCK && gran != SAGE_PER_WARP && gran != SAGE_PER_THREAD && gran != SAGE_PER_TOKEN)
+    return SAGE_ERR_INVALID_ARG;
   if (pv != SAGE_PV_FP8 && pv != SAGE_PV_FP16) return SAGE_ERR_INVALID_ARG;
   if (acc != SAGE_ACC_FP32 && acc != SAGE_ACC_FP32_FP32) return SAGE_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return SAGE_ERR_UNSUPPORTED;

@@ -217,11 +217,21 @@ __device__ void quant_tile(const PrepassJob& j, int h, int t, const TileLoc& L, 
     for (int u = 0; u < 8; ++u) m = fmaxf(m, fabsf(x[u]));
 #pragma unroll
     for (int o = M::TPR / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    if (cc == 0) sm.rowmax[rg * M::NR + i] = m;
+    if (cc == 0) {
+      const int r = rg * M::NR + i;
+      if (IS_Q && j.gran == 3) {
+        // per-token Q: the row is its own group (rows past the sequence: 0)
+        const float am = r < L.nvalid ? m : 0.f;
+        sm.ginv[r] = am > 0.f ? __fdiv_rn(127.0f, am) : 0.f;
+        j.q_scale[((size_t)h * tiles + t) * kQGroupsMax + r] = __fdiv_rn(am, 127.0f);
+      } else {
+        sm.rowmax[r] = m;
+      }
+    }
   }
   __syncthreads();
   // group |max| -> the scale amax / 127 and the multiplier 127 / amax
-  const int ng = IS_Q ? q_ngroups(j.gran) : k_ngroups(j.gran);
+  const int ng = (IS_Q && j.gran == 3) ? 0 : IS_Q ? q_ngroups(j.gran) : k_ngroups(j.gran);
   for (int g = warp; g < ng; g += M::WARPS) {
     float m = 0.f;
 #pragma unroll

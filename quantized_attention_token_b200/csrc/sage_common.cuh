@@ -15,7 +15,7 @@ namespace sage {
 
 // ---------------------------------------------------------------- constants
 constexpr int kTile = 128;            // tokens per quantization block and per MMA tile
-constexpr int kQGroupsMax = 32;       // q_scale slots per tile (per_thread Q)
+constexpr int kQGroupsMax = 128;      // q_scale slots per tile (per_token Q)
 constexpr int kKGroupsMax = 16;       // k_scale slots per tile (per_thread K)
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kFp8Max = 448.0f;     // largest finite E4M3 value: the static P~ scale
@@ -63,12 +63,14 @@ struct Strides {
 // ---------------------------------------------------------------- groups
 // Group id of row r (0..127) of a 128-token block; see sage.h for the shapes.
 __host__ __device__ __forceinline__ int q_group(int gran, int r) {
-  return gran == 0 ? 0 : gran == 1 ? (r >> 5) : ((r >> 5) << 3) + (r & 7);
+  return gran == 0 ? 0 : gran == 1 ? (r >> 5) : gran == 3 ? r : ((r >> 5) << 3) + (r & 7);
 }
 __host__ __device__ __forceinline__ int k_group(int gran, int r) {
   return gran == 2 ? ((r >> 6) << 3) + (r & 7) : (r >> 6);
 }
-__host__ __device__ __forceinline__ int q_ngroups(int gran) { return gran == 0 ? 1 : gran == 1 ? 4 : 32; }
+__host__ __device__ __forceinline__ int q_ngroups(int gran) {
+  return gran == 0 ? 1 : gran == 1 ? 4 : gran == 3 ? 128 : 32;
+}
 __host__ __device__ __forceinline__ int k_ngroups(int gran) { return gran == 2 ? 16 : 2; }
 
 // Byte offset of (row, byte col) inside a swizzled operand tile whose rows are

@@ -54,6 +54,8 @@ def _ws_bytes(ws: torch.Tensor) -> np.ndarray:
     (64, 1000, "per_thread", "fp16", "HND"),
     (64, 129, "per_block", "bf16", "HND"),
     (128, 700, "per_thread", "bf16", "NHD"),
+    (128, 333, "per_token", "fp16", "HND"),
+    (64, 200, "per_token", "bf16", "NHD"),
 ])
 @pytest.mark.parametrize("smooth_k", [True, False])
 def test_prepass_codes_bit_exact(D, S, gran, dtype, layout, smooth_k):
@@ -69,7 +71,7 @@ def test_prepass_codes_bit_exact(D, S, gran, dtype, layout, smooth_k):
     tps = (S + 127) // 128
     qc = wsdecode.codes_int8(W, L, "q_codes", 4, L["tiles_q"], D)
     kc = wsdecode.codes_int8(W, L, "k_codes", 2, L["tiles_k"], D)
-    qs = wsdecode.scales(W, L, "q_scale", 4, L["tiles_q"], 32)
+    qs = wsdecode.scales(W, L, "q_scale", 4, L["tiles_q"], 128)
     ks = wsdecode.scales(W, L, "k_scale", 2, L["tiles_k"], 16)
     v8 = wsdecode.v_fp8(W, L, 2, L["tiles_k"], D)
     vs = wsdecode.f32(W, L, "v_scale", 2 * 2 * D).reshape(2, 2, D)
@@ -118,7 +120,7 @@ def test_prepass_smooth_q_bit_exact(D, S, gran, dtype, layout):
     tps = (S + 127) // 128
     tq = L["tiles_q"]
     qc = wsdecode.codes_int8(W, L, "q_codes", Hq, tq, D)
-    qs = wsdecode.scales(W, L, "q_scale", Hq, tq, 32)
+    qs = wsdecode.scales(W, L, "q_scale", Hq, tq, 128)
     qm = wsdecode.f32(W, L, "q_mean", Hq * tq * D).reshape(Hq, tq, D)
     qb = wsdecode.f32(W, L, "q_bias", Hq * tq * tps * 128).reshape(Hq, tq, tps * 128)
     pb = oracle.problem(q, k, v, layout)
@@ -179,6 +181,8 @@ CASES = [
     (64, 129, 2, 2, False, "per_thread", "fp8", "fp32+fp32", "bf16", "NHD"),
     (128, 1, 2, 2, False, "per_block", "fp8", "fp32", "fp16", "HND"),
     (128, 127, 2, 2, True, "per_block", "fp8", "fp32+fp32", "fp16", "HND"),
+    (128, 400, 4, 2, True, "per_token", "fp8", "fp32", "fp16", "HND"),
+    (64, 300, 2, 2, False, "per_token", "fp16", "fp32+fp32", "bf16", "NHD"),
 ]
 
 

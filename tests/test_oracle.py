@@ -148,7 +148,7 @@ def test_int8_quantizer_bounds(gran, is_q):
             assert r.row_scales[t] == np.float32(sub.max()) / np.float32(127)
 
 
-@pytest.mark.parametrize("gran", ["per_block", "per_warp", "per_thread"])
+@pytest.mark.parametrize("gran", ["per_block", "per_warp", "per_thread", "per_token"])
 @pytest.mark.parametrize("is_q", [True, False])
 def test_int8_group_membership_by_brute_force(gran, is_q):
     """Blowing up one token must change the scale of exactly the tokens that
@@ -156,7 +156,7 @@ def test_int8_group_membership_by_brute_force(gran, is_q):
     L, D = 256, 64
     base = np.ones((L, D), np.float32)
     ref = oracle._quant_int8(base, is_q, gran, None).row_scales
-    expect_groups = {"per_block": (1, 2), "per_warp": (4, 2), "per_thread": (32, 16)}[gran]
+    expect_groups = {"per_block": (1, 2), "per_warp": (4, 2), "per_thread": (32, 16), "per_token": (128, 2)}[gran]
     ng = expect_groups[0] if is_q else expect_groups[1]
     assert (oracle.q_groups_per_block if is_q else oracle.k_groups_per_block)(gran) == ng
     for t in range(0, L, 7):
@@ -166,7 +166,10 @@ def test_int8_group_membership_by_brute_force(gran, is_q):
         changed = set(np.nonzero(rs != ref)[0])
         blk = t // 128
         r = t % 128
-        if gran == "per_block":
+        if gran == "per_token":
+            size = 1 if is_q else 64
+            members = {u for u in range(L) if u // 128 == blk and (u % 128) // size == r // size}
+        elif gran == "per_block":
             size = 128 if is_q else 64
             members = {u for u in range(L) if u // 128 == blk and (u % 128) // size == r // size}
         elif gran == "per_warp":
@@ -177,6 +180,18 @@ def test_int8_group_membership_by_brute_force(gran, is_q):
             members = {u for u in range(L) if u // 128 == blk and (u % 128) // size == r // size
                        and u % 8 == t % 8}
         assert changed == members, (t, sorted(changed)[:8], sorted(members)[:8])
+
+
+def test_int8_per_token_scale_is_the_row_maximum():
+    """Per-token Q: every row's scale is its own |max| / 127 (closed form),
+    and its largest element gets code +-127."""
+    rng = np.random.default_rng(11)
+    L, D = 300, 64
+    xs = (rng.standard_normal((L, D)) * rng.uniform(0.01, 50, (L, 1))).astype(np.float32)
+    r = oracle._quant_int8(xs, True, "per_token", None)
+    am = np.abs(xs).max(axis=1)
+    assert np.array_equal(r.row_scales, (am / np.float32(127)).astype(np.float32))
+    assert np.all(np.abs(r.codes).max(axis=1) == 127)
 
 
 def test_int8_zero_group():
