@@ -168,6 +168,7 @@ class QuantQ:
 class QuantV:
     codes: np.ndarray             # [L, D] uint8 E4M3
     scales: np.ndarray            # [D] float32
+    mu: Optional[np.ndarray] = None   # [D] float32 channel mean (smooth V only)
 
 
 def quant_k(k: np.ndarray, gran: str, smooth_k: bool, is_fp16: bool) -> QuantK:
@@ -205,12 +206,24 @@ def _quant_int8(xs: np.ndarray, is_q: bool, gran: str, mu) -> QuantK:
     return QuantK(mu, codes, scales, rs)
 
 
-def quant_v(v: np.ndarray) -> QuantV:
+def quant_v(v: np.ndarray, smooth: bool = False, is_fp16: bool = True) -> QuantV:
+    """Per-channel E4M3 V [SA2, FP8 quantization of P~V].  smooth: the
+    optional smooth-V step the same page names next to the FP32 buffer (no
+    formula given; reading): V is first reduced by its channel mean over the
+    sequence's tokens (exact sum, as for K) with one float32 subtraction, and
+    attention adds the mean back to its output (rows of softmax sum to 1)."""
     L, D = v.shape
     codes = np.empty((L, D), dtype=np.uint8)
     dv = np.empty(D, dtype=np.float32)
+    mu = None
+    if smooth:
+        mu = np.empty(D, dtype=np.float32)
+        lib().orc_channel_mean(_p(v), L, D, int(is_fp16), _p(mu))
+        xs = np.empty((L, D), dtype=np.float32)
+        lib().orc_subtract_channel(_p(v), L, D, _p(mu), _p(xs))
+        v = xs.astype(np.float64)
     lib().orc_quant_v_fp8(_p(v), L, D, _p(codes), _p(dv))
-    return QuantV(codes, dv)
+    return QuantV(codes, dv, mu)
 
 
 def scores_int32(qc: np.ndarray, kc: np.ndarray) -> np.ndarray:
@@ -242,6 +255,8 @@ def attn_head(qq: QuantQ, kq: QuantK, vq: Optional[QuantV], v16: Optional[np.nda
         _p(vq.codes) if vq is not None else None, _p(vq.scales) if vq is not None else None,
         _p(v16), PV[pv], int(v_is_bf16), _p(bias), Lq, Lk, D, int(causal),
         ctypes.c_float(sm_scale), r0, r1, _p(out), _p(allow))
+    if vq is not None and vq.mu is not None:
+        out[r0:r1] += vq.mu.astype(np.float64)      # smooth V: the mean comes back
     return out
 
 
@@ -297,7 +312,7 @@ def quantize(pb: Problem, gran: str = "per_block", smooth_k: bool = True, smooth
 def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout: str = "HND",
               causal: bool = False, sm_scale: Optional[float] = None, gran: str = "per_block",
               pv: str = "fp8", smooth_k: bool = True, smooth_q: bool = False,
-              cu_seqlens: Optional[np.ndarray] = None,
+              cu_seqlens: Optional[np.ndarray] = None, smooth_v: bool = False,
               q_rows: Optional[Dict[Tuple[int, int], Tuple[int, int]]] = None,
               heads: Optional[List[Tuple[int, int]]] = None, with_allowance: bool = False):
     """The quantized forward pass; returns fp64 output shaped like q.
@@ -314,7 +329,7 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout: str = "
     for b in range(len(pb.q)):
         needed_kv = {h // group for h in range(pb.Hq) if heads is None or (b, h) in heads}
         kq = {hk: quant_k(pb.k[b][hk], gran, smooth_k, pb.is_fp16) for hk in needed_kv}
-        vq = {hk: (quant_v(pb.v[b][hk]) if pv == "fp8" else None) for hk in needed_kv}
+        vq = {hk: (quant_v(pb.v[b][hk], smooth_v, pb.is_fp16) if pv == "fp8" else None) for hk in needed_kv}
         row, arow = [], []
         for h in range(pb.Hq):
             al = np.zeros_like(pb.q[b][h])

@@ -466,3 +466,39 @@ def test_allowance_is_sparse_and_bounded(pv):
     step = 32.0 / 448 if pv == "fp8" else 2 ** -11
     vmax = float(v.abs().max())
     assert np.max(allow) <= 512 * step * vmax
+
+
+# ----------------------------------------------------------------------------- smooth V
+def test_smooth_v_constant_channels_are_exact():
+    """Smooth V with V constant per channel: V - mean is exactly 0, so every
+    code and scale is 0 and the output is the mean itself, exactly."""
+    rng = np.random.default_rng(21)
+    B, H, S, D = 1, 2, 200, 64
+    q = torch.from_numpy(rng.standard_normal((B, H, S, D)).astype(np.float16))
+    k = torch.from_numpy(rng.standard_normal((B, H, S, D)).astype(np.float16))
+    v0 = rng.standard_normal((1, H, 1, D)).astype(np.float16)
+    v = torch.from_numpy(np.broadcast_to(v0, (B, H, S, D)).copy())
+    pb = oracle.problem(q, k, v)
+    r = oracle.quant_v(pb.v[0][0], smooth=True, is_fp16=True)
+    assert np.all(r.codes == 0) and np.all(r.scales == 0)
+    assert np.array_equal(r.mu, v0[0, 0, 0].astype(np.float32))
+    out = oracle.attention(q, k, v, pv="fp8", smooth_v=True)
+    assert np.array_equal(out, np.broadcast_to(v0.astype(np.float64), out.shape))
+
+
+def test_smooth_v_reduces_error_on_channel_offsets():
+    """The method's purpose: with large per-channel V offsets, FP8 V carries
+    the offset's rounding error; smoothing V removes it (reading of the
+    page's optional smooth-V step).  Error against exact fp64 attention."""
+    rng = np.random.default_rng(22)
+    B, H, S, D = 1, 2, 384, 64
+    q = torch.from_numpy(rng.standard_normal((B, H, S, D)).astype(np.float16))
+    k = torch.from_numpy(rng.standard_normal((B, H, S, D)).astype(np.float16))
+    v = (rng.standard_normal((B, H, S, D)) + rng.normal(0, 20, (1, H, 1, D))).astype(np.float16)
+    v = torch.from_numpy(v)
+    ex = oracle.attention_exact(q, k, v)
+    plain = oracle.attention(q, k, v, pv="fp8")
+    smooth = oracle.attention(q, k, v, pv="fp8", smooth_v=True)
+    e_plain = np.abs(plain - ex).mean()
+    e_smooth = np.abs(smooth - ex).mean()
+    assert e_smooth < 0.5 * e_plain, (e_smooth, e_plain)
