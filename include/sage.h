@@ -83,8 +83,12 @@ typedef enum { SAGE_F16 = 0, SAGE_BF16 = 1 } sage_dtype_t;
 typedef enum { SAGE_PER_BLOCK = 0, SAGE_PER_WARP = 1, SAGE_PER_THREAD = 2, SAGE_PER_TOKEN = 3 } sage_gran_t;
 
 /* P~V precision: FP8 E4M3 (P~ scale 1/448 static, V scale per channel) or
- * 16-bit (P~ rounded to the input's 16-bit type, V unquantized). */
-typedef enum { SAGE_PV_FP8 = 0, SAGE_PV_FP16 = 1 } sage_pv_t;
+ * 16-bit (P~ rounded to the input's 16-bit type, V unquantized).
+ * FP8_SMOOTH_V: FP8 with V smoothed first -- V less its per-channel mean over
+ * the sequence's tokens is quantized, and the mean is added to the output
+ * (softmax rows sum to 1) [SageAttention2 summary, SageAttention2方法: the
+ * optional smooth-V step]. */
+typedef enum { SAGE_PV_FP8 = 0, SAGE_PV_FP16 = 1, SAGE_PV_FP8_SMOOTH_V = 2 } sage_pv_t;
 
 /* P~V accumulation: FP32 = one FP32 tensor-memory accumulator across all KV
  * tiles; FP32_FP32 = a fresh FP32 partial sum per 128-key tile added into a
@@ -114,6 +118,7 @@ size_t sage_varlen_workspace_bytes(int n_seqs, int total_q, int total_k, int max
  *   v_codes : [Hkv][tiles_k][D rows][128 keys]    E4M3 (1 byte) or 16-bit
  *             (2 bytes, as two [D][64-key] halves of 128-byte rows)
  *   v_scale : float [n_seqs][Hkv][D]              (FP8 mode)
+ *   v_mean  : float [n_seqs][Hkv][D]              (FP8_SMOOTH_V; else unwritten)
  *   q_mean  : float [Hq][tiles_q][D]              (smooth_q)
  *   q_bias  : float [Hq][tiles_q][tiles_k_seq*128] (smooth_q, dense only)
  * Swizzle of every 128-byte row r (D=128 codes, E4M3 V rows, 16-bit V halves):
@@ -124,8 +129,8 @@ size_t sage_varlen_workspace_bytes(int n_seqs, int total_q, int total_k, int max
 typedef struct {
   size_t err;       /* uint32 device error word */
   size_t tile_off_q, tile_off_k;   /* int32 [n_seqs+1] (varlen) */
-  size_t k_stat, v_stat;           /* pre-pass accumulators */
-  size_t k_mean, v_scale;
+  size_t k_stat, v_sum, v_stat;    /* pre-pass accumulators */
+  size_t k_mean, v_scale, v_mean;
   size_t q_codes, q_scale, k_codes, k_scale, v_codes;
   size_t q_mean, q_bias;
   size_t total;
@@ -158,8 +163,9 @@ sage_status_t sage_quant_qkv(const void* q, const void* k, const void* v, sage_d
                              sage_gran_t gran, sage_pv_t pv, int smooth_k, int smooth_q, void* ws,
                              size_t ws_bytes, void* stream);
 
-/* Quantize V per channel to E4M3 (pv == SAGE_PV_FP8) or re-lay it out in 16
- * bits (SAGE_PV_FP16), transposed to [D][keys] tiles.  [SageAttention2
+/* Quantize V per channel to E4M3 (SAGE_PV_FP8; smoothed first with
+ * SAGE_PV_FP8_SMOOTH_V) or re-lay it out in 16 bits (SAGE_PV_FP16),
+ * transposed to [D][keys] tiles.  [SageAttention2
  * summary, SageAttention2方法, FP8 quantization of P~V]  Writes v_stat,
  * v_scale, v_codes. */
 sage_status_t sage_quant_v(const void* v, sage_dtype_t dtype, sage_layout_t layout, int B, int Hkv,

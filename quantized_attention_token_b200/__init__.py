@@ -28,7 +28,7 @@ LIB_PATH = os.path.join(HERE, "libsage.so")
 OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = range(6)
 LAYOUT = {"HND": 0, "NHD": 1}
 GRAN = {"per_block": 0, "per_warp": 1, "per_thread": 2, "per_token": 3}
-PV = {"fp8": 0, "fp16": 1}
+PV = {"fp8": 0, "fp16": 1, "fp8_smooth_v": 2}   # fp8_smooth_v: FP8 with V smoothed by its channel mean
 ACC = {"fp32": 0, "fp32+fp32": 1, "fp32fp32": 1}
 
 
@@ -40,8 +40,8 @@ class SageError(RuntimeError):
 
 class WsLayout(ctypes.Structure):
     _fields_ = [(n, ctypes.c_size_t) for n in (
-        "err", "tile_off_q", "tile_off_k", "k_stat", "v_stat", "k_mean", "v_scale", "q_codes",
-        "q_scale", "k_codes", "k_scale", "v_codes", "q_mean", "q_bias", "total")] + [
+        "err", "tile_off_q", "tile_off_k", "k_stat", "v_sum", "v_stat", "k_mean", "v_scale", "v_mean",
+        "q_codes", "q_scale", "k_codes", "k_scale", "v_codes", "q_mean", "q_bias", "total")] + [
         ("tiles_q", ctypes.c_int), ("tiles_k", ctypes.c_int)]
 
 
@@ -147,13 +147,21 @@ def _contig(t, name):
     return t
 
 
+def _pv_mode(pv_dtype: str, smooth_v: bool) -> str:
+    if smooth_v and pv_dtype not in ("fp8", "fp8_smooth_v"):
+        raise ValueError("smooth_v applies to FP8 P~V only")
+    return "fp8_smooth_v" if smooth_v else pv_dtype
+
+
 def sageattn(q, k, v, tensor_layout: str = "HND", is_causal: bool = False, sm_scale: Optional[float] = None,
              qk_quant_gran: str = "per_block", pv_dtype: str = "fp8", pv_accum_dtype: str = "fp32+fp32",
-             smooth_k: bool = True, smooth_q: bool = False, out=None, workspace=None):
+             smooth_k: bool = True, smooth_q: bool = False, smooth_v: bool = False, out=None,
+             workspace=None):
     """Quantized attention forward; returns a tensor shaped like q.
 
     q: [B, Hq, S, D] (HND) or [B, S, Hq, D] (NHD); k, v likewise with Hkv
-    heads; fp16 or bf16; D in {64, 128}.
+    heads; fp16 or bf16; D in {64, 128}.  smooth_v (FP8 P~V only) is the
+    pv_dtype "fp8_smooth_v".
     """
     torch = _torch()
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
@@ -170,7 +178,7 @@ def sageattn(q, k, v, tensor_layout: str = "HND", is_causal: bool = False, sm_sc
         Sk, Hkv = k.shape[1], k.shape[2]
     if Sk != S or k.shape[0] != B or k.shape[3] != D:
         raise ValueError("sageattn: q and k/v must share batch, sequence length and head dim")
-    pv, acc, gran = PV[pv_dtype], ACC[pv_accum_dtype], GRAN[qk_quant_gran]
+    pv, acc, gran = PV[_pv_mode(pv_dtype, smooth_v)], ACC[pv_accum_dtype], GRAN[qk_quant_gran]
     nbytes = sage_workspace_bytes(B, Hq, Hkv, S, D, pv, int(smooth_q))
     if nbytes == 0:
         raise ValueError("sageattn: unsupported sizes")
@@ -186,7 +194,8 @@ def sageattn(q, k, v, tensor_layout: str = "HND", is_causal: bool = False, sm_sc
 
 def sageattn_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen: int, is_causal: bool = False,
                     sm_scale: Optional[float] = None, qk_quant_gran: str = "per_block", pv_dtype: str = "fp8",
-                    pv_accum_dtype: str = "fp32+fp32", smooth_k: bool = True, out=None, workspace=None):
+                    pv_accum_dtype: str = "fp32+fp32", smooth_k: bool = True, smooth_v: bool = False, out=None,
+                    workspace=None):
     """Packed variable-length attention with GQA: q [Tq, Hq, D], k/v [Tk, Hkv, D],
     cu_seqlens_* int32 CUDA tensors [n+1]."""
     torch = _torch()
@@ -199,7 +208,7 @@ def sageattn_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen: int, is_cau
         raise ValueError("sageattn_varlen: cu_seqlens_q/k must have the same n+1 >= 2 entries")
     Tq, Hq, D = q.shape
     Tk, Hkv = k.shape[0], k.shape[1]
-    pv, acc, gran = PV[pv_dtype], ACC[pv_accum_dtype], GRAN[qk_quant_gran]
+    pv, acc, gran = PV[_pv_mode(pv_dtype, smooth_v)], ACC[pv_accum_dtype], GRAN[qk_quant_gran]
     nbytes = sage_varlen_workspace_bytes(n, Tq, Tk, max_seqlen, Hq, Hkv, D, pv)
     if nbytes == 0:
         raise ValueError("sageattn_varlen: unsupported sizes")

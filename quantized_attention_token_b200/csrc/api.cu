@@ -44,7 +44,7 @@ sage_status_t plan(int nseq, int total_q, int total_k, int max_seqlen, int Hq, i
     return SAGE_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return SAGE_ERR_UNSUPPORTED;
   if (Hq % Hkv != 0) return SAGE_ERR_UNSUPPORTED;
-  if (pv != SAGE_PV_FP8 && pv != SAGE_PV_FP16) return SAGE_ERR_INVALID_ARG;
+  if (pv != SAGE_PV_FP8 && pv != SAGE_PV_FP16 && pv != SAGE_PV_FP8_SMOOTH_V) return SAGE_ERR_INVALID_ARG;
   if (smooth_q && varlen) return SAGE_ERR_UNSUPPORTED;
   if (max_seqlen > (1 << 24) || nseq > (1 << 20) || Hq > 4096) return SAGE_ERR_UNSUPPORTED;
   const long long tps = cdiv(max_seqlen, kTile);
@@ -60,12 +60,15 @@ sage_status_t plan(int nseq, int total_q, int total_k, int max_seqlen, int Hq, i
   L->err = take(256, 256);
   L->tile_off_q = take(varlen ? sizeof(int) * (nseq + 1) : 0, 256);
   L->tile_off_k = take(varlen ? sizeof(int) * (nseq + 1) : 0, 256);
-  // k_stat and v_stat are contiguous: one memset zeroes them before each
-  // pre-pass
+  // k_stat, v_sum and v_stat are contiguous: one memset zeroes them before
+  // each pre-pass.  v_stat: per channel two uint32 (|max| bits; smooth V:
+  // order-preserving keys of the maximum and of the negated minimum).
   L->k_stat = take(nd * 8, 256);
-  L->v_stat = take(nd * 4, 4);
+  L->v_sum = take(nd * 8, 8);
+  L->v_stat = take(nd * 8, 8);
   L->k_mean = take(nd * 4, 256);
   L->v_scale = take(nd * 4, 256);
+  L->v_mean = take(nd * 4, 256);
   L->k_codes = take((size_t)Hkv * tk * kTile * D, 1024);
   L->k_scale = take((size_t)Hkv * tk * kKGroupsMax * 4, 256);
   // sized for 16-bit V in both modes, so every region's offset is the same
@@ -93,7 +96,7 @@ sage_status_t check_common(sage_dtype_t dtype, int D, sage_gran_t gran, sage_pv_
   if (dtype != SAGE_F16 && dtype != SAGE_BF16) return SAGE_ERR_INVALID_ARG;
   if (gran != SAGE_PER_BLOCK && gran != SAGE_PER_WARP && gran != SAGE_PER_THREAD && gran != SAGE_PER_TOKEN)
     return SAGE_ERR_INVALID_ARG;
-  if (pv != SAGE_PV_FP8 && pv != SAGE_PV_FP16) return SAGE_ERR_INVALID_ARG;
+  if (pv != SAGE_PV_FP8 && pv != SAGE_PV_FP16 && pv != SAGE_PV_FP8_SMOOTH_V) return SAGE_ERR_INVALID_ARG;
   if (acc != SAGE_ACC_FP32 && acc != SAGE_ACC_FP32_FP32) return SAGE_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return SAGE_ERR_UNSUPPORTED;
   return SAGE_OK;
@@ -101,7 +104,7 @@ sage_status_t check_common(sage_dtype_t dtype, int D, sage_gran_t gran, sage_pv_
 
 // Bytes of the pre-pass accumulators k_stat .. v_stat (zeroed per pre-pass).
 size_t stats_zero_bytes(const sage_ws_layout_t& L, int nseq, int Hkv, int D) {
-  return L.v_stat + 4 * (size_t)nseq * Hkv * D - L.k_stat;
+  return L.v_stat + 8 * (size_t)nseq * Hkv * D - L.k_stat;
 }
 
 // The pre-pass over any of Q, K, V (dense or varlen).
@@ -126,7 +129,8 @@ sage_status_t run_prepass(const void* q, const void* k, const void* v, int bf16,
   j.gran = gran;
   j.smooth_k = smooth_k ? 1 : 0;
   j.smooth_q = smooth_q ? 1 : 0;
-  j.pv8 = pv == SAGE_PV_FP8;
+  j.pv8 = pv != SAGE_PV_FP16;
+  j.smooth_v = pv == SAGE_PV_FP8_SMOOTH_V;
   j.do_q = q != nullptr;
   j.do_k = k != nullptr;
   j.do_v = v != nullptr;
@@ -135,6 +139,8 @@ sage_status_t run_prepass(const void* q, const void* k, const void* v, int bf16,
   j.err = at<uint32_t>(ws, L.err);
   j.k_stat = at<unsigned long long>(ws, L.k_stat);
   j.v_stat = at<uint32_t>(ws, L.v_stat);
+  j.v_sum = at<unsigned long long>(ws, L.v_sum);
+  j.v_mean = at<float>(ws, L.v_mean);
   j.k_mean = at<float>(ws, L.k_mean);
   j.v_scale = at<float>(ws, L.v_scale);
   j.q_codes = at<int8_t>(ws, L.q_codes);
@@ -178,7 +184,8 @@ sage_status_t run_attn(void* out, int bf16, Strides so, const Seqs& seqs, int ns
   p.gran = gran;
   p.causal = causal ? 1 : 0;
   p.out_bf16 = bf16;
-  return cuda_status(attn_forward(p, D, pv == SAGE_PV_FP8, acc == SAGE_ACC_FP32_FP32, seqs.max_seqlen, nseq, s));
+  p.v_mean = pv == SAGE_PV_FP8_SMOOTH_V ? at<float>(w, L.v_mean) : nullptr;
+  return cuda_status(attn_forward(p, D, pv != SAGE_PV_FP16, acc == SAGE_ACC_FP32_FP32, seqs.max_seqlen, nseq, s));
 }
 
 Seqs dense_seqs(int S) {

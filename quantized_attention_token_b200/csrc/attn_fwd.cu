@@ -228,7 +228,8 @@ __device__ __forceinline__ float tile_exp_store(const uint32_t (&r)[128], const 
 // 448 * P~ and O sums P8 * V8, so the 448 cancels); 16-bit rounding, one row.
 template <int D, bool PV8, bool FROM_REGS>
 __device__ __forceinline__ void store_row(uint16_t* orow, uint32_t ob, const float* oacc, float inv_l,
-                                          const float* vsc, bool bf16, bool have_o, bool valid) {
+                                          const float* vsc, const float* vmu, bool bf16, bool have_o,
+                                          bool valid) {
 #pragma unroll
   for (int ch = 0; ch < D / 32; ++ch) {
     float o[32];
@@ -251,6 +252,10 @@ __device__ __forceinline__ void store_row(uint16_t* orow, uint32_t ob, const flo
       if (PV8) {
         a *= __ldg(vsc + ch * 32 + 2 * k);
         bb *= __ldg(vsc + ch * 32 + 2 * k + 1);
+        if (vmu) {                                   // smooth V: the channel mean comes back
+          a += __ldg(vmu + ch * 32 + 2 * k);
+          bb += __ldg(vmu + ch * 32 + 2 * k + 1);
+        }
       }
       w[k] = bf16 ? pack_bf16x2(a, bb) : pack_f16x2(a, bb);
     }
@@ -267,7 +272,7 @@ __device__ __forceinline__ void store_row(uint16_t* orow, uint32_t ob, const flo
 template <int D, bool PV8, bool ACC2, bool KPT, bool BF16P, bool SMQ>
 __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, uint32_t tmem, int warp, int tid,
                                              int pair, int b, int h, int hk, int qs, int Lq, int Lk, int tq0,
-                                             int tk0, const int* n, const float* vsc) {
+                                             int tk0, const int* n, const float* vsc, const float* vmu) {
   using C = AttnCfg<D, PV8, ACC2>;
   constexpr int NQ = C::NQ;
   auto bar = [&](int i) -> uint32_t { return sb + C::OFF_BAR + 8 * i; };
@@ -423,7 +428,7 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
     if (ok) {
       uint16_t* orow = reinterpret_cast<uint16_t*>(p.out) + (long long)b * p.os.sb + (long long)h * p.os.sh +
                        (long long)(qs + row) * p.os.ss;
-      store_row<D, PV8, false>(orow, ob, nullptr, l > 0.f ? 1.0f / l : 0.f, vsc, bf16, n[q] > 0, row < Lq);
+      store_row<D, PV8, false>(orow, ob, nullptr, l > 0.f ? 1.0f / l : 0.f, vsc, vmu, bf16, n[q] > 0, row < Lq);
     }
   }
 }
@@ -486,6 +491,7 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
   tc_fence_after();
   const uint32_t tmem = misc[0];
   const float* vsc = p.v_scale + ((size_t)b * p.Hkv + hk) * D;
+  const float* vmu = p.v_mean ? p.v_mean + ((size_t)b * p.Hkv + hk) * D : nullptr;
 
   if (warp == 0) {
     // ------------------------------------------------------------ loader
@@ -620,7 +626,7 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
     const bool bf16p = !PV8 && p.out_bf16;
     const int variant = (p.gran == 2 ? 4 : 0) + (bf16p ? 2 : 0) + (p.q_bias ? 1 : 0);
 #define SAGE_SOFTMAX(KPT, BF16P, SMQ) \
-  softmax_role<D, PV8, ACC2, KPT, BF16P, SMQ>(p, sb, tmem, warp, tid, pair, b, h, hk, qs, Lq, Lk, tq0, tk0, n, vsc)
+  softmax_role<D, PV8, ACC2, KPT, BF16P, SMQ>(p, sb, tmem, warp, tid, pair, b, h, hk, qs, Lq, Lk, tq0, tk0, n, vsc, vmu)
     switch (variant) {
       case 0: SAGE_SOFTMAX(false, false, false); break;
       case 1: SAGE_SOFTMAX(false, false, true); break;
@@ -671,7 +677,8 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
       if (ok) {
         uint16_t* orow = reinterpret_cast<uint16_t*>(p.out) + (long long)b * p.os.sb + (long long)h * p.os.sh +
                          (long long)(qs + row) * p.os.ss;
-        store_row<D, PV8, true>(orow, ob, oacc, l > 0.f ? 1.0f / l : 0.f, vsc, p.out_bf16 != 0, true, row < Lq);
+        store_row<D, PV8, true>(orow, ob, oacc, l > 0.f ? 1.0f / l : 0.f, vsc, vmu, p.out_bf16 != 0, true,
+                                row < Lq);
       }
     }
   }

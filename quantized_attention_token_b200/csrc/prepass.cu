@@ -132,11 +132,22 @@ template <int D>
 struct StatSmem {
   double sum[Map<D>::WARPS][D];
   uint32_t amax[Map<D>::WARPS][D];
+  uint32_t kneg[Map<D>::WARPS][D];   // smooth V: keys of the negated values
 };
+
+// Order-preserving 16-bit key of a finite fp16 / bf16 bit pattern (larger
+// value, larger key) and its inverse.
+__device__ __forceinline__ uint32_t key16(uint16_t h) {
+  return (h & 0x8000u) ? (~(uint32_t)h & 0xFFFFu) : ((uint32_t)h | 0x8000u);
+}
+__device__ __forceinline__ uint16_t unkey16(uint32_t k) {
+  return (k & 0x8000u) ? (uint16_t)(k ^ 0x8000u) : (uint16_t)(~k & 0xFFFFu);
+}
 template <int D>
 struct VSmem {
   uint32_t tile[kTile * D / 2];   // the 16-bit tile, row-major, two values per word
   float inv[D];                   // 448 / channel amax (FP8 mode)
+  float mu[D];                    // channel mean (smooth V), else 0
 };
 
 // Sum or max of a per-lane value over the lanes of a warp that own the same
@@ -298,28 +309,72 @@ __device__ void kstat_tile(const PrepassJob& j, int h, const TileLoc& L, StatSme
 }
 
 // Channel |max| of a V tile (|x| bit patterns of 16-bit floats order like the
-// values).
-template <int D, bool BF16>
+// values).  Smooth V: the exact channel sums (as for K) and the keys of the
+// channel maximum and of the negated minimum, from which launch B gets the
+// mean and |max| of V - mean: float32 subtraction of a fixed mean is monotone,
+// so that |max| comes from the two extremes.
+template <int D, bool BF16, bool SMOOTH>
 __device__ void vstat_tile(const PrepassJob& j, int h, const TileLoc& L, StatSmem<D>& sm) {
   using M = Map<D>;
-  const int tid = threadIdx.x, cc = tid % M::TPR, warp = tid >> 5, lane = tid & 31;
+  const int tid = threadIdx.x, cc = tid % M::TPR, rg = tid / M::TPR, warp = tid >> 5, lane = tid & 31;
   const uint16_t* head = j.v + (long long)L.b * j.sv.sb + (long long)h * j.sv.sh;
   uint4 v[M::NR];
   load_tile<D, false>(head, j.sv.ss, L, v);
+  const size_t o = ((size_t)L.b * j.Hkv + h) * D;
+  if (!SMOOTH) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      uint32_t a = 0;
+#pragma unroll
+      for (int i = 0; i < M::NR; ++i) a = max(a, (uint32_t)(h16(v[i], u) & 0x7FFF));
+      a = reduce_same_chunk<D>(a, [](uint32_t x, uint32_t y) { return max(x, y); });
+      if (lane < M::TPR) sm.amax[warp][cc * 8 + u] = a;
+    }
+    __syncthreads();
+    if (tid < D) {
+      uint32_t m = 0;
+#pragma unroll
+      for (int w = 0; w < M::WARPS; ++w) m = max(m, sm.amax[w][tid]);
+      atomicMax(&j.v_stat[2 * (o + tid)], __float_as_uint(h16_to_f32((uint16_t)m, BF16)));
+    }
+    return;
+  }
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
-    uint32_t a = 0;
+    double a = 0.0;
+    uint32_t kmax = 0, kneg = 0;
 #pragma unroll
-    for (int i = 0; i < M::NR; ++i) a = max(a, (uint32_t)(h16(v[i], u) & 0x7FFF));
-    a = reduce_same_chunk<D>(a, [](uint32_t x, uint32_t y) { return max(x, y); });
-    if (lane < M::TPR) sm.amax[warp][cc * 8 + u] = a;
+    for (int i = 0; i < M::NR; ++i) {
+      const uint16_t x = h16(v[i], u);
+      a += (double)h16_to_f32(x, BF16);                 // rows past the sequence hold 0
+      if (rg * M::NR + i < L.nvalid) {
+        kmax = max(kmax, key16(x));
+        kneg = max(kneg, key16(x ^ 0x8000u));
+      }
+    }
+    a = reduce_same_chunk<D>(a, [](double x, double y) { return x + y; });
+    kmax = reduce_same_chunk<D>(kmax, [](uint32_t x, uint32_t y) { return max(x, y); });
+    kneg = reduce_same_chunk<D>(kneg, [](uint32_t x, uint32_t y) { return max(x, y); });
+    if (lane < M::TPR) {
+      sm.sum[warp][cc * 8 + u] = a;
+      sm.amax[warp][cc * 8 + u] = kmax;
+      sm.kneg[warp][cc * 8 + u] = kneg;
+    }
   }
   __syncthreads();
   if (tid < D) {
-    uint32_t m = 0;
+    double sum = 0.0;
+    uint32_t kmax = 0, kneg = 0;
 #pragma unroll
-    for (int w = 0; w < M::WARPS; ++w) m = max(m, sm.amax[w][tid]);
-    atomicMax(&j.v_stat[((size_t)L.b * j.Hkv + h) * D + tid], __float_as_uint(h16_to_f32((uint16_t)m, BF16)));
+    for (int w = 0; w < M::WARPS; ++w) {
+      sum += sm.sum[w][tid];
+      kmax = max(kmax, sm.amax[w][tid]);
+      kneg = max(kneg, sm.kneg[w][tid]);
+    }
+    if (BF16) atomicAdd(reinterpret_cast<double*>(&j.v_sum[o + tid]), sum);
+    else atomicAdd(&j.v_sum[o + tid], (unsigned long long)(long long)(sum * 0x1p24));
+    atomicMax(&j.v_stat[2 * (o + tid)], kmax);
+    atomicMax(&j.v_stat[2 * (o + tid) + 1], kneg);
   }
 }
 
@@ -327,7 +382,7 @@ __device__ void vstat_tile(const PrepassJob& j, int h, const TileLoc& L, StatSme
 // V written transposed: FP8 rows of 128 keys, or 16-bit rows split in two
 // 64-key halves.  The tile is staged in shared memory; each output unit
 // gathers two adjacent channels (one 32-bit word per key).
-template <int D, bool BF16>
+template <int D, bool BF16, bool SMOOTH>
 __device__ void v_tile(const PrepassJob& j, int h, int t, const TileLoc& L, VSmem<D>& sm) {
   using M = Map<D>;
   const int tid = threadIdx.x, cc = tid % M::TPR, rg = tid / M::TPR;
@@ -335,9 +390,23 @@ __device__ void v_tile(const PrepassJob& j, int h, int t, const TileLoc& L, VSme
   uint4 v[M::NR];
   load_tile<D, true>(head, j.sv.ss, L, v);
   if (j.pv8 && tid < D) {
-    const float am = __uint_as_float(__ldcg(&j.v_stat[((size_t)L.b * j.Hkv + h) * D + tid]));
+    const size_t o = ((size_t)L.b * j.Hkv + h) * D + tid;
+    float am, mu = 0.f;
+    if (SMOOTH) {
+      // the channel mean from the exact sum, then |max| of V - mean
+      const unsigned long long w = __ldcg(&j.v_sum[o]);
+      const double sum = BF16 ? __longlong_as_double((long long)w) : (double)(long long)w * 0x1p-24;
+      mu = (float)(sum / (double)L.len);
+      const float vmax = h16_to_f32(unkey16(__ldcg(&j.v_stat[2 * o])), BF16);
+      const float vmin = -h16_to_f32(unkey16(__ldcg(&j.v_stat[2 * o + 1])), BF16);
+      am = fmaxf(fabsf(__fsub_rn(vmax, mu)), fabsf(__fsub_rn(vmin, mu)));
+      if (L.tile == 0) j.v_mean[o] = mu;
+    } else {
+      am = __uint_as_float(__ldcg(&j.v_stat[2 * o]));
+    }
+    sm.mu[tid] = mu;
     sm.inv[tid] = am > 0.f ? __fdiv_rn(kFp8Max, am) : 0.f;
-    if (L.tile == 0) j.v_scale[((size_t)L.b * j.Hkv + h) * D + tid] = __fdiv_rn(am, kFp8Max);
+    if (L.tile == 0) j.v_scale[o] = __fdiv_rn(am, kFp8Max);
   }
 #pragma unroll
   for (int i = 0; i < M::NR; ++i)
@@ -349,15 +418,24 @@ __device__ void v_tile(const PrepassJob& j, int h, int t, const TileLoc& L, VSme
     for (int w = tid; w < (D / 2) * 8; w += kPrepassThreads) {
       const int p = w % (D / 2), k = w / (D / 2);
       const float i0 = sm.inv[2 * p], i1 = sm.inv[2 * p + 1];
+      const float m0 = SMOOTH ? sm.mu[2 * p] : 0.f, m1 = SMOOTH ? sm.mu[2 * p + 1] : 0.f;
       uint32_t o0[4], o1[4];
 #pragma unroll
       for (int q4 = 0; q4 < 4; ++q4) {
         float f0[4], f1[4];
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const uint32_t x = sm.tile[(16 * k + 4 * q4 + e) * (D / 2) + p];
-          f0[e] = __fmul_rn(h16_to_f32((uint16_t)(x & 0xFFFF), BF16), i0);
-          f1[e] = __fmul_rn(h16_to_f32((uint16_t)(x >> 16), BF16), i1);
+          const int key = 16 * k + 4 * q4 + e;
+          const uint32_t x = sm.tile[key * (D / 2) + p];
+          const float x0 = h16_to_f32((uint16_t)(x & 0xFFFF), BF16), x1 = h16_to_f32((uint16_t)(x >> 16), BF16);
+          if (SMOOTH) {        // (V - mean) * 448 / |max|; keys past the sequence stay 0
+            const bool in = key < L.nvalid;
+            f0[e] = in ? __fmul_rn(__fsub_rn(x0, m0), i0) : 0.f;
+            f1[e] = in ? __fmul_rn(__fsub_rn(x1, m1), i1) : 0.f;
+          } else {             // rows past the sequence hold 0
+            f0[e] = __fmul_rn(x0, i0);
+            f1[e] = __fmul_rn(x1, i1);
+          }
         }
         o0[q4] = pack_e4m3x4(f0[0], f0[1], f0[2], f0[3]);
         o1[q4] = pack_e4m3x4(f1[0], f1[1], f1[2], f1[3]);
@@ -388,7 +466,7 @@ __device__ void v_tile(const PrepassJob& j, int h, int t, const TileLoc& L, VSme
 // ---------------------------------------------------------------- kernels
 // Launch A: blockIdx.x = tile slot, blockIdx.y over [Q heads | K-statistics
 // heads | V-statistics heads] (each part present only when asked for).
-template <int D, bool BF16>
+template <int D, bool BF16, bool SV>
 __global__ void __launch_bounds__(kPrepassThreads, 3) prepass_a_kernel(const PrepassJob j) {
   __shared__ union {
     QuantSmem<D> q;
@@ -405,13 +483,13 @@ __global__ void __launch_bounds__(kPrepassThreads, 3) prepass_a_kernel(const Pre
     if (t < j.tiles_k && locate(j, false, t, L)) kstat_tile<D, BF16>(j, y, L, sm.s);
   } else {
     y -= nks;
-    if (t < j.tiles_k && locate(j, false, t, L)) vstat_tile<D, BF16>(j, y, L, sm.s);
+    if (t < j.tiles_k && locate(j, false, t, L)) vstat_tile<D, BF16, SV>(j, y, L, sm.s);
   }
 }
 
 // Launch B: blockIdx.y over [K heads | V heads], both axes walked backwards
 // (the last V head's last tile first).
-template <int D, bool BF16>
+template <int D, bool BF16, bool SV>
 __global__ void __launch_bounds__(kPrepassThreads, 3) prepass_b_kernel(const PrepassJob j) {
   __shared__ union {
     QuantSmem<D> q;
@@ -423,7 +501,7 @@ __global__ void __launch_bounds__(kPrepassThreads, 3) prepass_b_kernel(const Pre
   TileLoc L;
   if (!locate(j, false, t, L)) return;
   if (y < nk) quant_tile<D, false, BF16>(j, y, t, L, sm.q);
-  else v_tile<D, BF16>(j, y - nk, t, L, sm.v);
+  else v_tile<D, BF16, SV>(j, y - nk, t, L, sm.v);
 }
 
 // ---------------------------------------------------------------- smooth-Q bias
@@ -483,20 +561,20 @@ __global__ void varlen_offsets_kernel(const int* cu_q, const int* cu_k, int n, i
 }
 
 // ---------------------------------------------------------------- launchers
-template <int D, bool BF16>
+template <int D, bool BF16, bool SV>
 static cudaError_t launch_prepass(const PrepassJob& j, cudaStream_t s) {
   const int nq = j.do_q ? j.Hq : 0;
   const int nks = (j.do_k && j.smooth_k) ? j.Hkv : 0;
   const int nvs = (j.do_v && j.pv8) ? j.Hkv : 0;
   const int xa = max(nq ? j.tiles_q : 0, (nks + nvs) ? j.tiles_k : 0);
   if (nq + nks + nvs > 0 && xa > 0) {
-    prepass_a_kernel<D, BF16><<<dim3(xa, nq + nks + nvs), kPrepassThreads, 0, s>>>(j);
+    prepass_a_kernel<D, BF16, SV><<<dim3(xa, nq + nks + nvs), kPrepassThreads, 0, s>>>(j);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
   const int nb = (j.do_k ? j.Hkv : 0) + (j.do_v ? j.Hkv : 0);
   if (nb > 0 && j.tiles_k > 0) {
-    prepass_b_kernel<D, BF16><<<dim3(j.tiles_k, nb), kPrepassThreads, 0, s>>>(j);
+    prepass_b_kernel<D, BF16, SV><<<dim3(j.tiles_k, nb), kPrepassThreads, 0, s>>>(j);
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
@@ -505,9 +583,14 @@ static cudaError_t launch_prepass(const PrepassJob& j, cudaStream_t s) {
   return cudaGetLastError();
 }
 
+template <bool SV>
+static cudaError_t prepass_dispatch(const PrepassJob& j, int D, cudaStream_t s) {
+  if (D == 128) return j.bf16 ? launch_prepass<128, true, SV>(j, s) : launch_prepass<128, false, SV>(j, s);
+  return j.bf16 ? launch_prepass<64, true, SV>(j, s) : launch_prepass<64, false, SV>(j, s);
+}
+
 cudaError_t prepass_run(const PrepassJob& j, int D, cudaStream_t s) {
-  if (D == 128) return j.bf16 ? launch_prepass<128, true>(j, s) : launch_prepass<128, false>(j, s);
-  return j.bf16 ? launch_prepass<64, true>(j, s) : launch_prepass<64, false>(j, s);
+  return j.smooth_v ? prepass_dispatch<true>(j, D, s) : prepass_dispatch<false>(j, D, s);
 }
 
 cudaError_t prepass_varlen_offsets(const int* cu_q, const int* cu_k, int n, int max_seqlen, int cap_q, int cap_k,

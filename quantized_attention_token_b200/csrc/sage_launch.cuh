@@ -15,12 +15,15 @@ struct PrepassJob {
   Strides sq{}, sk{}, sv{};
   Seqs seqs;
   int nseq = 0, Hq = 0, Hkv = 0, group = 1;
-  int bf16 = 0, gran = 0, smooth_k = 0, smooth_q = 0, pv8 = 1;
+  int bf16 = 0, gran = 0, smooth_k = 0, smooth_q = 0, pv8 = 1, smooth_v = 0;
   int do_q = 0, do_k = 0, do_v = 0;
   int tiles_q = 0, tiles_k = 0;    // workspace tiles per head
   uint32_t* err = nullptr;
   unsigned long long* k_stat = nullptr;   // [nseq][Hkv][D] int64 (fp16) / fp64 bits (bf16) channel sums
-  uint32_t* v_stat = nullptr;             // [nseq][Hkv][D] float bits of channel |max|
+  uint32_t* v_stat = nullptr;             // [nseq][Hkv][D][2]: float bits of channel |max|;
+                                          // smooth V: keys of the max and of the negated min
+  unsigned long long* v_sum = nullptr;    // [nseq][Hkv][D] channel sums of V (smooth V), like k_stat
+  float* v_mean = nullptr;                // [nseq][Hkv][D] (smooth V)
   float* k_mean = nullptr;                // [nseq][Hkv][D]
   float* v_scale = nullptr;               // [nseq][Hkv][D]
   int8_t* q_codes = nullptr;
@@ -39,6 +42,7 @@ struct AttnParams {
   const float* k_scale;
   const uint8_t* v_codes;
   const float* v_scale;
+  const float* v_mean;       // smooth V: per-channel mean added to the output, else null
   uint32_t* err;
   Seqs seqs;
   int Hq, Hkv, group;

@@ -137,6 +137,34 @@ def test_prepass_smooth_q_bit_exact(D, S, gran, dtype, layout):
             assert np.array_equal(qb[h, sl, :S], ref), (b, h)
 
 
+@pytest.mark.parametrize("D,S,dtype,layout", [(128, 300, "fp16", "HND"), (64, 517, "bf16", "NHD")])
+def test_prepass_smooth_v_bit_exact(D, S, dtype, layout):
+    """Smooth V: channel mean (exact sum), E4M3 codes of V - mean and the
+    scales, against the oracle; keys past the sequence stay 0."""
+    Hq, Hkv, B = 2, 2, 2
+    sp = synth.Spec("t", Hq=Hq, Hkv=Hkv, D=D, B=B, S=S, dtype=dtype, layout=layout, seed=36)
+    q, k, v = synth.make(sp)
+    v = v + torch.from_numpy(np.random.default_rng(7).normal(0, 8, D).astype(np.float32)).to(v.dtype)
+    ws = torch.zeros(sage.sage_workspace_bytes(B, Hq, Hkv, S, D, 2, 0), dtype=torch.uint8, device="cuda")
+    sage.quant_v(_dev(v), ws, layout, "fp8_smooth_v")
+    assert sage.get_device_error(ws) == (0, 0)
+    L = sage.workspace_layout(B, B * S, B * S, S, Hq, Hkv, D, pv=2)
+    W = _ws_bytes(ws)
+    tps = (S + 127) // 128
+    v8 = wsdecode.v_fp8(W, L, Hkv, L["tiles_k"], D)
+    vs = wsdecode.f32(W, L, "v_scale", B * Hkv * D).reshape(B, Hkv, D)
+    vm = wsdecode.f32(W, L, "v_mean", B * Hkv * D).reshape(B, Hkv, D)
+    pb = oracle.problem(q, k, v, layout)
+    for b in range(B):
+        for h in range(Hkv):
+            rv = oracle.quant_v(pb.v[b][h], smooth=True, is_fp16=dtype == "fp16")
+            g = v8[h, b * tps:(b + 1) * tps].reshape(-1, D)
+            assert np.array_equal(vm[b, h], rv.mu), (b, h)
+            assert np.array_equal(vs[b, h], rv.scales), (b, h)
+            assert np.array_equal(g[:S], rv.codes), (b, h)
+            assert np.all(g[S:] == 0)
+
+
 def test_prepass_v16_layout():
     sp = synth.Spec("t", Hq=2, Hkv=2, D=128, B=1, S=200, dtype="bf16", seed=32)
     q, k, v = synth.make(sp)
@@ -223,6 +251,41 @@ def test_attention_smooth_q_matches_oracle(D, S, causal, gran, pv, acc, dtype, l
     o = out.double().cpu().numpy().ravel()
     cos = o @ ex.ravel() / (np.linalg.norm(o) * np.linalg.norm(ex))
     assert cos >= 0.999, cos
+
+
+@pytest.mark.parametrize("D,S,causal,acc,dtype,layout", [
+    (128, 384, False, "fp32", "fp16", "HND"),
+    (128, 300, True, "fp32+fp32", "bf16", "NHD"),
+    (64, 257, False, "fp32", "bf16", "HND"),
+])
+def test_attention_smooth_v_matches_oracle(D, S, causal, acc, dtype, layout):
+    """Smooth V on inputs whose V carries large per-channel offsets."""
+    sp = synth.Spec("t", Hq=4, Hkv=2, D=D, B=2, S=S, dtype=dtype, layout=layout, causal=causal, k_bias_std=3.0,
+                    seed=80 + S)
+    q, k, v = synth.make(sp)
+    v = v + torch.from_numpy(np.random.default_rng(8).normal(0, 8, D).astype(np.float32)).to(v.dtype)
+    out = sage.sageattn(_dev(q), _dev(k), _dev(v), layout, causal, pv_dtype="fp8", pv_accum_dtype=acc,
+                        smooth_v=True)
+    torch.cuda.synchronize()
+    ref = oracle.attention(q, k, v, layout, causal, pv="fp8", smooth_v=True, with_allowance=True)
+    _assert_close(out, ref, dtype, "smooth V vs oracle")
+    ex = oracle.attention_exact(q, k, v, layout, causal)
+    o = out.double().cpu().numpy().ravel()
+    cos = o @ ex.ravel() / (np.linalg.norm(o) * np.linalg.norm(ex))
+    assert cos >= 0.999, cos
+
+
+def test_varlen_smooth_v_matches_oracle():
+    sp = synth.Spec("t", Hq=4, Hkv=2, D=128, seqlens=[200, 77, 512], causal=True, seed=90)
+    q, k, v = synth.make(sp)
+    v = v + torch.from_numpy(np.random.default_rng(9).normal(0, 8, 128).astype(np.float32)).to(v.dtype)
+    cu = sp.cu_seqlens()
+    cu_d = torch.from_numpy(cu).cuda()
+    out = sage.sageattn_varlen(_dev(q), _dev(k), _dev(v), cu_d, cu_d, max(sp.seqlens), True, pv_dtype="fp8",
+                               pv_accum_dtype="fp32", smooth_v=True)
+    torch.cuda.synchronize()
+    ref = oracle.attention(q, k, v, causal=True, pv="fp8", smooth_v=True, cu_seqlens=cu, with_allowance=True)
+    _assert_close(out, ref, "fp16", "varlen smooth V vs oracle")
 
 
 def test_tiny_config():
