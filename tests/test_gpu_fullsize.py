@@ -13,7 +13,7 @@ from tests.test_gpu_parity import _assert_close
 pytestmark = pytest.mark.gpu
 
 
-def _oracle_rows(spec, q, k, v, b, h, rows, gran, pv):
+def _oracle_rows(spec, q, k, v, b, h, rows, gran, pv, smooth_q=False, smooth_v=False):
     """Oracle output and allowance for rows [r0, r1) of (sequence b, head h),
     computed on that sequence / head alone."""
     grp = spec.Hq // spec.Hkv
@@ -30,7 +30,7 @@ def _oracle_rows(spec, q, k, v, b, h, rows, gran, pv):
         qs, ks, vs = q[b:b + 1, :, h:h + 1], k[b:b + 1, :, hk:hk + 1], v[b:b + 1, :, hk:hk + 1]
         lay = "NHD"
     out, allow = oracle.attention(qs, ks, vs, lay, spec.causal, gran=gran, pv=pv, q_rows={(0, 0): rows},
-                                  with_allowance=True)
+                                  smooth_q=smooth_q, smooth_v=smooth_v, with_allowance=True)
     sel = (slice(0, 1), slice(0, 1), slice(*rows)) if lay == "HND" else (slice(0, 1), slice(*rows), slice(0, 1))
     pb = oracle.problem(qs, ks, vs, lay)
     ex = oracle.attn_exact_head(pb.q[0][0][rows[0]:rows[1]], pb.k[0][0], pb.v[0][0], spec.causal,
@@ -47,26 +47,26 @@ def _gpu_rows(spec, out, b, h, rows):
     return out[b, rows[0]:rows[1], h]
 
 
-def _run(spec, gran="per_block", pv="fp8", acc="fp32+fp32"):
+def _run(spec, gran="per_block", pv="fp8", acc="fp32+fp32", smooth_q=False, smooth_v=False):
     q, k, v = synth.make(spec)
     qd, kd, vd = (t.cuda() for t in (q, k, v))
     if spec.varlen:
         cu = torch.from_numpy(spec.cu_seqlens()).cuda()
         out = sage.sageattn_varlen(qd, kd, vd, cu, cu, max(spec.seqlens), spec.causal, qk_quant_gran=gran,
-                                   pv_dtype=pv, pv_accum_dtype=acc)
+                                   pv_dtype=pv, pv_accum_dtype=acc, smooth_v=smooth_v)
     else:
         out = sage.sageattn(qd, kd, vd, spec.layout, spec.causal, qk_quant_gran=gran, pv_dtype=pv,
-                            pv_accum_dtype=acc)
+                            pv_accum_dtype=acc, smooth_q=smooth_q, smooth_v=smooth_v)
     torch.cuda.synchronize()
     ws = sage.Workspace._cache[0]
     assert sage.get_device_error(ws) == (0, 0)
     return q, k, v, out.cpu()
 
 
-def _check(spec, samples, gran="per_block", pv="fp8", acc="fp32+fp32"):
-    q, k, v, out = _run(spec, gran, pv, acc)
+def _check(spec, samples, gran="per_block", pv="fp8", acc="fp32+fp32", smooth_q=False, smooth_v=False):
+    q, k, v, out = _run(spec, gran, pv, acc, smooth_q, smooth_v)
     for b, h, rows in samples:
-        ref, allow, ex = _oracle_rows(spec, q, k, v, b, h, rows, gran, pv)
+        ref, allow, ex = _oracle_rows(spec, q, k, v, b, h, rows, gran, pv, smooth_q, smooth_v)
         got = _gpu_rows(spec, out, b, h, rows)
         _assert_close(got, (ref, allow), spec.dtype, f"{spec.name} b{b} h{h} rows{rows}")
         o = got.double().numpy().ravel()
@@ -96,3 +96,20 @@ def test_sweep_points(name, gran):
     spec = synth.CONFIGS[name]
     last = spec.S - 128
     _check(spec, [(0, 0, (0, 128)), (spec.B - 1, 31, (last, spec.S))], gran=gran)
+
+
+def test_b2_h32_s4096_d128_per_token():
+    spec = synth.CONFIGS["b2_h32_s4096_d128"]
+    _check(spec, [(0, 3, (0, 128)), (1, 30, (2048, 2176))], gran="per_token", acc="fp32")
+
+
+def test_video_dit_smooth_q_and_v():
+    """The video-DiT workload (Q with per-block offsets) with both smoothing
+    options of the method on."""
+    spec = synth.CONFIGS["video_dit"]
+    _check(spec, [(0, 2, (0, 128)), (0, 11, (20480, 20608))], acc="fp32", smooth_q=True, smooth_v=True)
+
+
+def test_varlen_gqa_smooth_v():
+    spec = synth.CONFIGS["varlen_gqa"]
+    _check(spec, [(2, 5, (7040, 7168)), (3, 16, (8192, 8320))], acc="fp32", smooth_v=True)
