@@ -58,8 +58,8 @@ def lib():
             "orc_scores_int32": (None, [P, P, i64, i64, i32, P]),
             "orc_smooth_q_bias": (None, [P, i64, P, P, i64, i32, P]),
             "orc_attn_quant_head": (None, [P, P, P, P, P, P, P, i32, i32, P, i64, i64, i32,
-                                           i32, f32, i64, i64, P, P]),
-            "orc_attn_tiled_fp64_head": (None, [P, P, P, i64, i64, i32, i32, f64, P]),
+                                           i32, f32, i64, i64, P, P, i32]),
+            "orc_attn_tiled_fp64_head": (None, [P, P, P, i64, i64, i32, i32, f64, P, i32]),
             "orc_attn_exact_head": (None, [P, P, P, i64, i64, i32, i32, f64, i64, P]),
         }
         for name, (res, args) in sig.items():
@@ -245,7 +245,7 @@ def smooth_q_bias(qq: QuantQ, kq: QuantK) -> np.ndarray:
 def attn_head(qq: QuantQ, kq: QuantK, vq: Optional[QuantV], v16: Optional[np.ndarray],
               pv: str, v_is_bf16: bool, causal: bool, sm_scale: float,
               rows: Optional[Tuple[int, int]] = None, bias: Optional[np.ndarray] = None,
-              allow: Optional[np.ndarray] = None) -> np.ndarray:
+              allow: Optional[np.ndarray] = None, lazy_tau: int = 0) -> np.ndarray:
     Lq, D = qq.codes.shape
     Lk = kq.codes.shape[0]
     r0, r1 = rows if rows is not None else (0, Lq)
@@ -254,7 +254,7 @@ def attn_head(qq: QuantQ, kq: QuantK, vq: Optional[QuantV], v16: Optional[np.nda
         _p(qq.codes), _p(qq.row_scales), _p(kq.codes), _p(kq.row_scales),
         _p(vq.codes) if vq is not None else None, _p(vq.scales) if vq is not None else None,
         _p(v16), PV[pv], int(v_is_bf16), _p(bias), Lq, Lk, D, int(causal),
-        ctypes.c_float(sm_scale), r0, r1, _p(out), _p(allow))
+        ctypes.c_float(sm_scale), r0, r1, _p(out), _p(allow), int(lazy_tau))
     if vq is not None and vq.mu is not None:
         out[r0:r1] += vq.mu.astype(np.float64)      # smooth V: the mean comes back
     return out
@@ -268,10 +268,10 @@ def attn_exact_head(q, k, v, causal, sm_scale, row_offset: int = 0) -> np.ndarra
     return out
 
 
-def attn_tiled_fp64_head(q, k, v, causal, sm_scale) -> np.ndarray:
+def attn_tiled_fp64_head(q, k, v, causal, sm_scale, lazy_tau: int = 0) -> np.ndarray:
     out = np.zeros(q.shape, dtype=np.float64)
     lib().orc_attn_tiled_fp64_head(_p(q), _p(k), _p(v), q.shape[0], k.shape[0], q.shape[1],
-                                   int(causal), float(sm_scale), _p(out))
+                                   int(causal), float(sm_scale), _p(out), int(lazy_tau))
     return out
 
 
@@ -312,7 +312,7 @@ def quantize(pb: Problem, gran: str = "per_block", smooth_k: bool = True, smooth
 def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout: str = "HND",
               causal: bool = False, sm_scale: Optional[float] = None, gran: str = "per_block",
               pv: str = "fp8", smooth_k: bool = True, smooth_q: bool = False,
-              cu_seqlens: Optional[np.ndarray] = None, smooth_v: bool = False,
+              cu_seqlens: Optional[np.ndarray] = None, smooth_v: bool = False, lazy_tau: int = 0,
               q_rows: Optional[Dict[Tuple[int, int], Tuple[int, int]]] = None,
               heads: Optional[List[Tuple[int, int]]] = None, with_allowance: bool = False):
     """The quantized forward pass; returns fp64 output shaped like q.
@@ -343,7 +343,7 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout: str = "
             rows = q_rows.get((b, h)) if q_rows else None
             row.append(attn_head(qq, kq[hk], vq[hk], pb.v[b][hk] if pv != "fp8" else None, pv,
                                  not pb.is_fp16, causal, scale, rows, bias,
-                                 al if with_allowance else None))
+                                 al if with_allowance else None, lazy_tau))
         outs.append(row)
         allows.append(arow)
     out = assemble(outs, q, layout, cu_seqlens)

@@ -379,6 +379,13 @@ ORC_EXPORT double orc_h16_alt_step(double p, int bf16) { return h16_alt_step(p, 
 /*                                                                          */
 /* Causal (reading): top-left aligned, key j visible to query i iff j <= i.  */
 /* Smooth Q: s_ij += bias[i/128][j] * float(sm_scale * log2 e).              */
+/* Conditional (lazy) rescaling, lazy_tau > 0 [reading of the NEXT item     */
+/* "skip the alpha update unless the maximum grows by more than tau"]: the  */
+/* reference r that P~ and O are kept relative to moves to the running      */
+/* maximum only when a tile's maximum exceeds float(r + tau); otherwise     */
+/* alpha = 1.  P~ = 2^(s - r) <= 2^tau, so the FP8 static scale becomes      */
+/* 448 * 2^-tau (P8 <= 448); the output divides it out again.  lazy_tau = 0 */
+/* is the plain online softmax above.                                       */
 /*                                                                          */
 /*   qc [Lq][D] int8, q_rs [Lq] row scales; kc [Lk][D], k_rs [Lk];           */
 /*   pv_mode 0: v8 [Lk][D] E4M3 codes, dv [D];                               */
@@ -395,8 +402,9 @@ ORC_EXPORT void orc_attn_quant_head(const int8_t* qc, const float* q_rs, const i
                                     const double* v16, int pv_mode, int v_is_bf16,
                                     const double* bias, int64_t Lq, int64_t Lk, int D,
                                     int causal, float sm_scale, int64_t row0, int64_t row1,
-                                    double* out, double* allow) {
+                                    double* out, double* allow, int lazy_tau) {
     const float sl2 = sm_scale * 1.44269504f;             /* float(log2 e) */
+    const double pscale = 448.0 * ldexp(1.0, -lazy_tau);  /* FP8 static P~ scale */
     int64_t ntile = (Lk + 127) / 128;
     #pragma omp parallel
     {
@@ -427,7 +435,8 @@ ORC_EXPORT void orc_attn_quant_head(const int8_t* qc, const float* q_rs, const i
                     s[j - j0] = sj;
                     if (sj > mt) mt = sj;
                 }
-                float mn = m > mt ? m : mt;
+                const int move = (m == -INFINITY) || (mt > m + (float)lazy_tau);
+                float mn = move ? (m > mt ? m : mt) : m;
                 double alpha = (m == -INFINITY) ? 0.0 : exp2((double)m - (double)mn);
                 double lt = 0.0;
                 for (int c = 0; c < D; ++c) Op[c] = Ap[c] = 0.0;
@@ -435,10 +444,10 @@ ORC_EXPORT void orc_attn_quant_head(const int8_t* qc, const float* q_rs, const i
                     double p = exp2((double)s[j - j0] - (double)mn);
                     lt += p;
                     if (pv_mode == 0) {
-                        double p8 = v8f[orc_e4m3_from_float((float)(p * 448.0))];
+                        double p8 = v8f[orc_e4m3_from_float((float)(p * pscale))];
                         const uint8_t* vr = v8 + j * D;
                         for (int c = 0; c < D; ++c) Op[c] += p8 * v8f[vr[c]];
-                        double st = allow ? e4m3_alt_step(p * 448.0) : 0.0;
+                        double st = allow ? e4m3_alt_step(p * pscale) : 0.0;
                         if (st > 0.0)
                             for (int c = 0; c < D; ++c) Ap[c] += st * fabs(v8f[vr[c]]);
                     } else {
@@ -460,12 +469,12 @@ ORC_EXPORT void orc_attn_quant_head(const int8_t* qc, const float* q_rs, const i
             for (int c = 0; c < D; ++c) {
                 double o;
                 if (l <= 0.0) o = 0.0;                     /* no visible key at all */
-                else if (pv_mode == 0) o = O[c] * (double)dv[c] / (448.0 * l);
+                else if (pv_mode == 0) o = O[c] * (double)dv[c] / (pscale * l);
                 else o = O[c] / l;
                 out[i * D + c] = o;
                 if (allow)
                     allow[i * D + c] = l <= 0.0 ? 0.0
-                                     : pv_mode == 0 ? A[c] * (double)dv[c] / (448.0 * l) : A[c] / l;
+                                     : pv_mode == 0 ? A[c] * (double)dv[c] / (pscale * l) : A[c] / l;
             }
         }
         free(O); free(Op); free(A); free(Ap); free(s); free(v8f);
@@ -482,7 +491,7 @@ ORC_EXPORT void orc_attn_quant_head(const int8_t* qc, const float* q_rs, const i
 /* ------------------------------------------------------------------------ */
 ORC_EXPORT void orc_attn_tiled_fp64_head(const double* q, const double* k, const double* v,
                                          int64_t Lq, int64_t Lk, int D, int causal,
-                                         double sm_scale, double* out) {
+                                         double sm_scale, double* out, int lazy_tau) {
     const double sl2 = sm_scale * 1.4426950408889634;
     int64_t ntile = (Lk + 127) / 128;
     #pragma omp parallel
@@ -504,7 +513,8 @@ ORC_EXPORT void orc_attn_tiled_fp64_head(const double* q, const double* k, const
                     s[j - j0] = d * sl2;
                     if (s[j - j0] > mt) mt = s[j - j0];
                 }
-                double mn = m > mt ? m : mt;
+                const int move = (m == -INFINITY) || (mt > m + (double)lazy_tau);
+                double mn = move ? (m > mt ? m : mt) : m;
                 double alpha = (m == -INFINITY) ? 0.0 : exp2(m - mn);
                 for (int c = 0; c < D; ++c) O[c] *= alpha;
                 l *= alpha;

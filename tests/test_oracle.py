@@ -502,3 +502,51 @@ def test_smooth_v_reduces_error_on_channel_offsets():
     e_plain = np.abs(plain - ex).mean()
     e_smooth = np.abs(smooth - ex).mean()
     assert e_smooth < 0.5 * e_plain, (e_smooth, e_plain)
+
+
+# ----------------------------------------------------------------------------- lazy rescaling
+@pytest.mark.parametrize("tau", [1, 2, 8, 1000])
+@pytest.mark.parametrize("causal", [False, True])
+def test_lazy_online_softmax_equals_exact(tau, causal):
+    """The conditional-rescaling bookkeeping (reference moves only when a
+    tile's maximum exceeds it by more than tau) is still exact softmax
+    attention in fp64, for any tau (1000: the reference never moves after
+    the first tile)."""
+    sp = synth.Spec("t", Hq=2, Hkv=2, D=64, B=1, S=333, causal=causal, k_bias_std=3.0, seed=13)
+    q, k, v = synth.make(sp)
+    pb = oracle.problem(q, k, v)
+    sc = oracle.default_scale(64, None)
+    for h in range(2):
+        a = oracle.attn_exact_head(pb.q[0][h], pb.k[0][h], pb.v[0][h], causal, sc)
+        b = oracle.attn_tiled_fp64_head(pb.q[0][h], pb.k[0][h], pb.v[0][h], causal, sc, lazy_tau=tau)
+        assert np.max(np.abs(a - b)) < 1e-12
+
+
+def test_lazy_without_moves_equals_plain_16bit():
+    """Every row's maximum in the first key tile (K zero except key 0, so all
+    later scores are 0 <= that maximum): the reference never moves, and with
+    16-bit P~ the lazy result equals the plain online softmax exactly."""
+    rng = np.random.default_rng(31)
+    B, H, S, D = 1, 2, 300, 64
+    q = torch.from_numpy(rng.standard_normal((B, H, S, D)).astype(np.float16))
+    kk = np.zeros((B, H, S, D), np.float16)
+    kk[:, :, 0] = rng.standard_normal((B, H, D)) * 3
+    k = torch.from_numpy(kk)
+    v = torch.from_numpy(rng.standard_normal((B, H, S, D)).astype(np.float16))
+    plain = oracle.attention(q, k, v, pv="fp16", smooth_k=False)
+    lazy = oracle.attention(q, k, v, pv="fp16", smooth_k=False, lazy_tau=8)
+    assert np.array_equal(plain, lazy)
+
+
+def test_lazy_fp8_accuracy():
+    """FP8 P~ with the 448 * 2^-2 scale the lazy mode needs keeps the
+    method's accuracy against exact attention."""
+    sp = synth.Spec("t", Hq=2, Hkv=2, D=128, B=1, S=1024, k_bias_std=3.0, seed=14)
+    q, k, v = synth.make(sp)
+    ex = oracle.attention_exact(q, k, v)
+    plain = oracle.attention(q, k, v, pv="fp8")
+    lazy = oracle.attention(q, k, v, pv="fp8", lazy_tau=2)
+    cos_l, rl1_l = _accuracy(lazy, ex)
+    cos_p, rl1_p = _accuracy(plain, ex)
+    assert cos_l >= 0.999, cos_l
+    assert rl1_l <= 1.5 * rl1_p, (rl1_l, rl1_p)
