@@ -49,7 +49,7 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default=WORKLOAD)
     ap.add_argument("--pv", default="fp8", choices=["fp8", "fp16"])
-    ap.add_argument("--pv-accum", default="fp32", choices=["fp32", "fp32+fp32"])
+    ap.add_argument("--pv-accum", default="fp32", choices=["fp32", "fp32+fp32", "fp32_lazy"])
     ap.add_argument("--gran", default="per_block", choices=["per_block", "per_warp", "per_thread", "per_token"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)

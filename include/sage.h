@@ -92,8 +92,12 @@ typedef enum { SAGE_PV_FP8 = 0, SAGE_PV_FP16 = 1, SAGE_PV_FP8_SMOOTH_V = 2 } sag
 
 /* P~V accumulation: FP32 = one FP32 tensor-memory accumulator across all KV
  * tiles; FP32_FP32 = a fresh FP32 partial sum per 128-key tile added into a
- * separate FP32 register accumulator (two-level accumulation). */
-typedef enum { SAGE_ACC_FP32 = 0, SAGE_ACC_FP32_FP32 = 1 } sage_acc_t;
+ * separate FP32 register accumulator (two-level accumulation).
+ * FP32_LAZY = FP32 with conditional rescaling: P~ and O stay relative to a
+ * reference maximum that moves only when a tile's maximum exceeds it by more
+ * than tau (tau = 2 with FP8 P~V, whose static P~ scale becomes 448 * 2^-2;
+ * tau = 8 with 16-bit P~V), so most tiles skip the rescale of O. */
+typedef enum { SAGE_ACC_FP32 = 0, SAGE_ACC_FP32_FP32 = 1, SAGE_ACC_FP32_LAZY = 2 } sage_acc_t;
 
 /* ------------------------------------------------------------------------ */
 /* Workspace.                                                               */

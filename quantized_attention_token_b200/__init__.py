@@ -29,7 +29,7 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = ran
 LAYOUT = {"HND": 0, "NHD": 1}
 GRAN = {"per_block": 0, "per_warp": 1, "per_thread": 2, "per_token": 3}
 PV = {"fp8": 0, "fp16": 1, "fp8_smooth_v": 2}   # fp8_smooth_v: FP8 with V smoothed by its channel mean
-ACC = {"fp32": 0, "fp32+fp32": 1, "fp32fp32": 1}
+ACC = {"fp32": 0, "fp32+fp32": 1, "fp32fp32": 1, "fp32_lazy": 2}   # fp32_lazy: one-level, conditional rescaling
 
 
 class SageError(RuntimeError):

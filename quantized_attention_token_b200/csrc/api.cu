@@ -97,7 +97,7 @@ sage_status_t check_common(sage_dtype_t dtype, int D, sage_gran_t gran, sage_pv_
   if (gran != SAGE_PER_BLOCK && gran != SAGE_PER_WARP && gran != SAGE_PER_THREAD && gran != SAGE_PER_TOKEN)
     return SAGE_ERR_INVALID_ARG;
   if (pv != SAGE_PV_FP8 && pv != SAGE_PV_FP16 && pv != SAGE_PV_FP8_SMOOTH_V) return SAGE_ERR_INVALID_ARG;
-  if (acc != SAGE_ACC_FP32 && acc != SAGE_ACC_FP32_FP32) return SAGE_ERR_INVALID_ARG;
+  if (acc != SAGE_ACC_FP32 && acc != SAGE_ACC_FP32_FP32 && acc != SAGE_ACC_FP32_LAZY) return SAGE_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return SAGE_ERR_UNSUPPORTED;
   return SAGE_OK;
 }
@@ -182,6 +182,7 @@ sage_status_t run_attn(void* out, int bf16, Strides so, const Seqs& seqs, int ns
   p.q_bias = smooth_q ? at<float>(w, L.q_bias) : nullptr;
   p.bias_ld = seqs.tps * kTile;
   p.gran = gran;
+  p.lazy_tau = acc == SAGE_ACC_FP32_LAZY ? (pv == SAGE_PV_FP16 ? 8 : 2) : 0;
   p.causal = causal ? 1 : 0;
   p.out_bf16 = bf16;
   p.v_mean = pv == SAGE_PV_FP8_SMOOTH_V ? at<float>(w, L.v_mean) : nullptr;

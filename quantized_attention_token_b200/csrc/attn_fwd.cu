@@ -341,7 +341,13 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(C::B_SCONS + q));
-      const float m_new = fmaxf(m, mt);
+      // Conditional rescaling: P~ and O stay relative to the reference m,
+      // which moves to the running maximum only when this tile's maximum
+      // passes m + tau (tau = 0: the plain online softmax).  P~ <= 2^tau, so
+      // FP8 P~ takes the static scale 448 * 2^-tau; the epilogue's 1/l, with
+      // l summing the scaled P~, divides it out again.
+      const bool move = (m == -INFINITY) || (mt > m + (float)p.lazy_tau);
+      const float m_new = move ? fmaxf(m, mt) : m;
       const float alpha = (m == -INFINITY) ? 0.f : ex2(m - m_new);
       if (!PV8 && NQ == 2 && q == 0 && j == 0) mbar_arrive(bar(C::B_GO));
       // PV_{j-1} must be done before the P~ buffer it reads is rewritten (one
@@ -359,12 +365,12 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
         alpha_s[(q * 2 + ab) * 128 + t] = alpha;
         mbar_arrive(bar(C::B_AFULL + 2 * q + ab));
       }
-      const float nb = -(PV8 ? (m_new - kLog2Fp8Max) : m_new);
-      // Two query tiles: their exponential phases take turns (tile 0's of KV
-      // tile j, then tile 1's, then tile 0's of j+1, ...), so that each runs
-      // at the MUFU's full rate while the other warpgroup does its maximum and
-      // O rescale.  A tile waits only for turns its partner has (causal: the
-      // second query tile can have one KV tile more than the first).
+      const float nb = -(PV8 ? (m_new - kLog2Fp8Max + (float)p.lazy_tau) : m_new);
+      // FP8 P~V, two query tiles: their exponential phases take turns (tile
+      // 0's of KV tile j, then tile 1's, then tile 0's of j+1, ...), so that
+      // each runs at the MUFU's full rate while the other warpgroup does its
+      // maximum and O rescale.  A tile waits only for turns its partner has
+      // (causal: the second query tile can have one KV tile more).
       if (PV8 && NQ == 2) {
         const bool wait_turn = q == 0 ? (j > 0 && j - 1 < n[1]) : (j < n[0]);
         if (wait_turn &&

@@ -321,7 +321,7 @@ __device__ void vstat_tile(const PrepassJob& j, int h, const TileLoc& L, StatSme
   uint4 v[M::NR];
   load_tile<D, false>(head, j.sv.ss, L, v);
   const size_t o = ((size_t)L.b * j.Hkv + h) * D;
-  if (!SMOOTH) {
+  if constexpr (!SMOOTH) {
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       uint32_t a = 0;
@@ -338,43 +338,44 @@ __device__ void vstat_tile(const PrepassJob& j, int h, const TileLoc& L, StatSme
       atomicMax(&j.v_stat[2 * (o + tid)], __float_as_uint(h16_to_f32((uint16_t)m, BF16)));
     }
     return;
-  }
+  } else {
 #pragma unroll
-  for (int u = 0; u < 8; ++u) {
-    double a = 0.0;
-    uint32_t kmax = 0, kneg = 0;
+    for (int u = 0; u < 8; ++u) {
+      double a = 0.0;
+      uint32_t kmax = 0, kneg = 0;
 #pragma unroll
-    for (int i = 0; i < M::NR; ++i) {
-      const uint16_t x = h16(v[i], u);
-      a += (double)h16_to_f32(x, BF16);                 // rows past the sequence hold 0
-      if (rg * M::NR + i < L.nvalid) {
-        kmax = max(kmax, key16(x));
-        kneg = max(kneg, key16(x ^ 0x8000u));
+      for (int i = 0; i < M::NR; ++i) {
+        const uint16_t x = h16(v[i], u);
+        a += (double)h16_to_f32(x, BF16);                 // rows past the sequence hold 0
+        if (rg * M::NR + i < L.nvalid) {
+          kmax = max(kmax, key16(x));
+          kneg = max(kneg, key16(x ^ 0x8000u));
+        }
+      }
+      a = reduce_same_chunk<D>(a, [](double x, double y) { return x + y; });
+      kmax = reduce_same_chunk<D>(kmax, [](uint32_t x, uint32_t y) { return max(x, y); });
+      kneg = reduce_same_chunk<D>(kneg, [](uint32_t x, uint32_t y) { return max(x, y); });
+      if (lane < M::TPR) {
+        sm.sum[warp][cc * 8 + u] = a;
+        sm.amax[warp][cc * 8 + u] = kmax;
+        sm.kneg[warp][cc * 8 + u] = kneg;
       }
     }
-    a = reduce_same_chunk<D>(a, [](double x, double y) { return x + y; });
-    kmax = reduce_same_chunk<D>(kmax, [](uint32_t x, uint32_t y) { return max(x, y); });
-    kneg = reduce_same_chunk<D>(kneg, [](uint32_t x, uint32_t y) { return max(x, y); });
-    if (lane < M::TPR) {
-      sm.sum[warp][cc * 8 + u] = a;
-      sm.amax[warp][cc * 8 + u] = kmax;
-      sm.kneg[warp][cc * 8 + u] = kneg;
-    }
-  }
-  __syncthreads();
-  if (tid < D) {
-    double sum = 0.0;
-    uint32_t kmax = 0, kneg = 0;
+    __syncthreads();
+    if (tid < D) {
+      double sum = 0.0;
+      uint32_t kmax = 0, kneg = 0;
 #pragma unroll
-    for (int w = 0; w < M::WARPS; ++w) {
-      sum += sm.sum[w][tid];
-      kmax = max(kmax, sm.amax[w][tid]);
-      kneg = max(kneg, sm.kneg[w][tid]);
+      for (int w = 0; w < M::WARPS; ++w) {
+        sum += sm.sum[w][tid];
+        kmax = max(kmax, sm.amax[w][tid]);
+        kneg = max(kneg, sm.kneg[w][tid]);
+      }
+      if (BF16) atomicAdd(reinterpret_cast<double*>(&j.v_sum[o + tid]), sum);
+      else atomicAdd(&j.v_sum[o + tid], (unsigned long long)(long long)(sum * 0x1p24));
+      atomicMax(&j.v_stat[2 * (o + tid)], kmax);
+      atomicMax(&j.v_stat[2 * (o + tid) + 1], kneg);
     }
-    if (BF16) atomicAdd(reinterpret_cast<double*>(&j.v_sum[o + tid]), sum);
-    else atomicAdd(&j.v_sum[o + tid], (unsigned long long)(long long)(sum * 0x1p24));
-    atomicMax(&j.v_stat[2 * (o + tid)], kmax);
-    atomicMax(&j.v_stat[2 * (o + tid) + 1], kneg);
   }
 }
 

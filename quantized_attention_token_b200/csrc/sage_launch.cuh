@@ -53,6 +53,7 @@ struct AttnParams {
   const float* q_bias;       // smooth Q: [Hq][tiles_q][bias_ld] per-key score corrections, else null
   int bias_ld;
   int gran;
+  int lazy_tau;              // conditional rescaling: the reference maximum moves only past +tau (0: always)
   int causal;
   int out_bf16;
 };

@@ -64,7 +64,7 @@ def test_workspace_planner(L):
     (dict(ws=0x1010), sage.ERR_INVALID_ARG),         # ws must be 256-byte aligned
     (dict(gran=7), sage.ERR_INVALID_ARG),
     (dict(pv=3), sage.ERR_INVALID_ARG),
-    (dict(acc=2), sage.ERR_INVALID_ARG),
+    (dict(acc=3), sage.ERR_INVALID_ARG),
     (dict(layout=2), sage.ERR_INVALID_ARG),
     (dict(dtype=2), sage.ERR_INVALID_ARG),
     (dict(ws_bytes=1000), sage.ERR_WORKSPACE),

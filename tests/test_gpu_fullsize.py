@@ -13,7 +13,7 @@ from tests.test_gpu_parity import _assert_close
 pytestmark = pytest.mark.gpu
 
 
-def _oracle_rows(spec, q, k, v, b, h, rows, gran, pv, smooth_q=False, smooth_v=False):
+def _oracle_rows(spec, q, k, v, b, h, rows, gran, pv, smooth_q=False, smooth_v=False, lazy_tau=0):
     """Oracle output and allowance for rows [r0, r1) of (sequence b, head h),
     computed on that sequence / head alone."""
     grp = spec.Hq // spec.Hkv
@@ -30,7 +30,7 @@ def _oracle_rows(spec, q, k, v, b, h, rows, gran, pv, smooth_q=False, smooth_v=F
         qs, ks, vs = q[b:b + 1, :, h:h + 1], k[b:b + 1, :, hk:hk + 1], v[b:b + 1, :, hk:hk + 1]
         lay = "NHD"
     out, allow = oracle.attention(qs, ks, vs, lay, spec.causal, gran=gran, pv=pv, q_rows={(0, 0): rows},
-                                  smooth_q=smooth_q, smooth_v=smooth_v, with_allowance=True)
+                                  smooth_q=smooth_q, smooth_v=smooth_v, lazy_tau=lazy_tau, with_allowance=True)
     sel = (slice(0, 1), slice(0, 1), slice(*rows)) if lay == "HND" else (slice(0, 1), slice(*rows), slice(0, 1))
     pb = oracle.problem(qs, ks, vs, lay)
     ex = oracle.attn_exact_head(pb.q[0][0][rows[0]:rows[1]], pb.k[0][0], pb.v[0][0], spec.causal,
@@ -66,7 +66,8 @@ def _run(spec, gran="per_block", pv="fp8", acc="fp32+fp32", smooth_q=False, smoo
 def _check(spec, samples, gran="per_block", pv="fp8", acc="fp32+fp32", smooth_q=False, smooth_v=False):
     q, k, v, out = _run(spec, gran, pv, acc, smooth_q, smooth_v)
     for b, h, rows in samples:
-        ref, allow, ex = _oracle_rows(spec, q, k, v, b, h, rows, gran, pv, smooth_q, smooth_v)
+        tau = (2 if pv == "fp8" else 8) if acc == "fp32_lazy" else 0
+        ref, allow, ex = _oracle_rows(spec, q, k, v, b, h, rows, gran, pv, smooth_q, smooth_v, tau)
         got = _gpu_rows(spec, out, b, h, rows)
         _assert_close(got, (ref, allow), spec.dtype, f"{spec.name} b{b} h{h} rows{rows}")
         o = got.double().numpy().ravel()
@@ -113,3 +114,8 @@ def test_video_dit_smooth_q_and_v():
 def test_varlen_gqa_smooth_v():
     spec = synth.CONFIGS["varlen_gqa"]
     _check(spec, [(2, 5, (7040, 7168)), (3, 16, (8192, 8320))], acc="fp32", smooth_v=True)
+
+
+def test_b2_h32_s4096_d128_lazy_rescale():
+    spec = synth.CONFIGS["b2_h32_s4096_d128"]
+    _check(spec, [(0, 5, (0, 128)), (1, 27, (3968, 4096))], acc="fp32_lazy")

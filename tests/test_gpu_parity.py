@@ -288,6 +288,29 @@ def test_varlen_smooth_v_matches_oracle():
     _assert_close(out, ref, "fp16", "varlen smooth V vs oracle")
 
 
+@pytest.mark.parametrize("D,S,causal,gran,pv,dtype,layout", [
+    (128, 640, False, "per_block", "fp8", "fp16", "HND"),
+    (128, 300, True, "per_thread", "fp8", "bf16", "NHD"),
+    (64, 517, False, "per_token", "fp16", "fp16", "HND"),
+    (128, 384, True, "per_warp", "fp16", "bf16", "HND"),
+])
+def test_attention_lazy_rescale_matches_oracle(D, S, causal, gran, pv, dtype, layout):
+    """Conditional rescaling (tau = 2 with FP8 P~V, 8 with 16-bit)."""
+    sp = synth.Spec("t", Hq=4, Hkv=2, D=D, B=2, S=S, dtype=dtype, layout=layout, causal=causal, k_bias_std=3.0,
+                    seed=100 + S)
+    q, k, v = synth.make(sp)
+    out = sage.sageattn(_dev(q), _dev(k), _dev(v), layout, causal, qk_quant_gran=gran, pv_dtype=pv,
+                        pv_accum_dtype="fp32_lazy")
+    torch.cuda.synchronize()
+    ref = oracle.attention(q, k, v, layout, causal, gran=gran, pv=pv, lazy_tau=2 if pv == "fp8" else 8,
+                           with_allowance=True)
+    _assert_close(out, ref, dtype, "lazy rescale vs oracle")
+    ex = oracle.attention_exact(q, k, v, layout, causal)
+    o = out.double().cpu().numpy().ravel()
+    cos = o @ ex.ravel() / (np.linalg.norm(o) * np.linalg.norm(ex))
+    assert cos >= 0.999, cos
+
+
 def test_tiny_config():
     sp = synth.CONFIGS["tiny"]
     q, k, v = synth.make(sp)
