@@ -285,6 +285,29 @@ def main():
     ms_per_step = elapsed_ms / args.steps
     value = job_tops(world, ops, args.steps, elapsed_ms)
 
+    # the attention kernel alone in the other modes the workload names (and
+    # the conditional-rescaling mode), inputs resident, CUDA events
+    def kernel_tops(pv, acc, n=100):
+        sage.quant_qkv(q, k, v, ws, layout, args.gran, pv)
+
+        def f():
+            sage.attn_quantized(out, ws, B, spec.Hq, spec.Hkv, S, D, layout, spec.causal, None, args.gran, pv, acc)
+
+        for _ in range(3):
+            f()
+        m0, m1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        m0.record(stream)
+        for _ in range(n):
+            f()
+        m1.record(stream)
+        torch.cuda.synchronize()
+        return ops / (m0.elapsed_time(m1) / n * 1e-3) / 1e12
+
+    other_modes = {f"{pv}/{acc}": kernel_tops(pv, acc)
+                   for pv, acc in [("fp8", "fp32+fp32"), ("fp8", "fp32_lazy"), ("fp16", "fp32"), ("fp16", "fp32+fp32"),
+                                   ("fp16", "fp32_lazy")] if (pv, acc) != (args.pv, args.pv_accum)}
+
     # end to end through the public API with host buffers: every step copies
     # q, k, v in from pinned host memory, runs sageattn and copies the output
     # back.  Steps are pipelined over three streams (inputs in, compute,
@@ -368,6 +391,7 @@ def main():
         "e2e": {"value": job_tops(world, ops, 1, e2e_ms), "unit": "TOPS",
                 "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))),
                 "d2h_bytes_per_step": int(q_h.numel() * q_h.element_size())},
+        "attention_modes_tops": other_modes,   # attention kernel alone, other P~V / accumulation modes
         "gpu_launches": 3 * args.steps,     # pre-pass launches A and B + the attention kernel
         "clocks": clk.summary(),
     }

@@ -223,9 +223,10 @@ __device__ void quant_tile(const PrepassJob& j, int h, int t, const TileLoc& L, 
   for (int i = 0; i < M::NR; ++i) {
     float x[8];
     X8(i, x);
-    float m = 0.f;
-#pragma unroll
-    for (int u = 0; u < 8; ++u) m = fmaxf(m, fabsf(x[u]));
+    float m = max3(fabsf(x[0]), fabsf(x[1]), fabsf(x[2]));
+    m = max3(m, fabsf(x[3]), fabsf(x[4]));
+    m = max3(m, fabsf(x[5]), fabsf(x[6]));
+    m = fmaxf(m, fabsf(x[7]));
 #pragma unroll
     for (int o = M::TPR / 2; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (cc == 0) {
@@ -267,14 +268,16 @@ __device__ void quant_tile(const PrepassJob& j, int h, int t, const TileLoc& L, 
     const float inv = sm.ginv[IS_Q ? q_group(j.gran, r) : k_group(j.gran, r)];
     float x[8];
     X8(i, x);
-    uint32_t w[2] = {0u, 0u};
+    // code = rne(x * inv): adding 1.5 * 2^23 rounds the product to an integer
+    // (ties to even) and leaves it, two's complement, in the low bits.  No
+    // clamp is needed: |x| <= amax and inv = fl(127/amax) give |x * inv| <=
+    // 127 (1 + 2^-24), which rounds to at most 127.
+    uint32_t b[8];
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-      int c = __float2int_rn(__fmul_rn(x[u], inv));
-      c = max(-127, min(127, c));
-      w[u >> 2] |= ((uint32_t)(c & 0xFF)) << ((u & 3) * 8);
-    }
-    *reinterpret_cast<uint2*>(tbase + swz(r, cc * 8, D)) = make_uint2(w[0], w[1]);
+    for (int u = 0; u < 8; ++u) b[u] = __float_as_uint(__fadd_rn(__fmul_rn(x[u], inv), 12582912.0f));
+    const uint32_t w0 = __byte_perm(__byte_perm(b[0], b[1], 0x0040), __byte_perm(b[2], b[3], 0x0040), 0x5410);
+    const uint32_t w1 = __byte_perm(__byte_perm(b[4], b[5], 0x0040), __byte_perm(b[6], b[7], 0x0040), 0x5410);
+    *reinterpret_cast<uint2*>(tbase + swz(r, cc * 8, D)) = make_uint2(w0, w1);
   }
 }
 
