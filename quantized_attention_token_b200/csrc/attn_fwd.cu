@@ -10,8 +10,10 @@
 // FP32 tensor-memory accumulator (fp32) or, per tile, into a separate FP32
 // register accumulator (fp32+fp32, the two-level scheme).
 //
-// B200 design.  One CTA (384 threads) owns NQ query tiles of 128 rows of one
-// (sequence, head):
+// B200 design.  A persistent grid, one CTA (384 threads) per SM, walks work
+// items of NQ query tiles of 128 rows of one (sequence, head); the mbarrier
+// phases and the K/V ring run on from one item to the next, and the next
+// item's first QK^T runs during the current item's epilogue:
 //   warp 0        loader: one bulk copy per MMA-ready tile (the pre-pass wrote
 //                 tiles already in the swizzled operand layout), NST stages;
 //   warp 1        MMA issuer: tcgen05.mma kind::i8 (S = Q K^T, SMEM x SMEM ->
@@ -25,6 +27,8 @@
 //                 also rescales O in TMEM and writes the epilogue;
 //   WG 2 (two-level mode, NQ = 1) correction: adds each tile's fresh FP32
 //                 partial O into an FP32 register accumulator; epilogue.
+// Warpgroup 0 (loader, MMA, allocator) hands registers to WG 1..2 with
+// setmaxnreg (56 / 224 / 224 per thread).
 // Every mbarrier wait is bounded (sage_common.cuh): a wait that never ends sets
 // the device error word and the CTA tears down instead of hanging.
 #include "sage_launch.cuh"
@@ -35,7 +39,11 @@ template <int D, bool PV8, bool ACC2>
 struct AttnCfg {
   static constexpr int NQ = ACC2 ? 1 : 2;          // query tiles per CTA
   static constexpr int NST = PV8 ? 3 : 2;          // K/V pipeline stages
-  static constexpr int NTHREADS = 384;             // 3 warpgroups (168 registers per thread)
+  static constexpr int NTHREADS = 384;             // 3 warpgroups (168 registers per thread at launch)
+  // per-thread registers after the split: loader / MMA warpgroup, compute
+  // warpgroups; 128 * (REGS_LOAD + 2 * REGS_COMPUTE) = NTHREADS * REGS_LAUNCH
+  static constexpr int REGS_LAUNCH = 168, REGS_LOAD = 56, REGS_COMPUTE = 224;
+  static_assert(128 * (REGS_LOAD + 2 * REGS_COMPUTE) == NTHREADS * REGS_LAUNCH, "register split");
   static constexpr int QT = kTile * D;             // bytes of a Q or K tile
   static constexpr int VT = D * kTile * (PV8 ? 1 : 2);
   static constexpr int PT = kTile * kTile * (PV8 ? 1 : 2);   // P~ tile in shared memory
@@ -52,7 +60,8 @@ struct AttnCfg {
   static constexpr int OFF_BAR = OFF_BIAS + NST * NQ * 128 * 4;
   enum {
     B_QFULL = 0,
-    B_KFULL = B_QFULL + NQ,
+    B_QEMPTY = B_QFULL + NQ,         // MMA -> loader: the item's last QK^T with this Q tile is done
+    B_KFULL = B_QEMPTY + NQ,
     B_KEMPTY = B_KFULL + NST,
     B_VFULL = B_KEMPTY + NST,
     B_VEMPTY = B_VFULL + NST,
@@ -64,7 +73,8 @@ struct AttnCfg {
     B_AFULL = B_OREADY + NQ,         // softmax -> correction: alpha (two-level)
     B_AEMPTY = B_AFULL + 2 * NQ,
     B_LFULL = B_AEMPTY + 2 * NQ,     // softmax -> correction: final row sum (two-level)
-    B_DONE = B_LFULL + NQ,
+    B_LEMPTY = B_LFULL + NQ,         // correction -> softmax: row sum read
+    B_DONE = B_LEMPTY + NQ,
     B_TOK = B_DONE + 1,              // FP8: exponential-phase token, [0] query tile 0 may run, [1] tile 1 may
     B_GO = B_TOK + 2,                // 16-bit: softmax 0 -> softmax 1, start after tile 0's maximum
     NBAR = B_GO + 1
@@ -267,12 +277,76 @@ __device__ __forceinline__ void store_row(uint16_t* orow, uint32_t ob, const flo
   }
 }
 
-// One softmax warpgroup: the online softmax of query tile q over its KV
-// tiles; in one-level mode also the O rescale and the epilogue.
+// ---------------------------------------------------------------- work items
+// A copy of x that the compiler cannot see through, so that values derived
+// from it are recomputed instead of kept live.
+__device__ __forceinline__ int opaque(int x) {
+  int y;
+  asm volatile("mov.b32 %0, %1;" : "=r"(y) : "r"(x));
+  return y;
+}
+
+// A work item is NQ consecutive query tiles (a "pair") of one (sequence,
+// head).  The grid is persistent, one CTA per SM: CTA c takes items c,
+// c + gridDim.x, c + 2 gridDim.x, ...  Every role walks the same list, so all
+// mbarrier phases simply continue from one item to the next.  Non-causal
+// items run pair-fastest (the CTAs that run at the same time share K/V in L2);
+// causal items run longest first.
+template <int NQ>
+struct Item {
+  int b, h, hk, pair, qs, Lq, Lk, tq0, tk0;
+  int n[NQ];   // KV tiles of each query tile (0: the query tile is past the sequence)
+  int maxn;
+};
+
+// false: the item is empty (past its sequence) or fails a check that the
+// pre-pass or the host already reported.
+template <int NQ>
+__device__ __forceinline__ bool decode_item(const AttnParams& p, int idx, Item<NQ>& it) {
+  const int nbh = p.Hq * p.nseq;
+  int bh;
+  if (p.causal) {
+    it.pair = p.n_pairs - 1 - idx / nbh;
+    bh = idx % nbh;
+  } else {
+    it.pair = idx % p.n_pairs;
+    bh = idx / p.n_pairs;
+  }
+  it.h = bh % p.Hq;
+  it.b = bh / p.Hq;
+  int ks;
+  p.seqs.q(it.b, it.qs, it.Lq, it.tq0);
+  p.seqs.k(it.b, ks, it.Lk, it.tk0);
+  if (p.seqs.cu_q && (it.Lq > p.seqs.max_seqlen || it.Lk > p.seqs.max_seqlen || it.Lq < 0 || it.Lk < 0))
+    return false;
+  if (it.pair * NQ * kTile >= it.Lq) return false;
+  it.hk = it.h / p.group;
+  const int nk = (it.Lk + kTile - 1) / kTile;
+  // the workspace must hold every tile the item reads (varlen: the offsets
+  // kernel has already flagged an overflow)
+  if (it.tq0 + (it.Lq + kTile - 1) / kTile > p.tiles_q || it.tk0 + nk > p.tiles_k) return false;
+  it.maxn = 0;
+#pragma unroll
+  for (int q = 0; q < NQ; ++q) {
+    const int qt = it.pair * NQ + q;
+    it.n[q] = qt * kTile >= it.Lq ? 0 : (p.causal ? min(nk, qt + 1) : nk);
+    it.maxn = max(it.maxn, it.n[q]);
+  }
+  return true;
+}
+
+// The next item after idx in this CTA's list that has KV tiles.
+template <int NQ>
+__device__ __forceinline__ bool next_busy_item(const AttnParams& p, int idx, Item<NQ>& it) {
+  for (idx += gridDim.x; idx < p.n_items; idx += gridDim.x)
+    if (decode_item<NQ>(p, idx, it) && it.maxn > 0) return true;
+  return false;
+}
+
+// One softmax warpgroup: for each item, the online softmax of query tile q
+// over its KV tiles; in one-level mode also the O rescale and the epilogue.
 template <int D, bool PV8, bool ACC2, bool KPT, bool BF16P, bool SMQ>
-__device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, uint32_t tmem, int warp, int tid,
-                                             int pair, int b, int h, int hk, int qs, int Lq, int Lk, int tq0,
-                                             int tk0, const int* n, const float* vsc, const float* vmu) {
+__device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, uint32_t tmem, int warp, int tid) {
   using C = AttnCfg<D, PV8, ACC2>;
   constexpr int NQ = C::NQ;
   auto bar = [&](int i) -> uint32_t { return sb + C::OFF_BAR + 8 * i; };
@@ -284,157 +358,217 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
 
   const int q = (warp - 4) >> 2;
   const int t = tid - 128 * (1 + q);
-  const int qt = pair * NQ + q;
   const uint32_t lane_off = (uint32_t)((t & ~31)) << 16;
-  const int row = qt * kTile + t;
   const bool bf16 = BF16P || (PV8 && p.out_bf16 != 0);
   const uint32_t taddr = tmem + C::TM_S + q * 128 + lane_off;
   const uint32_t ob = tmem + C::TM_O + q * D + lane_off;
-  float m = -INFINITY, l = 0.f;
   bool ok = true;
-  int n_stop = n[q];
-  if (n[q] > 0) {
-    const float qsc = p.q_scale[((size_t)h * p.tiles_q + tq0 + qt) * kQGroupsMax + q_group(p.gran, t)];
-    const float* ksb = p.k_scale + ((size_t)hk * p.tiles_k + tk0) * kKGroupsMax;
-    // K group scales of the next tile are fetched one tile ahead
-    float ksn[KPT ? 16 : 2];
-#pragma unroll
-    for (int g = 0; g < (KPT ? 16 : 2); ++g) ksn[g] = __ldg(ksb + g);
-    // seed the S columns for the first QK^T (see tile_max)
-    tmem_fill128(taddr, 0x4B400000u);
-    tmem_wait_st();
-    tc_fence_before();
-    mbar_arrive(bar(C::B_SCONS + q));
-    if (!PV8 && NQ == 2 && q == 1 && n[0] > 0) {
-      if (!(ok = mbar_wait(bar(C::B_GO), 0, abort_flag, p.err, kErrTimeoutSoftmax))) n_stop = 0;
+  // Phases that run on across items, packed into one register (the tile loop
+  // is at the register limit): parity of S_j arrivals, of P~ tiles handed to
+  // the MMA (= PVs issued) and whether there was one, of FP8 token turns and
+  // 16-bit go signals, the two-level alpha slot (mod 4) and l hand-off parity
+  // and whether there was one, and the warpgroup of the previous busy item's
+  // last exponential phase (FP8 token; 3 = none).
+  enum : uint32_t { PH_S = 1, PH_PV = 2, PH_PVANY = 4, PH_TOK = 8, PH_GO = 16, PH_L = 32, PH_LANY = 64,
+                    PH_A0 = 128 /* 2 bits */, PH_LAST0 = 512 /* 2 bits */ };
+  uint32_t ph = 3u * PH_LAST0;
+  int kvbase = 0;       // K/V ring index of the item's first tile (smooth Q)
+
+  // seed the S columns for the first QK^T (see tile_max)
+  tmem_fill128(taddr, 0x4B400000u);
+  tmem_wait_st();
+  tc_fence_before();
+  mbar_arrive(bar(C::B_SCONS + q));
+
+  for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
+    Item<NQ> it;
+    if (!decode_item<NQ>(p, idx, it)) continue;
+    const int qt = it.pair * NQ + q;
+    const int row = qt * kTile + t;
+    const int nq = it.n[q];
+    // FP8 token: warpgroup of the next busy item's first exponential phase
+    int next_first = -1;
+    if (PV8 && NQ == 2 && it.maxn > 0) {
+      Item<NQ> nx;
+      if (next_busy_item<NQ>(p, idx, nx)) next_first = nx.n[0] > 0 ? 0 : 1;
     }
-    for (int j = 0; j < n_stop; ++j) {
-      float c[16];
+    float m = -INFINITY, l = 0.f;
+    if (nq > 0) {
+      const float qsc = p.q_scale[((size_t)it.h * p.tiles_q + it.tq0 + qt) * kQGroupsMax + q_group(p.gran, t)];
+      const float* ksb = p.k_scale + ((size_t)it.hk * p.tiles_k + it.tk0) * kKGroupsMax;
+      // K group scales of the next tile are fetched one tile ahead
+      float ksn[KPT ? 16 : 2];
 #pragma unroll
-      for (int g = 0; g < 16; ++g) c[g] = g < (KPT ? 16 : 2) ? fmaxf((qsc * ksn[g]) * p.sl2, 1e-30f) : 1e-30f;
-      if (j + 1 < n[q]) {
+      for (int g = 0; g < (KPT ? 16 : 2); ++g) ksn[g] = __ldg(ksb + g);
+      if (!PV8 && NQ == 2 && q == 1 && it.n[0] > 0) {
+        if (!(ok = mbar_wait(bar(C::B_GO), (ph / PH_GO) & 1, abort_flag, p.err, kErrTimeoutSoftmax))) break;
+      }
+      for (int j = 0; j < nq; ++j) {
+        float c[16];
 #pragma unroll
-        for (int g = 0; g < (KPT ? 16 : 2); ++g) ksn[g] = __ldg(ksb + (j + 1) * kKGroupsMax + g);
-      }
-      if (!(ok = mbar_wait(bar(C::B_SFULL + q), j & 1, abort_flag, p.err, kErrTimeoutSoftmax))) break;
-      tc_fence_after();
-      uint32_t r[128];
-      tmem_ld128_sync(taddr, r);
-      // the S columns are read: re-seed them (the stores complete during the
-      // max below) and then let the next QK^T in
-      tmem_fill128(taddr, 0x4B400000u);
-      // keys past the sequence, or (causal) past this row, are masked
-      const int col0 = j * kTile;
-      const bool masked = (col0 + kTile > Lk) || (p.causal && j == qt);
-      const int lim = p.causal ? min(Lk, row + 1) : Lk;
-      float mt;
-      if (SMQ) {
-        // the tile's key corrections arrive with its V tile
-        if (!(ok = mbar_wait(bar(C::B_VFULL + j % C::NST), (j / C::NST) & 1, abort_flag, p.err,
-                             kErrTimeoutSoftmax)))
-          break;
-        const float* bias = reinterpret_cast<const float*>(smem + C::OFF_BIAS + ((j % C::NST) * NQ + q) * 512);
-        mt = tile_max_bias<KPT>(r, c, bias, p.sl2, masked, col0, lim);
-      } else {
-        mt = tile_max<KPT>(r, c, masked, col0, lim);
-      }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(bar(C::B_SCONS + q));
-      // Conditional rescaling: P~ and O stay relative to the reference m,
-      // which moves to the running maximum only when this tile's maximum
-      // passes m + tau (tau = 0: the plain online softmax).  P~ <= 2^tau, so
-      // FP8 P~ takes the static scale 448 * 2^-tau; the epilogue's 1/l, with
-      // l summing the scaled P~, divides it out again.
-      const bool move = (m == -INFINITY) || (mt > m + (float)p.lazy_tau);
-      const float m_new = move ? fmaxf(m, mt) : m;
-      const float alpha = (m == -INFINITY) ? 0.f : ex2(m - m_new);
-      if (!PV8 && NQ == 2 && q == 0 && j == 0) mbar_arrive(bar(C::B_GO));
-      // PV_{j-1} must be done before the P~ buffer it reads is rewritten (one
-      // buffer) and before O is rescaled (both cases)
-      if (C::NPB == 1 && j > 0) {
-        if (!(ok = mbar_wait(bar(C::B_OFULL + q), (j - 1) & 1, abort_flag, p.err, kErrTimeoutSoftmax))) break;
+        for (int g = 0; g < 16; ++g) c[g] = g < (KPT ? 16 : 2) ? fmaxf((qsc * ksn[g]) * p.sl2, 1e-30f) : 1e-30f;
+        if (j + 1 < nq) {
+#pragma unroll
+          for (int g = 0; g < (KPT ? 16 : 2); ++g) ksn[g] = __ldg(ksb + (j + 1) * kKGroupsMax + g);
+        }
+        if (!(ok = mbar_wait(bar(C::B_SFULL + q), ph & PH_S, abort_flag, p.err, kErrTimeoutSoftmax))) break;
+        ph ^= PH_S;
         tc_fence_after();
-      }
-      const uint32_t p_smem = sb + C::OFF_P + ((j % C::NPB) * NQ + q) * C::PT;
-      if (ACC2) {
-        const int ab = j & 1;
-        if (!(ok = mbar_wait(bar(C::B_AEMPTY + 2 * q + ab), ((j >> 1) & 1) ^ 1, abort_flag, p.err,
-                             kErrTimeoutSoftmax)))
-          break;
-        alpha_s[(q * 2 + ab) * 128 + t] = alpha;
-        mbar_arrive(bar(C::B_AFULL + 2 * q + ab));
-      }
-      const float nb = -(PV8 ? (m_new - kLog2Fp8Max + (float)p.lazy_tau) : m_new);
-      // FP8 P~V, two query tiles: their exponential phases take turns (tile
-      // 0's of KV tile j, then tile 1's, then tile 0's of j+1, ...), so that
-      // each runs at the MUFU's full rate while the other warpgroup does its
-      // maximum and O rescale.  A tile waits only for turns its partner has
-      // (causal: the second query tile can have one KV tile more).
-      if (PV8 && NQ == 2) {
-        const bool wait_turn = q == 0 ? (j > 0 && j - 1 < n[1]) : (j < n[0]);
-        if (wait_turn &&
-            !(ok = mbar_wait(bar(C::B_TOK + q), q == 0 ? ((j - 1) & 1) : (j & 1), abort_flag, p.err,
-                             kErrTimeoutSoftmax)))
-          break;
-      }
-      const float lt = tile_exp_store<PV8, KPT, BF16P, SMQ>(r, c, nb, p_smem, t);
-      if (PV8 && NQ == 2 && (q == 0 ? j < n[1] : j + 1 < n[0])) mbar_arrive(bar(C::B_TOK + (q ^ 1)));
-      l = alpha * l + lt;
-      m = m_new;
-      if (C::NPB == 2 && j > 0) {
-        if (!(ok = mbar_wait(bar(C::B_OFULL + q), (j - 1) & 1, abort_flag, p.err, kErrTimeoutSoftmax))) break;
-        tc_fence_after();
-      }
-      if (!ACC2 && j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
-        // O(q) holds the sums of tiles < j
-        if (D == 128) {
-          uint32_t o[128];
-          tmem_ld128_sync(ob, o);
-#pragma unroll
-          for (int u = 0; u < 128; u += 2) {
-            float x0, x1;
-            mul2(x0, x1, __uint_as_float(o[u]), __uint_as_float(o[u + 1]), alpha, alpha);
-            o[u] = __float_as_uint(x0);
-            o[u + 1] = __float_as_uint(x1);
-          }
-          tmem_st128(ob, o);
+        uint32_t r[128];
+        tmem_ld128_sync(taddr, r);
+        // the S columns are read: re-seed them (the stores complete during the
+        // max below) and then let the next QK^T in -- of this item or the next
+        tmem_fill128(taddr, 0x4B400000u);
+        // keys past the sequence, or (causal) past this row, are masked
+        const int col0 = j * kTile;
+        const bool masked = (col0 + kTile > it.Lk) || (p.causal && j == qt);
+        const int lim = p.causal ? min(it.Lk, row + 1) : it.Lk;
+        float mt;
+        if (SMQ) {
+          // the tile's key corrections arrive with its V tile
+          const int kv = kvbase + j;
+          if (!(ok = mbar_wait(bar(C::B_VFULL + kv % C::NST), (kv / C::NST) & 1, abort_flag, p.err,
+                               kErrTimeoutSoftmax)))
+            break;
+          const float* bias =
+              reinterpret_cast<const float*>(smem + C::OFF_BIAS + ((kv % C::NST) * NQ + q) * 512);
+          mt = tile_max_bias<KPT>(r, c, bias, p.sl2, masked, col0, lim);
         } else {
+          mt = tile_max<KPT>(r, c, masked, col0, lim);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(bar(C::B_SCONS + q));
+        // Conditional rescaling: P~ and O stay relative to the reference m,
+        // which moves to the running maximum only when this tile's maximum
+        // passes m + tau (tau = 0: the plain online softmax).  P~ <= 2^tau, so
+        // FP8 P~ takes the static scale 448 * 2^-tau; the epilogue's 1/l, with
+        // l summing the scaled P~, divides it out again.
+        const bool move = (m == -INFINITY) || (mt > m + (float)p.lazy_tau);
+        const float m_new = move ? fmaxf(m, mt) : m;
+        const float alpha = (m == -INFINITY) ? 0.f : ex2(m - m_new);
+        if (!PV8 && NQ == 2 && q == 0 && j == 0) mbar_arrive(bar(C::B_GO));
+        // the PV that last read the P~ buffer must be done before it is
+        // rewritten (one buffer; the item's first tile too, since two-level
+        // mode has no epilogue wait)
+        if (C::NPB == 1 && (ph & PH_PVANY)) {
+          if (!(ok = mbar_wait(bar(C::B_OFULL + q), ((ph / PH_PV) & 1) ^ 1, abort_flag, p.err, kErrTimeoutSoftmax)))
+            break;
+          tc_fence_after();
+        }
+        const uint32_t p_smem = sb + C::OFF_P + ((j % C::NPB) * NQ + q) * C::PT;
+        if (ACC2) {
+          const uint32_t a = (ph / PH_A0) & 3;
+          const int ab = a & 1;
+          if (!(ok = mbar_wait(bar(C::B_AEMPTY + 2 * q + ab), ((a >> 1) & 1) ^ 1, abort_flag, p.err,
+                               kErrTimeoutSoftmax)))
+            break;
+          ph = (ph & ~(3u * PH_A0)) | (((a + 1) & 3) * PH_A0);
+          alpha_s[(q * 2 + ab) * 128 + t] = alpha;
+          mbar_arrive(bar(C::B_AFULL + 2 * q + ab));
+        }
+        const float nb = -(PV8 ? (m_new - kLog2Fp8Max + (float)p.lazy_tau) : m_new);
+        // FP8 P~V, two query tiles: their exponential phases take turns (tile
+        // 0's of KV tile j, then tile 1's, then tile 0's of j+1, ...; over the
+        // items of the CTA one after the other), so that each runs at the
+        // MUFU's full rate while the other warpgroup does its maximum and O
+        // rescale.  A phase waits for the one before it in that order when the
+        // other warpgroup ran it, and hands over when the next one is the other's.
+        bool give_turn = false;
+        if (PV8 && NQ == 2) {
+          bool wait_turn;
+          const uint32_t prev_last = (ph / PH_LAST0) & 3;
+          if (q == 0) {
+            wait_turn = j > 0 ? (j - 1 < it.n[1]) : (prev_last == 1);
+            give_turn = j < it.n[1] || (j + 1 >= it.n[0] && next_first == 1);
+          } else {
+            wait_turn = j < it.n[0] || (j == 0 && prev_last == 0);
+            give_turn = j + 1 < it.n[0] || (j + 1 >= it.n[1] && next_first == 0);
+          }
+          if (wait_turn) {
+            if (!(ok = mbar_wait(bar(C::B_TOK + q), (ph / PH_TOK) & 1, abort_flag, p.err, kErrTimeoutSoftmax))) break;
+            ph ^= PH_TOK;
+          }
+        }
+        const float lt = tile_exp_store<PV8, KPT, BF16P, SMQ>(r, c, nb, p_smem, t);
+        if (PV8 && NQ == 2 && give_turn) mbar_arrive(bar(C::B_TOK + (q ^ 1)));
+        l = alpha * l + lt;
+        m = m_new;
+        if (C::NPB == 2 && j > 0) {
+          if (!(ok = mbar_wait(bar(C::B_OFULL + q), ((ph / PH_PV) & 1) ^ 1, abort_flag, p.err, kErrTimeoutSoftmax)))
+            break;
+          tc_fence_after();
+        }
+        if (!ACC2 && j > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+          // O(q) holds the sums of tiles < j
+          if (D == 128) {
+            uint32_t o[128];
+            tmem_ld128_sync(ob, o);
 #pragma unroll
-          for (int ch = 0; ch < D / 32; ++ch) {
-            uint32_t o[32];
-            tmem_ld32(ob + ch * 32, o);
-            tmem_wait_ld(o);
-#pragma unroll
-            for (int u = 0; u < 32; u += 2) {
+            for (int u = 0; u < 128; u += 2) {
               float x0, x1;
               mul2(x0, x1, __uint_as_float(o[u]), __uint_as_float(o[u + 1]), alpha, alpha);
               o[u] = __float_as_uint(x0);
               o[u + 1] = __float_as_uint(x1);
             }
-            tmem_st32(ob + ch * 32, o);
+            tmem_st128(ob, o);
+          } else {
+#pragma unroll
+            for (int ch = 0; ch < D / 32; ++ch) {
+              uint32_t o[32];
+              tmem_ld32(ob + ch * 32, o);
+              tmem_wait_ld(o);
+#pragma unroll
+              for (int u = 0; u < 32; u += 2) {
+                float x0, x1;
+                mul2(x0, x1, __uint_as_float(o[u]), __uint_as_float(o[u + 1]), alpha, alpha);
+                o[u] = __float_as_uint(x0);
+                o[u + 1] = __float_as_uint(x1);
+              }
+              tmem_st32(ob + ch * 32, o);
+            }
           }
         }
+        tmem_wait_st();
+        fence_proxy_async_smem();
+        tc_fence_before();
+        mbar_arrive(bar(C::B_PFULL + q));
+        ph = (ph ^ PH_PV) | PH_PVANY;
       }
-      tmem_wait_st();
-      fence_proxy_async_smem();
-      tc_fence_before();
-      mbar_arrive(bar(C::B_PFULL + q));
+      if (!ok) break;
     }
-  }
-  if (ACC2) {
-    l_s[q * 128 + t] = l;
-    mbar_arrive(bar(C::B_LFULL + q));
-  } else if (ok && qt * kTile < Lq) {
-    // epilogue of this query tile
-    if (n[q] > 0) {
-      ok = mbar_wait(bar(C::B_OFULL + q), (n[q] - 1) & 1, abort_flag, p.err, kErrTimeoutSoftmax);
-      tc_fence_after();
+    if (!PV8 && NQ == 2 && q == 1 && it.n[0] > 0) ph ^= PH_GO;   // tile 0 signals once per item
+    if (it.maxn > 0) {
+      kvbase += it.maxn;
+      ph = (ph & ~(3u * PH_LAST0)) | ((it.n[NQ - 1] == it.maxn ? NQ - 1u : 0u) * PH_LAST0);
     }
-    if (ok) {
-      uint16_t* orow = reinterpret_cast<uint16_t*>(p.out) + (long long)b * p.os.sb + (long long)h * p.os.sh +
-                       (long long)(qs + row) * p.os.ss;
-      store_row<D, PV8, false>(orow, ob, nullptr, l > 0.f ? 1.0f / l : 0.f, vsc, vmu, bf16, n[q] > 0, row < Lq);
+    if (ACC2) {
+      if (nq > 0) {
+        // the correction warpgroup has read the previous item's l
+        if ((ph & PH_LANY) &&
+            !(ok = mbar_wait(bar(C::B_LEMPTY + q), ((ph / PH_L) & 1) ^ 1, abort_flag, p.err, kErrTimeoutSoftmax)))
+          break;
+        l_s[q * 128 + t] = l;
+        mbar_arrive(bar(C::B_LFULL + q));
+        ph = (ph ^ PH_L) | PH_LANY;
+      }
+    } else if (qt * kTile < it.Lq) {
+      // epilogue of this query tile; the MMA already runs the next item's
+      // first QK^T meanwhile
+      if (nq > 0) {
+        if (!(ok = mbar_wait(bar(C::B_OFULL + q), ((ph / PH_PV) & 1) ^ 1, abort_flag, p.err, kErrTimeoutSoftmax)))
+          break;
+        tc_fence_after();
+      }
+      // the item's output coordinates, recomputed here rather than kept in
+      // registers through the tile loop
+      Item<NQ> io;
+      decode_item<NQ>(p, opaque(idx), io);
+      const float* vsc = p.v_scale + ((size_t)io.b * p.Hkv + io.hk) * D;
+      const float* vmu = p.v_mean ? p.v_mean + ((size_t)io.b * p.Hkv + io.hk) * D : nullptr;
+      uint16_t* orow = reinterpret_cast<uint16_t*>(p.out) + (long long)io.b * p.os.sb + (long long)io.h * p.os.sh +
+                       (long long)(io.qs + row) * p.os.ss;
+      store_row<D, PV8, false>(orow, ob, nullptr, l > 0.f ? 1.0f / l : 0.f, vsc, vmu, bf16, nq > 0, row < io.Lq);
     }
   }
 }
@@ -454,34 +588,12 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
   float* l_s = reinterpret_cast<float*>(smem + C::OFF_L);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int b = blockIdx.z, h = blockIdx.y;
-  const int pair = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
-  int qs, Lq, tq0, ks, Lk, tk0;
-  p.seqs.q(b, qs, Lq, tq0);
-  p.seqs.k(b, ks, Lk, tk0);
-  if (p.seqs.cu_q && (Lq > p.seqs.max_seqlen || Lk > p.seqs.max_seqlen || Lq < 0 || Lk < 0)) return;
-  if (pair * NQ * kTile >= Lq) return;             // uniform: before any setup
-  const int hk = h / p.group;
-  const int nk = (Lk + kTile - 1) / kTile;
-  int n[NQ];
-  int maxn = 0;
-#pragma unroll
-  for (int q = 0; q < NQ; ++q) {
-    const int qt = pair * NQ + q;
-    const bool valid = qt * kTile < Lq;
-    n[q] = !valid ? 0 : (p.causal ? min(nk, qt + 1) : nk);
-    maxn = max(maxn, n[q]);
-  }
-  // the workspace must hold every tile this CTA reads (varlen: the offsets
-  // kernel has already flagged an overflow)
-  if (tq0 + (Lq + kTile - 1) / kTile > p.tiles_q || tk0 + nk > p.tiles_k) return;
-
   if (tid == 0) {
     for (int i = 0; i < C::NBAR; ++i) {
       uint32_t cnt = 1;
       if ((i >= C::B_SCONS && i < C::B_SCONS + NQ) || (i >= C::B_PFULL && i < C::B_PFULL + NQ) ||
           (i >= C::B_OREADY && i < C::B_OREADY + NQ) || (i >= C::B_AFULL && i < C::B_AFULL + 4 * NQ) ||
-          (i >= C::B_LFULL && i < C::B_LFULL + NQ) || i == C::B_TOK || i == C::B_TOK + 1 || i == C::B_GO)
+          (i >= C::B_LFULL && i < C::B_LFULL + 2 * NQ) || i == C::B_TOK || i == C::B_TOK + 1 || i == C::B_GO)
         cnt = 128;
       mbar_init(bar(i), cnt);
     }
@@ -496,39 +608,66 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = misc[0];
-  const float* vsc = p.v_scale + ((size_t)b * p.Hkv + hk) * D;
-  const float* vmu = p.v_mean ? p.v_mean + ((size_t)b * p.Hkv + hk) * D : nullptr;
 
+  // Register split: the loader / MMA warpgroup gives registers to the two
+  // compute warpgroups (softmax, softmax or correction), whose tile loops run
+  // at the limit.  There is one release (warpgroup 0, first thing, never
+  // waits) and one request per compute warpgroup, and they add up exactly to
+  // the launch's 384 x 168 (the host checks that the kernel was built with
+  // 168), so every request is met once warpgroup 0 has released.  Nothing
+  // gives registers back: the two sides end the CTA separately, through a
+  // named barrier, so their register budgets never meet again.
+  if (warp < 4) {
+    setmaxnreg_dec<C::REGS_LOAD>();
   if (warp == 0) {
     // ------------------------------------------------------------ loader
+    // Per item: the Q tiles (once the MMA has finished the previous item's
+    // QK^T with them), then K_t, V_t (+ smooth-Q corrections) for every KV
+    // tile through the NST-stage ring, whose index runs on across items.
     if (lane == 0) {
-      const int8_t* qb = p.q_codes + ((size_t)h * p.tiles_q + tq0 + pair * NQ) * C::QT;
-      for (int q = 0; q < NQ; ++q)
-        if (n[q] > 0) {
+      bool ok = true;
+      int kv = 0, issued_k = 0, issued_v = 0;
+      uint32_t q_loads = 0;   // bit q: parity of Q loads of query tile q so far
+      uint32_t q_any = 0;     // bit q: Q tile q was loaded at least once
+      for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
+        Item<NQ> it;
+        if (!decode_item<NQ>(p, idx, it) || it.maxn == 0) continue;
+        const int8_t* qb = p.q_codes + ((size_t)it.h * p.tiles_q + it.tq0 + it.pair * NQ) * C::QT;
+        for (int q = 0; q < NQ && ok; ++q) {
+          if (it.n[q] == 0) continue;
+          if (((q_any >> q) & 1) &&
+              !(ok = mbar_wait_poll(bar(C::B_QEMPTY + q), ((q_loads >> q) & 1) ^ 1, abort_flag, p.err, kErrTimeoutLoad)))
+            break;
           mbar_expect_tx(bar(C::B_QFULL + q), C::QT);
           bulk_g2s(sb + C::OFF_Q + q * C::QT, qb + (size_t)q * C::QT, C::QT, bar(C::B_QFULL + q));
+          q_loads ^= 1u << q;
+          q_any |= 1u << q;
         }
-      const int8_t* kb = p.k_codes + ((size_t)hk * p.tiles_k + tk0) * C::QT;
-      const uint8_t* vb = p.v_codes + ((size_t)hk * p.tiles_k + tk0) * (size_t)C::VT;
-      // smooth Q: bias rows of the valid query tiles (n[q] > 0 for a prefix of q)
-      int nbias = 0;
-      if (p.q_bias)
-        for (int q = 0; q < NQ; ++q) nbias += n[q] > 0;
-      const float* bias_b = p.q_bias ? p.q_bias + ((size_t)h * p.tiles_q + tq0 + pair * NQ) * p.bias_ld : nullptr;
-      int issued_k = 0, issued_v = 0;
-      for (int t = 0; t < maxn; ++t) {
-        const int st = t % NST, u = t / NST;
-        if (u > 0 && !mbar_wait_poll(bar(C::B_KEMPTY + st), (u - 1) & 1, abort_flag, p.err, kErrTimeoutLoad)) break;
-        mbar_expect_tx(bar(C::B_KFULL + st), C::QT);
-        bulk_g2s(sb + C::OFF_K + st * C::QT, kb + (size_t)t * C::QT, C::QT, bar(C::B_KFULL + st));
-        issued_k = t + 1;
-        if (u > 0 && !mbar_wait_poll(bar(C::B_VEMPTY + st), (u - 1) & 1, abort_flag, p.err, kErrTimeoutLoad)) break;
-        mbar_expect_tx(bar(C::B_VFULL + st), C::VT + nbias * 512);
-        bulk_g2s(sb + C::OFF_V + st * C::VT, vb + (size_t)t * C::VT, C::VT, bar(C::B_VFULL + st));
-        for (int q = 0; q < nbias; ++q)     // smooth Q: the query tiles' corrections for key tile t
-          bulk_g2s(sb + C::OFF_BIAS + (st * NQ + q) * 512, bias_b + (size_t)q * p.bias_ld + (size_t)t * kTile, 512,
-                   bar(C::B_VFULL + st));
-        issued_v = t + 1;
+        if (!ok) break;
+        const int8_t* kb = p.k_codes + ((size_t)it.hk * p.tiles_k + it.tk0) * C::QT;
+        const uint8_t* vb = p.v_codes + ((size_t)it.hk * p.tiles_k + it.tk0) * (size_t)C::VT;
+        // smooth Q: bias rows of the valid query tiles (n[q] > 0 for a prefix of q)
+        int nbias = 0;
+        if (p.q_bias)
+          for (int q = 0; q < NQ; ++q) nbias += it.n[q] > 0;
+        const float* bias_b =
+            p.q_bias ? p.q_bias + ((size_t)it.h * p.tiles_q + it.tq0 + it.pair * NQ) * p.bias_ld : nullptr;
+        for (int t = 0; t < it.maxn; ++t, ++kv) {
+          const int st = kv % NST, u = kv / NST;
+          if (u > 0 && !(ok = mbar_wait_poll(bar(C::B_KEMPTY + st), (u - 1) & 1, abort_flag, p.err, kErrTimeoutLoad)))
+            break;
+          mbar_expect_tx(bar(C::B_KFULL + st), C::QT);
+          bulk_g2s(sb + C::OFF_K + st * C::QT, kb + (size_t)t * C::QT, C::QT, bar(C::B_KFULL + st));
+          issued_k = kv + 1;
+          if (u > 0 && !(ok = mbar_wait_poll(bar(C::B_VEMPTY + st), (u - 1) & 1, abort_flag, p.err, kErrTimeoutLoad)))
+            break;
+          mbar_expect_tx(bar(C::B_VFULL + st), C::VT + nbias * 512);
+          bulk_g2s(sb + C::OFF_V + st * C::VT, vb + (size_t)t * C::VT, C::VT, bar(C::B_VFULL + st));
+          for (int q = 0; q < nbias; ++q)   // smooth Q: the query tiles' corrections for key tile t
+            bulk_g2s(sb + C::OFF_BIAS + (st * NQ + q) * 512, bias_b + (size_t)q * p.bias_ld + (size_t)t * kTile, 512,
+                     bar(C::B_VFULL + st));
+          issued_v = kv + 1;
+        }
       }
       if (*abort_flag) {
         // let copies in flight land before the CTA's shared memory is released
@@ -541,23 +680,27 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
           while (!mbar_try_wait(bar(C::B_VFULL + t % NST), (t / NST) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {}
         }
         for (int q = 0; q < NQ; ++q)
-          if (n[q] > 0) {
+          if ((q_any >> q) & 1) {
             const uint64_t t0 = global_timer_ns();
-            while (!mbar_try_wait(bar(C::B_QFULL + q), 0) && global_timer_ns() - t0 < kWaitLimitNs) {}
+            while (!mbar_try_wait(bar(C::B_QFULL + q), ((q_loads >> q) & 1) ^ 1) &&
+                   global_timer_ns() - t0 < kWaitLimitNs) {}
           }
       }
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Per KV tile j: for each query tile, once the softmax has read S_j,
-    // S_{j+1} = Q K_{j+1}^T; then for each query tile, once P~_j is in shared
-    // memory (and, two-level, the last partial O was consumed), O (+)= P~_j V_j.
-    if (lane == 0 && maxn > 0) {
+    // Per KV tile j of an item: for each query tile, once the softmax has read
+    // S_j, S_{j+1} = Q K_{j+1}^T -- after the item's last tile, S_0 of the next
+    // item, so that it runs during this item's epilogue; then for each query
+    // tile, once P~_j is in shared memory (and, two-level, the last partial O
+    // was consumed), O (+)= P~_j V_j.
+    if (lane == 0) {
       constexpr uint32_t ID_QK = idesc_i8(128, 128);
       const uint32_t ID_PV = PV8 ? idesc_e4m3(128, D) : idesc_f16(128, D, p.out_bf16 != 0);
       bool ok = true;
-      for (int q = 0; q < NQ && ok; ++q)
-        if (n[q] > 0) ok = mbar_wait_poll(bar(C::B_QFULL + q), 0, abort_flag, p.err, kErrTimeoutMma);
+      int kvs = 0, kvp = 0;                  // ring index of the next K tile (QK^T) and V tile (PV)
+      uint32_t s_ph = 0, q_ph = 0, p_ph = 0;  // bit q: parity of S_j seeds, Q loads, P~ tiles consumed
+      uint32_t pv_any = 0;                    // bit q: a PV of query tile q was issued
       auto mma_s = [&](int q, int st) {
         const uint32_t d = tmem + C::TM_S + q * 128;
 #pragma unroll
@@ -586,53 +729,80 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
         }
         tc_commit(bar(C::B_OFULL + q));
       };
-      // S_0 (once the softmax warpgroups have seeded the S columns)
-      if (ok && (ok = mbar_wait_poll(bar(C::B_KFULL), 0, abort_flag, p.err, kErrTimeoutMma))) {
-        for (int q = 0; q < NQ && ok; ++q)
-          if (n[q] > 0 && (ok = mbar_wait_poll(bar(C::B_SCONS + q), 0, abort_flag, p.err, kErrTimeoutMma))) {
-            tc_fence_after();
-            mma_s(q, 0);
+      // S_t of item `it` for every query tile that has KV tile t
+      auto issue_s = [&](const Item<NQ>& it, int t) -> bool {
+        const int st = kvs % NST;
+        if (!mbar_wait_poll(bar(C::B_KFULL + st), (kvs / NST) & 1, abort_flag, p.err, kErrTimeoutMma)) return false;
+        for (int q = 0; q < NQ; ++q) {
+          if (t >= it.n[q]) continue;
+          if (t == 0) {
+            if (!mbar_wait_poll(bar(C::B_QFULL + q), (q_ph >> q) & 1, abort_flag, p.err, kErrTimeoutMma)) return false;
+            q_ph ^= 1u << q;
           }
-        tc_commit(bar(C::B_KEMPTY));
-      }
-      for (int j = 0; j < maxn && ok; ++j) {
-        const int st = j % NST, t = j + 1;
-        // next QK^T as soon as each softmax has read S_j
-        if (t < maxn) {
-          if (!(ok = mbar_wait_poll(bar(C::B_KFULL + t % NST), (t / NST) & 1, abort_flag, p.err, kErrTimeoutMma))) break;
-          for (int q = 0; q < NQ && ok; ++q) {
-            if (t >= n[q]) continue;
-            if (!(ok = mbar_wait_poll(bar(C::B_SCONS + q), t & 1, abort_flag, p.err, kErrTimeoutMma))) break;
-            tc_fence_after();
-            mma_s(q, t % NST);
-          }
-          if (!ok) break;
-          tc_commit(bar(C::B_KEMPTY + t % NST));
-        }
-        if (!(ok = mbar_wait_poll(bar(C::B_VFULL + st), (j / NST) & 1, abort_flag, p.err, kErrTimeoutMma))) break;
-        for (int q = 0; q < NQ && ok; ++q) {
-          if (j >= n[q]) continue;
-          ok = mbar_wait_poll(bar(C::B_PFULL + q), j & 1, abort_flag, p.err, kErrTimeoutMma);
-          if (ok && ACC2 && j > 0)
-            ok = mbar_wait_poll(bar(C::B_OREADY + q), (j - 1) & 1, abort_flag, p.err, kErrTimeoutMma);
-          if (!ok) break;
+          if (!mbar_wait_poll(bar(C::B_SCONS + q), (s_ph >> q) & 1, abort_flag, p.err, kErrTimeoutMma)) return false;
+          s_ph ^= 1u << q;
           tc_fence_after();
-          mma_pv(q, j, st);
+          mma_s(q, st);
+          if (t == it.n[q] - 1) tc_commit(bar(C::B_QEMPTY + q));   // the Q tile may be replaced
         }
-        if (!ok) break;
-        tc_commit(bar(C::B_VEMPTY + st));
+        tc_commit(bar(C::B_KEMPTY + st));
+        ++kvs;
+        return true;
+      };
+      bool s0_issued = false;
+      for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
+        Item<NQ> it;
+        if (!decode_item<NQ>(p, idx, it) || it.maxn == 0) continue;
+        if (!s0_issued && !(ok = issue_s(it, 0))) break;
+        s0_issued = false;
+        for (int j = 0; j < it.maxn; ++j) {
+          if (j + 1 < it.maxn) {
+            if (!(ok = issue_s(it, j + 1))) break;
+          } else {
+            Item<NQ> nx;
+            if (next_busy_item<NQ>(p, idx, nx)) {
+              if (!(ok = issue_s(nx, 0))) break;
+              s0_issued = true;
+            }
+          }
+          const int st = kvp % NST;
+          if (!(ok = mbar_wait_poll(bar(C::B_VFULL + st), (kvp / NST) & 1, abort_flag, p.err, kErrTimeoutMma))) break;
+          for (int q = 0; q < NQ && ok; ++q) {
+            if (j >= it.n[q]) continue;
+            ok = mbar_wait_poll(bar(C::B_PFULL + q), (p_ph >> q) & 1, abort_flag, p.err, kErrTimeoutMma);
+            if (ok && ACC2 && ((pv_any >> q) & 1))
+              ok = mbar_wait_poll(bar(C::B_OREADY + q), ((p_ph >> q) & 1) ^ 1, abort_flag, p.err, kErrTimeoutMma);
+            if (!ok) break;
+            p_ph ^= 1u << q;
+            pv_any |= 1u << q;
+            tc_fence_after();
+            mma_pv(q, j, st);
+          }
+          if (!ok) break;
+          tc_commit(bar(C::B_VEMPTY + st));
+          ++kvp;
+        }
       }
       // all MMAs issued by this thread complete before teardown
       tc_commit(bar(C::B_DONE));
       const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(bar(C::B_DONE), 0) && global_timer_ns() - t0 < kWaitLimitNs) {}
     }
-  } else if (warp >= 4 && warp < 4 + 4 * NQ) {
+  }
+    __syncwarp();
+    tc_fence_before();
+    named_bar_sync(1, C::NTHREADS);          // every role has finished
+    if (warp == 2) {
+      tc_fence_after();
+      tmem_dealloc(tmem, C::TM_COLS);
+    }
+  } else {
+    setmaxnreg_inc<C::REGS_COMPUTE>();
+  if (warp < 4 + 4 * NQ) {
     // ------------------------------------------------------------ softmax
     const bool bf16p = !PV8 && p.out_bf16;
     const int variant = (p.gran == 2 ? 4 : 0) + (bf16p ? 2 : 0) + (p.q_bias ? 1 : 0);
-#define SAGE_SOFTMAX(KPT, BF16P, SMQ) \
-  softmax_role<D, PV8, ACC2, KPT, BF16P, SMQ>(p, sb, tmem, warp, tid, pair, b, h, hk, qs, Lq, Lk, tq0, tk0, n, vsc, vmu)
+#define SAGE_SOFTMAX(KPT, BF16P, SMQ) softmax_role<D, PV8, ACC2, KPT, BF16P, SMQ>(p, sb, tmem, warp, tid)
     switch (variant) {
       case 0: SAGE_SOFTMAX(false, false, false); break;
       case 1: SAGE_SOFTMAX(false, false, true); break;
@@ -644,56 +814,63 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
       default: SAGE_SOFTMAX(true, true, true); break;
     }
 #undef SAGE_SOFTMAX
-  } else if (ACC2 && warp >= 4 + 4 * NQ) {
+  } else if (ACC2) {
     // ------------------------------------------------------------ correction (two-level) + epilogue
     const int t = tid - 128 * (1 + NQ);
     const uint32_t lane_off = (uint32_t)((t & ~31)) << 16;
     const uint32_t ob = tmem + C::TM_O + lane_off;
     bool ok = true;
-    float oacc[D];
+    int a_cnt = 0;
+    uint32_t o_ph = 0, l_ph = 0;
+    for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
+      Item<NQ> it;
+      if (!decode_item<NQ>(p, idx, it)) continue;
+      float oacc[D];
 #pragma unroll
-    for (int i = 0; i < D; ++i) oacc[i] = 0.f;
-    for (int j = 0; j < n[0] && ok; ++j) {
-      const int ab = j & 1;
-      if (!(ok = mbar_wait(bar(C::B_AFULL + ab), (j >> 1) & 1, abort_flag, p.err, kErrTimeoutCorr))) break;
-      const float alpha = alpha_s[ab * 128 + t];
-      mbar_arrive(bar(C::B_AEMPTY + ab));
-      if (!(ok = mbar_wait(bar(C::B_OFULL), j & 1, abort_flag, p.err, kErrTimeoutCorr))) break;
-      tc_fence_after();
+      for (int i = 0; i < D; ++i) oacc[i] = 0.f;
+      for (int j = 0; j < it.n[0]; ++j) {
+        const int ab = a_cnt & 1;
+        if (!(ok = mbar_wait(bar(C::B_AFULL + ab), (a_cnt >> 1) & 1, abort_flag, p.err, kErrTimeoutCorr))) break;
+        ++a_cnt;
+        const float alpha = alpha_s[ab * 128 + t];
+        mbar_arrive(bar(C::B_AEMPTY + ab));
+        if (!(ok = mbar_wait(bar(C::B_OFULL), o_ph, abort_flag, p.err, kErrTimeoutCorr))) break;
+        o_ph ^= 1;
+        tc_fence_after();
 #pragma unroll
-      for (int ch = 0; ch < D / 16; ++ch) {
-        uint32_t r[16];
-        tmem_ld16(ob + ch * 16, r);
-        tmem_wait_ld(r);
+        for (int ch = 0; ch < D / 16; ++ch) {
+          uint32_t r[16];
+          tmem_ld16(ob + ch * 16, r);
+          tmem_wait_ld(r);
 #pragma unroll
-        for (int u = 0; u < 16; u += 2)
-          fma2(oacc[ch * 16 + u], oacc[ch * 16 + u + 1], alpha, alpha, oacc[ch * 16 + u], oacc[ch * 16 + u + 1],
-               __uint_as_float(r[u]), __uint_as_float(r[u + 1]));
+          for (int u = 0; u < 16; u += 2)
+            fma2(oacc[ch * 16 + u], oacc[ch * 16 + u + 1], alpha, alpha, oacc[ch * 16 + u], oacc[ch * 16 + u + 1],
+                 __uint_as_float(r[u]), __uint_as_float(r[u + 1]));
+        }
+        tc_fence_before();
+        mbar_arrive(bar(C::B_OREADY));
       }
-      tc_fence_before();
-      mbar_arrive(bar(C::B_OREADY));
-    }
-    const int row = pair * kTile + t;
-    if (ok && pair * kTile < Lq) {
+      if (!ok) break;
+      const int row = it.pair * kTile + t;
       float l = 0.f;
-      if (n[0] > 0) {
-        ok = mbar_wait(bar(C::B_LFULL), 0, abort_flag, p.err, kErrTimeoutCorr);
+      if (it.n[0] > 0) {
+        if (!(ok = mbar_wait(bar(C::B_LFULL), l_ph, abort_flag, p.err, kErrTimeoutCorr))) break;
+        l_ph ^= 1;
         l = l_s[t];
+        mbar_arrive(bar(C::B_LEMPTY));
       }
-      if (ok) {
-        uint16_t* orow = reinterpret_cast<uint16_t*>(p.out) + (long long)b * p.os.sb + (long long)h * p.os.sh +
-                         (long long)(qs + row) * p.os.ss;
-        store_row<D, PV8, true>(orow, ob, oacc, l > 0.f ? 1.0f / l : 0.f, vsc, vmu, p.out_bf16 != 0, true,
-                                row < Lq);
-      }
+      const float* vsc = p.v_scale + ((size_t)it.b * p.Hkv + it.hk) * D;
+      const float* vmu = p.v_mean ? p.v_mean + ((size_t)it.b * p.Hkv + it.hk) * D : nullptr;
+      uint16_t* orow = reinterpret_cast<uint16_t*>(p.out) + (long long)it.b * p.os.sb + (long long)it.h * p.os.sh +
+                       (long long)(it.qs + row) * p.os.ss;
+      store_row<D, PV8, true>(orow, ob, oacc, l > 0.f ? 1.0f / l : 0.f, vsc, vmu, p.out_bf16 != 0, true,
+                              row < it.Lq);
     }
   }
 
-  tc_fence_before();
-  __syncthreads();
-  if (warp == 2) {
-    tc_fence_after();
-    tmem_dealloc(tmem, C::TM_COLS);
+    __syncwarp();
+    tc_fence_before();
+    named_bar_sync(1, C::NTHREADS);
   }
   (void)alpha_s;
   (void)l_s;
@@ -760,13 +937,24 @@ __global__ void __launch_bounds__(128, 1) qk_tile_kernel(const int8_t* qt, const
 
 
 // ---------------------------------------------------------------- launchers
+// Persistent grid: one CTA per SM (each holds all of an SM's tensor memory),
+// fewer when there are fewer items.
 template <int D, bool PV8, bool ACC2>
-static cudaError_t launch_attn(const AttnParams& p, int n_pairs_x, int nseq, cudaStream_t s) {
+static cudaError_t launch_attn(const AttnParams& p, cudaStream_t s) {
   using C = AttnCfg<D, PV8, ACC2>;
   auto k = attn_fwd_kernel<D, PV8, ACC2>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
-  k<<<dim3(n_pairs_x, p.Hq, nseq), C::NTHREADS, C::SMEM_BYTES, s>>>(p);
+  // the register split needs the launch allocation it was sized for: with
+  // fewer registers a warpgroup's setmaxnreg.inc would wait for ever
+  cudaFuncAttributes fa;
+  if ((e = cudaFuncGetAttributes(&fa, k)) != cudaSuccess) return e;
+  if (fa.numRegs != C::REGS_LAUNCH) return cudaErrorInvalidConfiguration;
+  int dev = 0, sms = 0;
+  if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+  if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  const int grid = p.n_items < sms ? p.n_items : sms;
+  k<<<grid, C::NTHREADS, C::SMEM_BYTES, s>>>(p);
   return cudaGetLastError();
 }
 
@@ -776,17 +964,23 @@ int attn_tiles_per_cta(int D, bool pv8, bool acc2) {
   return acc2 ? 1 : 2;
 }
 
-cudaError_t attn_forward(const AttnParams& p, int D, bool pv8, bool acc2, int max_len_q, int nseq,
+cudaError_t attn_forward(const AttnParams& p0, int D, bool pv8, bool acc2, int max_len_q, int nseq,
                          cudaStream_t s) {
   const int per = attn_tiles_per_cta(D, pv8, acc2) * kTile;
-  const int nx = (max_len_q + per - 1) / per;
-  if (nx == 0 || nseq == 0) return cudaSuccess;
+  const long long nx = (max_len_q + per - 1) / per;
+  const long long items = nx * p0.Hq * nseq;
+  if (items == 0) return cudaSuccess;
+  if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
+  AttnParams p = p0;
+  p.n_pairs = (int)nx;
+  p.nseq = nseq;
+  p.n_items = (int)items;
   if (D == 128) {
-    if (pv8) return acc2 ? launch_attn<128, true, true>(p, nx, nseq, s) : launch_attn<128, true, false>(p, nx, nseq, s);
-    return acc2 ? launch_attn<128, false, true>(p, nx, nseq, s) : launch_attn<128, false, false>(p, nx, nseq, s);
+    if (pv8) return acc2 ? launch_attn<128, true, true>(p, s) : launch_attn<128, true, false>(p, s);
+    return acc2 ? launch_attn<128, false, true>(p, s) : launch_attn<128, false, false>(p, s);
   }
-  if (pv8) return acc2 ? launch_attn<64, true, true>(p, nx, nseq, s) : launch_attn<64, true, false>(p, nx, nseq, s);
-  return acc2 ? launch_attn<64, false, true>(p, nx, nseq, s) : launch_attn<64, false, false>(p, nx, nseq, s);
+  if (pv8) return acc2 ? launch_attn<64, true, true>(p, s) : launch_attn<64, true, false>(p, s);
+  return acc2 ? launch_attn<64, false, true>(p, s) : launch_attn<64, false, false>(p, s);
 }
 
 cudaError_t debug_qk_tile(const int8_t* qt, const int8_t* kt, int D, int32_t* out, uint32_t* err,

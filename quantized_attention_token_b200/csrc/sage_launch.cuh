@@ -56,6 +56,7 @@ struct AttnParams {
   int lazy_tau;              // conditional rescaling: the reference maximum moves only past +tau (0: always)
   int causal;
   int out_bf16;
+  int n_pairs, nseq, n_items;  // work items: n_pairs query-tile groups x Hq heads x nseq sequences (set by attn_forward)
 };
 
 // prepass.cu
