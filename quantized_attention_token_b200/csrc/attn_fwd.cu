@@ -277,6 +277,62 @@ __device__ __forceinline__ void store_row(uint16_t* orow, uint32_t ob, const flo
   }
 }
 
+// One-level epilogue of one warp's 32 rows (its quarter of the TMEM lanes):
+// out = O * 1/l (* delta_V[c] in FP8 mode, + the channel mean with smooth V),
+// rounded to 16 bits.  Each thread puts its row in shared memory, in 16-byte
+// chunks XOR-swizzled by row, and then the warp writes whole rows: one store
+// instruction covers 512 contiguous bytes of two (D = 128) or four (D = 64)
+// rows.  Rows 0-15 are staged at stage0, rows 16-31 at stage1, each 16 x 2D
+// bytes: the warp's own rows of the query tile's two P~ halves, which only
+// this warp writes next.
+template <int D, bool PV8>
+__device__ __forceinline__ void store_tile(uint16_t* orow0, long long ss, int nvalid, uint32_t stage0, uint32_t stage1,
+                                           uint32_t ob, float inv_l, const float* vsc, const float* vmu, bool bf16,
+                                           bool have_o, int lane) {
+  constexpr int RB = 2 * D;       // bytes of an output row
+  constexpr int CH = RB / 16;     // 16-byte chunks per row
+  constexpr int RPI = 32 / CH;    // rows per warp store instruction
+  const uint32_t my_row = (lane < 16 ? stage0 : stage1) + (lane & 15) * RB;
+#pragma unroll
+  for (int ch = 0; ch < D / 32; ++ch) {
+    uint32_t r[32];
+    if (have_o) {
+      tmem_ld32(ob + ch * 32, r);
+      tmem_wait_ld(r);
+    }
+    uint32_t w[16];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {                    // four columns
+      float a[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) a[e] = (have_o ? __uint_as_float(r[4 * u + e]) : 0.f) * inv_l;
+      if (PV8) {
+        const float4 sc = __ldg(reinterpret_cast<const float4*>(vsc + ch * 32) + u);
+        a[0] *= sc.x; a[1] *= sc.y; a[2] *= sc.z; a[3] *= sc.w;
+        if (vmu) {                                   // smooth V: the channel mean comes back
+          const float4 mu = __ldg(reinterpret_cast<const float4*>(vmu + ch * 32) + u);
+          a[0] += mu.x; a[1] += mu.y; a[2] += mu.z; a[3] += mu.w;
+        }
+      }
+      w[2 * u] = bf16 ? pack_bf16x2(a[0], a[1]) : pack_f16x2(a[0], a[1]);
+      w[2 * u + 1] = bf16 ? pack_bf16x2(a[2], a[3]) : pack_f16x2(a[2], a[3]);
+    }
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk) {
+      const int k = ch * 4 + kk;
+      st_shared_v4(my_row + ((k ^ (lane & (CH - 1))) << 4), w[4 * kk], w[4 * kk + 1], w[4 * kk + 2], w[4 * kk + 3]);
+    }
+  }
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < 32 / RPI; ++i) {
+    const int rr = i * RPI + lane / CH, k = lane % CH;
+    const uint4 v = ld_shared_v4((rr < 16 ? stage0 : stage1) + (rr & 15) * RB + ((k ^ (rr & (CH - 1))) << 4));
+    if (rr < nvalid) *reinterpret_cast<uint4*>(orow0 + rr * ss + k * 8) = v;
+  }
+  __syncwarp();
+}
+
 // ---------------------------------------------------------------- work items
 // A copy of x that the compiler cannot see through, so that values derived
 // from it are recomputed instead of kept live.
@@ -538,6 +594,24 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
       if (!ok) break;
     }
     if (!PV8 && NQ == 2 && q == 1 && it.n[0] > 0) ph ^= PH_GO;   // tile 0 signals once per item
+    if (!ACC2 && PV8) {
+      // this item's V scales (and means) for the epilogue, into L1
+      const size_t vo = ((size_t)it.b * p.Hkv + it.hk) * D;
+#pragma unroll
+      for (int c = 0; c < D; c += 32) {
+        prefetch_l1(p.v_scale + vo + c);
+        if (p.v_mean) prefetch_l1(p.v_mean + vo + c);
+      }
+    }
+    if (!ACC2) {
+      // the next item's Q and K scales, into L1 during the epilogue (in
+      // two-level mode the extra work in the softmax costs more than it saves)
+      Item<NQ> nx;
+      if (next_busy_item<NQ>(p, opaque(idx), nx) && nx.n[q] > 0) {
+        prefetch_l1(p.q_scale + ((size_t)nx.h * p.tiles_q + nx.tq0 + nx.pair * NQ + q) * kQGroupsMax + q_group(p.gran, t));
+        prefetch_l1(p.k_scale + ((size_t)nx.hk * p.tiles_k + nx.tk0) * kKGroupsMax);
+      }
+    }
     if (it.maxn > 0) {
       kvbase += it.maxn;
       ph = (ph & ~(3u * PH_LAST0)) | ((it.n[NQ - 1] == it.maxn ? NQ - 1u : 0u) * PH_LAST0);
@@ -566,9 +640,15 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
       decode_item<NQ>(p, opaque(idx), io);
       const float* vsc = p.v_scale + ((size_t)io.b * p.Hkv + io.hk) * D;
       const float* vmu = p.v_mean ? p.v_mean + ((size_t)io.b * p.Hkv + io.hk) * D : nullptr;
-      uint16_t* orow = reinterpret_cast<uint16_t*>(p.out) + (long long)io.b * p.os.sb + (long long)io.h * p.os.sh +
-                       (long long)(io.qs + row) * p.os.ss;
-      store_row<D, PV8, false>(orow, ob, nullptr, l > 0.f ? 1.0f / l : 0.f, vsc, vmu, bf16, nq > 0, row < io.Lq);
+      const int w = t >> 5, row0 = qt * kTile + 32 * w;
+      uint16_t* orow0 = reinterpret_cast<uint16_t*>(p.out) + (long long)io.b * p.os.sb + (long long)io.h * p.os.sh +
+                        (long long)(io.qs + row0) * p.os.ss;
+      // staging: this warp's rows of the two P~ halves (FP8: the two buffers;
+      // 16-bit: the two 64-key halves of the one buffer)
+      const uint32_t half = C::NPB == 2 ? (uint32_t)(NQ * C::PT) : (uint32_t)(C::PT / 2);
+      const uint32_t stage0 = sb + C::OFF_P + q * C::PT + w * 4096;
+      store_tile<D, PV8>(orow0, p.os.ss, min(32, max(0, io.Lq - row0)), stage0, stage0 + half, ob,
+                         l > 0.f ? 1.0f / l : 0.f, vsc, vmu, bf16, nq > 0, t & 31);
     }
   }
 }
@@ -690,10 +770,11 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
     // Per KV tile j of an item: for each query tile, once the softmax has read
-    // S_j, S_{j+1} = Q K_{j+1}^T -- after the item's last tile, S_0 of the next
-    // item, so that it runs during this item's epilogue; then for each query
-    // tile, once P~_j is in shared memory (and, two-level, the last partial O
-    // was consumed), O (+)= P~_j V_j.
+    // S_j, S_{j+1} = Q K_{j+1}^T; then for each query tile, once P~_j is in
+    // shared memory (and, two-level, the last partial O was consumed),
+    // O (+)= P~_j V_j.  S_0 of the next item comes right after the item's
+    // last PV (one-level) or before it (two-level) and runs during this item's
+    // epilogue.
     if (lane == 0) {
       constexpr uint32_t ID_QK = idesc_i8(128, 128);
       const uint32_t ID_PV = PV8 ? idesc_e4m3(128, D) : idesc_f16(128, D, p.out_bf16 != 0);
@@ -758,7 +839,9 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
         for (int j = 0; j < it.maxn; ++j) {
           if (j + 1 < it.maxn) {
             if (!(ok = issue_s(it, j + 1))) break;
-          } else {
+          } else if (ACC2) {
+            // two-level: the last PV waits for the correction warpgroup, so
+            // the next item's first QK^T goes ahead of it
             Item<NQ> nx;
             if (next_busy_item<NQ>(p, idx, nx)) {
               if (!(ok = issue_s(nx, 0))) break;
@@ -781,6 +864,16 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
           if (!ok) break;
           tc_commit(bar(C::B_VEMPTY + st));
           ++kvp;
+          if (!ACC2 && j + 1 == it.maxn) {
+            // one-level: the next item's first QK^T after this item's last PV
+            // (which need not wait for the next Q tile); it runs during the
+            // epilogue
+            Item<NQ> nx;
+            if (next_busy_item<NQ>(p, idx, nx)) {
+              if (!(ok = issue_s(nx, 0))) break;
+              s0_issued = true;
+            }
+          }
         }
       }
       // all MMAs issued by this thread complete before teardown
@@ -825,6 +918,15 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
     for (int idx = blockIdx.x; idx < p.n_items && ok; idx += gridDim.x) {
       Item<NQ> it;
       if (!decode_item<NQ>(p, idx, it)) continue;
+      if (PV8) {
+        // the item's V scales (and means) for the epilogue, into L1
+        const size_t vo = ((size_t)it.b * p.Hkv + it.hk) * D;
+#pragma unroll
+        for (int c = 0; c < D; c += 32) {
+          prefetch_l1(p.v_scale + vo + c);
+          if (p.v_mean) prefetch_l1(p.v_mean + vo + c);
+        }
+      }
       float oacc[D];
 #pragma unroll
       for (int i = 0; i < D; ++i) oacc[i] = 0.f;
