@@ -31,6 +31,8 @@
 // setmaxnreg (56 / 224 / 224 per thread).
 // Every mbarrier wait is bounded (sage_common.cuh): a wait that never ends sets
 // the device error word and the CTA tears down instead of hanging.
+#include <cstdlib>
+
 #include "sage_launch.cuh"
 
 namespace sage {
@@ -1055,6 +1057,12 @@ static cudaError_t launch_attn(const AttnParams& p, cudaStream_t s) {
   int dev = 0, sms = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+  // SAGE_MAX_CTAS caps the persistent grid (tests use it to make a few CTAs
+  // walk many items; results do not depend on it)
+  if (const char* cap = getenv("SAGE_MAX_CTAS")) {
+    const int c = atoi(cap);
+    if (c > 0 && c < sms) sms = c;
+  }
   const int grid = p.n_items < sms ? p.n_items : sms;
   k<<<grid, C::NTHREADS, C::SMEM_BYTES, s>>>(p);
   return cudaGetLastError();

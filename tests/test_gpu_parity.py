@@ -379,3 +379,60 @@ def test_one_level_accumulation_as_accurate_as_two_level(pv):
     e2 = float(np.mean(np.concatenate(errs["fp32+fp32"])))
     print(f"mean |gpu - oracle|: fp32 {e1:.3e}, fp32+fp32 {e2:.3e}")
     assert e1 <= 1.1 * e2 + 1e-7, (e1, e2)
+
+
+# ----------------------------------------------------------------------------- persistent grid
+@pytest.mark.parametrize("max_ctas", ["1", "3"])
+@pytest.mark.parametrize("D,S,causal,pv,acc,gran,dtype,layout", [
+    (128, 600, False, "fp8", "fp32", "per_block", "fp16", "HND"),
+    (128, 600, True, "fp8", "fp32", "per_warp", "bf16", "NHD"),
+    (64, 520, True, "fp16", "fp32", "per_block", "fp16", "HND"),
+    (128, 300, True, "fp8", "fp32+fp32", "per_thread", "fp16", "HND"),
+    (64, 700, False, "fp16", "fp32+fp32", "per_token", "bf16", "NHD"),
+])
+def test_persistent_items_match_oracle(monkeypatch, max_ctas, D, S, causal, pv, acc, gran, dtype, layout):
+    """A capped grid, so that each CTA walks many items one after the other:
+    the mbarrier phases, the K/V ring, the Q reloads and the FP8 token run on
+    across items, including tail items whose second query tile is empty."""
+    monkeypatch.setenv("SAGE_MAX_CTAS", max_ctas)
+    sp = synth.Spec("t", Hq=4, Hkv=2, D=D, B=2, S=S, dtype=dtype, layout=layout, causal=causal, k_bias_std=3.0,
+                    seed=120 + S)
+    q, k, v = synth.make(sp)
+    out = sage.sageattn(_dev(q), _dev(k), _dev(v), layout, causal, qk_quant_gran=gran, pv_dtype=pv,
+                        pv_accum_dtype=acc)
+    torch.cuda.synchronize()
+    ref = oracle.attention(q, k, v, layout, causal, gran=gran, pv=pv, with_allowance=True)
+    _assert_close(out, ref, dtype, f"{max_ctas} CTAs vs oracle")
+
+
+@pytest.mark.parametrize("pv,acc", [("fp8", "fp32"), ("fp16", "fp32"), ("fp8", "fp32+fp32")])
+def test_persistent_varlen_gqa_matches_oracle(monkeypatch, pv, acc):
+    """Two CTAs over the items of six sequences (one empty, one of a single
+    token), causal, grouped heads."""
+    monkeypatch.setenv("SAGE_MAX_CTAS", "2")
+    sp = synth.Spec("t", Hq=4, Hkv=2, D=128, seqlens=[200, 1, 0, 129, 384, 77], causal=True, seed=52)
+    q, k, v = synth.make(sp)
+    cu = sp.cu_seqlens()
+    cu_d = torch.from_numpy(cu).cuda()
+    out = sage.sageattn_varlen(_dev(q), _dev(k), _dev(v), cu_d, cu_d, max(sp.seqlens), True, pv_dtype=pv,
+                               pv_accum_dtype=acc)
+    torch.cuda.synchronize()
+    ref = oracle.attention(q, k, v, causal=True, pv=pv, cu_seqlens=cu, with_allowance=True)
+    _assert_close(out, ref, "fp16", "varlen, 2 CTAs")
+
+
+@pytest.mark.parametrize("acc", ["fp32", "fp32+fp32", "fp32_lazy"])
+def test_persistent_smooth_qv_matches_oracle(monkeypatch, acc):
+    """Smooth Q (its per-key corrections ride with each V tile through the
+    ring) and smooth V with one CTA walking all items."""
+    monkeypatch.setenv("SAGE_MAX_CTAS", "1")
+    sp = synth.Spec("t", Hq=4, Hkv=2, D=128, B=2, S=400, dtype="fp16", layout="HND", causal=False, k_bias_std=3.0,
+                    q_block_offset_std=1.0, seed=130)
+    q, k, v = synth.make(sp)
+    v = v + torch.from_numpy(np.random.default_rng(13).normal(0, 8, 128).astype(np.float32)).to(v.dtype)
+    out = sage.sageattn(_dev(q), _dev(k), _dev(v), "HND", False, pv_dtype="fp8", pv_accum_dtype=acc,
+                        smooth_q=True, smooth_v=True)
+    torch.cuda.synchronize()
+    ref = oracle.attention(q, k, v, "HND", False, pv="fp8", smooth_q=True, smooth_v=True,
+                           lazy_tau=2 if acc == "fp32_lazy" else 0, with_allowance=True)
+    _assert_close(out, ref, "fp16", "smooth Q+V, 1 CTA")
