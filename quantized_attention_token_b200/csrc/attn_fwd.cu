@@ -393,6 +393,13 @@ __device__ __forceinline__ bool decode_item(const AttnParams& p, int idx, Item<N
   return true;
 }
 
+// KV tiles of query tile q of an item, without indexing the array by a
+// run-time q (which would put the item in local memory).
+template <int NQ>
+__device__ __forceinline__ int item_n(const Item<NQ>& it, int q) {
+  return (NQ == 1 || q == 0) ? it.n[0] : it.n[NQ - 1];
+}
+
 // The next item after idx in this CTA's list that has KV tiles.
 template <int NQ>
 __device__ __forceinline__ bool next_busy_item(const AttnParams& p, int idx, Item<NQ>& it) {
@@ -443,7 +450,7 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
     if (!decode_item<NQ>(p, idx, it)) continue;
     const int qt = it.pair * NQ + q;
     const int row = qt * kTile + t;
-    const int nq = it.n[q];
+    const int nq = item_n<NQ>(it, q);
     // FP8 token: warpgroup of the next busy item's first exponential phase
     int next_first = -1;
     if (PV8 && NQ == 2 && it.maxn > 0) {
@@ -609,7 +616,7 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
       // the next item's Q and K scales, into L1 during the epilogue (in
       // two-level mode the extra work in the softmax costs more than it saves)
       Item<NQ> nx;
-      if (next_busy_item<NQ>(p, opaque(idx), nx) && nx.n[q] > 0) {
+      if (next_busy_item<NQ>(p, opaque(idx), nx) && item_n<NQ>(nx, q) > 0) {
         prefetch_l1(p.q_scale + ((size_t)nx.h * p.tiles_q + nx.tq0 + nx.pair * NQ + q) * kQGroupsMax + q_group(p.gran, t));
         prefetch_l1(p.k_scale + ((size_t)nx.hk * p.tiles_k + nx.tk0) * kKGroupsMax);
       }
@@ -715,7 +722,9 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
         Item<NQ> it;
         if (!decode_item<NQ>(p, idx, it) || it.maxn == 0) continue;
         const int8_t* qb = p.q_codes + ((size_t)it.h * p.tiles_q + it.tq0 + it.pair * NQ) * C::QT;
-        for (int q = 0; q < NQ && ok; ++q) {
+#pragma unroll
+        for (int q = 0; q < NQ; ++q) {
+          if (!ok) break;
           if (it.n[q] == 0) continue;
           if (((q_any >> q) & 1) &&
               !(ok = mbar_wait_poll(bar(C::B_QEMPTY + q), ((q_loads >> q) & 1) ^ 1, abort_flag, p.err, kErrTimeoutLoad)))
@@ -731,6 +740,7 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
         // smooth Q: bias rows of the valid query tiles (n[q] > 0 for a prefix of q)
         int nbias = 0;
         if (p.q_bias)
+#pragma unroll
           for (int q = 0; q < NQ; ++q) nbias += it.n[q] > 0;
         const float* bias_b =
             p.q_bias ? p.q_bias + ((size_t)it.h * p.tiles_q + it.tq0 + it.pair * NQ) * p.bias_ld : nullptr;
@@ -816,6 +826,7 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
       auto issue_s = [&](const Item<NQ>& it, int t) -> bool {
         const int st = kvs % NST;
         if (!mbar_wait_poll(bar(C::B_KFULL + st), (kvs / NST) & 1, abort_flag, p.err, kErrTimeoutMma)) return false;
+#pragma unroll
         for (int q = 0; q < NQ; ++q) {
           if (t >= it.n[q]) continue;
           if (t == 0) {
@@ -852,7 +863,9 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
           }
           const int st = kvp % NST;
           if (!(ok = mbar_wait_poll(bar(C::B_VFULL + st), (kvp / NST) & 1, abort_flag, p.err, kErrTimeoutMma))) break;
-          for (int q = 0; q < NQ && ok; ++q) {
+#pragma unroll
+          for (int q = 0; q < NQ; ++q) {
+            if (!ok) break;
             if (j >= it.n[q]) continue;
             ok = mbar_wait_poll(bar(C::B_PFULL + q), (p_ph >> q) & 1, abort_flag, p.err, kErrTimeoutMma);
             if (ok && ACC2 && ((pv_any >> q) & 1))
