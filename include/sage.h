@@ -178,6 +178,12 @@ sage_status_t sage_quant_v(const void* v, sage_dtype_t dtype, sage_layout_t layo
 /* ------------------------------------------------------------------------ */
 /* Attention.                                                               */
 /* ------------------------------------------------------------------------ */
+/* The attention kernel runs a persistent grid of one CTA per SM over the
+ * problem's work items (two 128-row query tiles, or one in two-level mode,
+ * of one sequence and head).  The environment variable SAGE_MAX_CTAS, when set
+ * to a positive number below the SM count, caps that grid; results do not
+ * depend on it (the tests use it to make few CTAs walk many items). */
+
 /* The whole forward pass: sage_quant_qkv + the attention kernel.  out has q's shape, layout and dtype.  [Install/tuning guide,
  * 五分钟跑通 and 性能调优实战] */
 sage_status_t sage_attn_fwd(const void* q, const void* k, const void* v, void* out,
