@@ -255,8 +255,8 @@ def attn_head(qq: QuantQ, kq: QuantK, vq: Optional[QuantV], v16: Optional[np.nda
         _p(vq.codes) if vq is not None else None, _p(vq.scales) if vq is not None else None,
         _p(v16), PV[pv], int(v_is_bf16), _p(bias), Lq, Lk, D, int(causal),
         ctypes.c_float(sm_scale), r0, r1, _p(out), _p(allow), int(lazy_tau))
-    if vq is not None and vq.mu is not None:
-        out[r0:r1] += vq.mu.astype(np.float64)      # smooth V: the mean comes back
+    if vq is not None and vq.mu is not None and Lk > 0:
+        out[r0:r1] += vq.mu.astype(np.float64)      # smooth V: the mean comes back (no keys: rows stay 0)
     return out
 
 
@@ -289,8 +289,13 @@ class Problem:
 
 
 def problem(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout: str = "HND",
-            cu_seqlens: Optional[np.ndarray] = None) -> Problem:
-    qs, ks, vs = (seq_heads(t, layout, cu_seqlens) for t in (q, k, v))
+            cu_seqlens: Optional[np.ndarray] = None, cu_seqlens_k: Optional[np.ndarray] = None) -> Problem:
+    """cu_seqlens splits packed q (and k, v unless cu_seqlens_k is given:
+    then sequence b attends with its queries cu_seqlens[b]..[b+1] to the keys
+    cu_seqlens_k[b]..[b+1])."""
+    cu_k = cu_seqlens if cu_seqlens_k is None else cu_seqlens_k
+    qs = seq_heads(q, layout, cu_seqlens)
+    ks, vs = (seq_heads(t, layout, cu_k) for t in (k, v))
     return Problem(qs, ks, vs, len(qs[0]), len(ks[0]), q.shape[-1], q.dtype == torch.float16)
 
 
@@ -314,15 +319,18 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout: str = "
               pv: str = "fp8", smooth_k: bool = True, smooth_q: bool = False,
               cu_seqlens: Optional[np.ndarray] = None, smooth_v: bool = False, lazy_tau: int = 0,
               q_rows: Optional[Dict[Tuple[int, int], Tuple[int, int]]] = None,
-              heads: Optional[List[Tuple[int, int]]] = None, with_allowance: bool = False):
+              heads: Optional[List[Tuple[int, int]]] = None, with_allowance: bool = False,
+              cu_seqlens_k: Optional[np.ndarray] = None):
     """The quantized forward pass; returns fp64 output shaped like q.
 
     q_rows optionally restricts (seq, head) -> [row0, row1); heads restricts
     which (seq, head) pairs are computed (others stay zero).  with_allowance:
     return (out, allow), allow being the per-output bound on what ambiguous
-    roundings of P~ can change (see sage_oracle.c).
+    roundings of P~ can change (see sage_oracle.c).  cu_seqlens_k: packed
+    keys with their own sequence boundaries (causal masks key j > query i,
+    both counted from their sequence's start; a row with no visible key is 0).
     """
-    pb = problem(q, k, v, layout, cu_seqlens)
+    pb = problem(q, k, v, layout, cu_seqlens, cu_seqlens_k)
     scale = default_scale(pb.D, sm_scale)
     group = pb.Hq // pb.Hkv
     outs, allows = [], []
@@ -354,10 +362,11 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout: str = "
 
 def attention_exact(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout: str = "HND",
                     causal: bool = False, sm_scale: Optional[float] = None,
-                    cu_seqlens: Optional[np.ndarray] = None, tiled: bool = False) -> np.ndarray:
+                    cu_seqlens: Optional[np.ndarray] = None, tiled: bool = False,
+                    cu_seqlens_k: Optional[np.ndarray] = None) -> np.ndarray:
     """fp64 softmax attention of the unquantized inputs (tiled=True: the
     128-key online-softmax loop with quantization switched off)."""
-    pb = problem(q, k, v, layout, cu_seqlens)
+    pb = problem(q, k, v, layout, cu_seqlens, cu_seqlens_k)
     scale = default_scale(pb.D, sm_scale)
     group = pb.Hq // pb.Hkv
     fn = attn_tiled_fp64_head if tiled else attn_exact_head

@@ -113,6 +113,15 @@ sage_status_t run_prepass(const void* q, const void* k, const void* v, int bf16,
                           int smooth_k, int smooth_q, void* ws, const sage_ws_layout_t& L, cudaStream_t s) {
   if (cudaMemsetAsync(at<char>(ws, L.k_stat), 0, stats_zero_bytes(L, nseq, Hkv, D), s) != cudaSuccess)
     return SAGE_ERR_CUDA;
+  if (seqs.cu_k) {
+    // A varlen sequence without keys gets no K / V tile, so nothing else
+    // writes its K means and V scales / means: zero them, so that its queries
+    // (no visible key: output 0) read zeros rather than stale workspace bytes.
+    const size_t nd = (size_t)nseq * Hkv * D;
+    if (k && cudaMemsetAsync(at<char>(ws, L.k_mean), 0, nd * 4, s) != cudaSuccess) return SAGE_ERR_CUDA;
+    if (v && cudaMemsetAsync(at<char>(ws, L.v_scale), 0, L.v_mean + nd * 4 - L.v_scale, s) != cudaSuccess)
+      return SAGE_ERR_CUDA;
+  }
   PrepassJob j;
   j.q = static_cast<const uint16_t*>(q);
   j.k = static_cast<const uint16_t*>(k);

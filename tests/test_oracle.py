@@ -550,3 +550,64 @@ def test_lazy_fp8_accuracy():
     cos_p, rl1_p = _accuracy(plain, ex)
     assert cos_l >= 0.999, cos_l
     assert rl1_l <= 1.5 * rl1_p, (rl1_l, rl1_p)
+
+
+def _cross_problem(seed=3, D=64):
+    """Packed q with its own sequence lengths and packed k/v with others:
+    longer and shorter key sets, an empty query set, an empty key set."""
+    rng = np.random.default_rng(seed)
+    H, Hk = 4, 2
+    lq, lk = [150, 40, 0, 200, 17], [90, 300, 10, 0, 17]
+    cq = np.concatenate([[0], np.cumsum(lq)]).astype(np.int32)
+    ck = np.concatenate([[0], np.cumsum(lk)]).astype(np.int32)
+    q = torch.from_numpy(rng.normal(size=(cq[-1], H, D)).astype(np.float16))
+    k = torch.from_numpy((rng.normal(size=(ck[-1], Hk, D)) + rng.normal(0, 3, size=(1, Hk, D))).astype(np.float16))
+    v = torch.from_numpy(rng.normal(size=(ck[-1], Hk, D)).astype(np.float16))
+    return q, k, v, lq, lk, cq, ck
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_cross_length_varlen_pins(causal):
+    """Queries and keys with their own sequence boundaries: each sequence
+    agrees with exact fp64 attention (cosine >= 0.999); a sequence without
+    keys gives zero rows; equal boundaries passed twice change nothing."""
+    q, k, v, lq, lk, cq, ck = _cross_problem()
+    o = oracle.attention(q, k, v, causal=causal, cu_seqlens=cq, cu_seqlens_k=ck)
+    e = oracle.attention_exact(q, k, v, causal=causal, cu_seqlens=cq, cu_seqlens_k=ck)
+    for b in range(len(lq)):
+        a, x = o[cq[b]:cq[b + 1]].ravel(), e[cq[b]:cq[b + 1]].ravel()
+        if a.size == 0:
+            continue
+        if lk[b] == 0:
+            assert np.all(a == 0) and np.all(x == 0)
+            continue
+        assert a @ x / (np.linalg.norm(a) * np.linalg.norm(x)) >= 0.999
+    # same boundaries for both: identical to the single-boundary call
+    lq2 = [130, 64, 201]
+    cu = np.concatenate([[0], np.cumsum(lq2)]).astype(np.int32)
+    rng = np.random.default_rng(4)
+    q2, k2, v2 = (torch.from_numpy(rng.normal(size=(cu[-1], 2, 64)).astype(np.float16)) for _ in range(3))
+    np.testing.assert_array_equal(oracle.attention(q2, k2, v2, causal=causal, cu_seqlens=cu),
+                                  oracle.attention(q2, k2, v2, causal=causal, cu_seqlens=cu, cu_seqlens_k=cu))
+
+
+def test_cross_length_causal_reduces_to_full_past_the_keys():
+    """Causal with fewer keys than queries: from query row Lk - 1 on every
+    key is visible, so those rows equal the non-causal rows exactly."""
+    q, k, v, lq, lk, cq, ck = _cross_problem(seed=5)
+    oc = oracle.attention(q, k, v, causal=True, cu_seqlens=cq, cu_seqlens_k=ck)
+    on = oracle.attention(q, k, v, causal=False, cu_seqlens=cq, cu_seqlens_k=ck)
+    b = 0                                                   # 150 queries, 90 keys
+    assert lk[b] < lq[b]
+    np.testing.assert_array_equal(oc[cq[b] + lk[b] - 1:cq[b + 1]], on[cq[b] + lk[b] - 1:cq[b + 1]])
+    assert not np.array_equal(oc[cq[b]:cq[b] + lk[b] - 1], on[cq[b]:cq[b] + lk[b] - 1])
+
+
+def test_cross_length_smooth_v_rows_without_keys_are_zero():
+    """Smooth V adds the channel mean back only where there are keys: a
+    sequence without keys still gives zero rows, the others stay finite."""
+    q, k, v, lq, lk, cq, ck = _cross_problem(seed=6)
+    o = oracle.attention(q, k, v, causal=True, cu_seqlens=cq, cu_seqlens_k=ck, smooth_v=True)
+    b = lk.index(0)
+    assert np.all(o[cq[b]:cq[b + 1]] == 0)
+    assert np.all(np.isfinite(o))
