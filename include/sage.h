@@ -206,7 +206,11 @@ sage_status_t sage_attn_quantized(void* out, sage_dtype_t dtype, int B, int Hq, 
  * sequence b holds tokens [cu[b], cu[b+1]).  max_seqlen bounds every
  * sequence's length (larger lengths are an error reported through the device
  * error word).  total_q/total_k are the token counts the buffers hold.
- * Causal masking is top-left aligned: query i sees key j iff j <= i. */
+ * Query and key sequences may differ in length (sequence b attends with its
+ * queries cu_seqlens_q[b].. to its keys cu_seqlens_k[b]..).  Causal masking
+ * is top-left aligned: query i sees key j iff j <= i, both counted from their
+ * sequence's start.  A query with no visible key (its sequence has no keys)
+ * gets a zero row. */
 sage_status_t sage_attn_varlen_fwd(const void* q, const void* k, const void* v, void* out,
                                    sage_dtype_t dtype, const int* cu_seqlens_q,
                                    const int* cu_seqlens_k, int n_seqs, int total_q, int total_k,
