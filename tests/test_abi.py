@@ -106,3 +106,20 @@ def test_varlen_rejects_bad_arguments(L):
 def test_status_strings(L):
     for s in range(6):
         assert L.sage_status_string(s)
+
+
+def test_varlen_layout_with_separate_query_and_key_tokens(L):
+    """Queries and keys with their own token counts: Q tiles follow total_q,
+    K/V tiles total_k; the K means, V scales and V means (zeroed before a
+    varlen pre-pass, one contiguous range for the V part) sit in that order
+    inside the workspace."""
+    n, Tq, Tk, mx, Hq, Hkv, D = 6, 707, 677, 300, 4, 2, 128
+    lay = sage.workspace_layout(n, Tq, Tk, mx, Hq, Hkv, D, varlen=1)
+    assert lay["tiles_q"] <= Tq // 128 + n and lay["tiles_k"] <= Tk // 128 + n
+    assert lay["tiles_q"] >= -(-Tq // 128) and lay["tiles_k"] >= -(-Tk // 128)
+    nd = n * Hkv * D
+    assert lay["k_mean"] + 4 * nd <= lay["v_scale"] and lay["v_scale"] + 4 * nd <= lay["v_mean"]
+    assert lay["v_mean"] + 4 * nd <= lay["total"]
+    assert sage.sage_varlen_workspace_bytes(n, Tq, Tk, mx, Hq, Hkv, D) == lay["total"]
+    more_k = sage.workspace_layout(n, Tq, 4 * Tk, mx, Hq, Hkv, D, varlen=1)
+    assert more_k["tiles_q"] == lay["tiles_q"] and more_k["tiles_k"] > lay["tiles_k"]
