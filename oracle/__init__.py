@@ -24,7 +24,8 @@ import torch
 from . import build as _build
 
 GRAN = {"per_block": 0, "per_warp": 1, "per_thread": 2, "per_token": 3}
-PV = {"fp8": 0, "fp16": 1}
+PV = {"fp8": 0, "fp16": 1, "identity": 2}
+ACC = {"fp32": 0, "fp32+fp32": 0, "fp32_lazy": 0, "fp32+fp16": 1}
 
 _lib = None
 
@@ -42,8 +43,9 @@ def lib():
             "orc_e4m3_from_float_array": (None, [P, P, i64]),
             "orc_e4m3_to_float_array": (None, [P, P, i64]),
             "orc_round_f16": (f64, [f64]),
-            "orc_e4m3_alt_step": (f64, [f64]),
-            "orc_h16_alt_step": (f64, [f64, i32]),
+            "orc_e4m3_alt_step": (f64, [f64, f64]),
+            "orc_h16_alt_step": (f64, [f64, i32, f64]),
+            "orc_p_band": (f64, [f64, f64, i32, i32, f64]),
             "orc_round_bf16": (f64, [f64]),
             "orc_q_groups_per_block": (i32, [i32]),
             "orc_k_groups_per_block": (i32, [i32]),
@@ -57,9 +59,8 @@ def lib():
             "orc_quant_v_fp8": (None, [P, i64, i32, P, P]),
             "orc_scores_int32": (None, [P, P, i64, i64, i32, P]),
             "orc_smooth_q_bias": (None, [P, i64, P, P, i64, i32, P]),
-            "orc_attn_quant_head": (None, [P, P, P, P, P, P, P, i32, i32, P, i64, i64, i32,
+            "orc_attn_quant_head": (None, [P, P, P, P, P, P, P, P, P, i32, i32, i32, P, i64, i64, i32,
                                            i32, f32, i64, i64, P, P, i32]),
-            "orc_attn_tiled_fp64_head": (None, [P, P, P, i64, i64, i32, i32, f64, P, i32]),
             "orc_attn_exact_head": (None, [P, P, P, i64, i64, i32, i32, f64, i64, P]),
         }
         for name, (res, args) in sig.items():
@@ -245,15 +246,19 @@ def smooth_q_bias(qq: QuantQ, kq: QuantK) -> np.ndarray:
 def attn_head(qq: QuantQ, kq: QuantK, vq: Optional[QuantV], v16: Optional[np.ndarray],
               pv: str, v_is_bf16: bool, causal: bool, sm_scale: float,
               rows: Optional[Tuple[int, int]] = None, bias: Optional[np.ndarray] = None,
-              allow: Optional[np.ndarray] = None, lazy_tau: int = 0) -> np.ndarray:
+              allow: Optional[np.ndarray] = None, lazy_tau: int = 0, acc: str = "fp32") -> np.ndarray:
+    """pv "fp8" / "fp16"; acc "fp32+fp16" selects the binary16 inner
+    accumulation of each tile's P~V (FP8 only; see sage_oracle.c)."""
     Lq, D = qq.codes.shape
     Lk = kq.codes.shape[0]
     r0, r1 = rows if rows is not None else (0, Lq)
+    if ACC[acc] == 1 and (pv != "fp8" or lazy_tau):
+        raise ValueError("fp32+fp16 accumulation is defined for FP8 P~V with the plain online softmax")
     out = np.zeros((Lq, D), dtype=np.float64)
     lib().orc_attn_quant_head(
         _p(qq.codes), _p(qq.row_scales), _p(kq.codes), _p(kq.row_scales),
         _p(vq.codes) if vq is not None else None, _p(vq.scales) if vq is not None else None,
-        _p(v16), PV[pv], int(v_is_bf16), _p(bias), Lq, Lk, D, int(causal),
+        _p(v16), None, None, PV[pv], ACC[acc], int(v_is_bf16), _p(bias), Lq, Lk, D, int(causal),
         ctypes.c_float(sm_scale), r0, r1, _p(out), _p(allow), int(lazy_tau))
     if vq is not None and vq.mu is not None and Lk > 0:
         out[r0:r1] += vq.mu.astype(np.float64)      # smooth V: the mean comes back (no keys: rows stay 0)
@@ -269,9 +274,14 @@ def attn_exact_head(q, k, v, causal, sm_scale, row_offset: int = 0) -> np.ndarra
 
 
 def attn_tiled_fp64_head(q, k, v, causal, sm_scale, lazy_tau: int = 0) -> np.ndarray:
+    """The quantized routine with its identity-quantizer switch: the same
+    tiled online-softmax loop on unquantized fp64 q, k, P~ and v."""
+    q, k, v = (np.ascontiguousarray(x, dtype=np.float64) for x in (q, k, v))
+    Lq, D = q.shape
     out = np.zeros(q.shape, dtype=np.float64)
-    lib().orc_attn_tiled_fp64_head(_p(q), _p(k), _p(v), q.shape[0], k.shape[0], q.shape[1],
-                                   int(causal), float(sm_scale), _p(out), int(lazy_tau))
+    lib().orc_attn_quant_head(None, None, None, None, None, None, _p(v), _p(q), _p(k), PV["identity"], 0, 0, None,
+                              Lq, k.shape[0], D, int(causal), ctypes.c_float(sm_scale), 0, Lq, _p(out), None,
+                              int(lazy_tau))
     return out
 
 
@@ -320,13 +330,16 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout: str = "
               cu_seqlens: Optional[np.ndarray] = None, smooth_v: bool = False, lazy_tau: int = 0,
               q_rows: Optional[Dict[Tuple[int, int], Tuple[int, int]]] = None,
               heads: Optional[List[Tuple[int, int]]] = None, with_allowance: bool = False,
-              cu_seqlens_k: Optional[np.ndarray] = None):
+              cu_seqlens_k: Optional[np.ndarray] = None, acc: str = "fp32"):
     """The quantized forward pass; returns fp64 output shaped like q.
 
     q_rows optionally restricts (seq, head) -> [row0, row1); heads restricts
     which (seq, head) pairs are computed (others stay zero).  with_allowance:
     return (out, allow), allow being the per-output bound on what ambiguous
-    roundings of P~ can change (see sage_oracle.c).  cu_seqlens_k: packed
+    roundings of P~ (and, with acc "fp32+fp16", the binary16 roundings of the
+    partial sums) can change (see sage_oracle.c).  acc: "fp32" / "fp32+fp32"
+    / "fp32_lazy" (the same exact per-tile sums; lazy_tau selects the lazy
+    bookkeeping) or "fp32+fp16".  cu_seqlens_k: packed
     keys with their own sequence boundaries (causal masks key j > query i,
     both counted from their sequence's start; a row with no visible key is 0).
     """
@@ -351,7 +364,7 @@ def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, layout: str = "
             rows = q_rows.get((b, h)) if q_rows else None
             row.append(attn_head(qq, kq[hk], vq[hk], pb.v[b][hk] if pv != "fp8" else None, pv,
                                  not pb.is_fp16, causal, scale, rows, bias,
-                                 al if with_allowance else None, lazy_tau))
+                                 al if with_allowance else None, lazy_tau, acc))
         outs.append(row)
         allows.append(arow)
     out = assemble(outs, q, layout, cu_seqlens)

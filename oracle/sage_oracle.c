@@ -316,27 +316,71 @@ ORC_EXPORT void orc_smooth_q_bias(const float* mu_blk, int64_t nqblk, const int8
 }
 
 /* ------------------------------------------------------------------------ */
-/* Ambiguous roundings.  An implementation computes P~ with its own exp2, a  */
-/* few ulps away from the exact value.  Where the exact P~*448 (or P~) lies  */
-/* within a relative distance ORC_AMBIG of the midpoint between two          */
-/* neighbouring E4M3 (or 16-bit) values, both neighbours are correct         */
-/* roundings.  orc_alt_step returns |other - chosen| for such a value, else  */
-/* 0; the attention routine turns these into a per-output allowance.         */
+/* Ambiguous roundings of P~.                                               */
+/*                                                                          */
+/* The oracle evaluates 2^x exactly (fp64).  An implementation reaches P~   */
+/* through float32 steps and an approximate exp2, so its P~ is off by a     */
+/* small relative amount; where the exact P~ (times its static scale) lies  */
+/* that close to the midpoint between two neighbouring E4M3 (or 16-bit)     */
+/* values, either neighbour is a correct rounding.  orc_p_band derives that */
+/* relative distance per score from the arithmetic of a kernel that         */
+/*   - keeps S*c exact inside one fused multiply-add, where the oracle      */
+/*     rounds s = float(S*c): half an ulp of s;                              */
+/*   - folds the FP8 static scale into the subtracted maximum in float32,   */
+/*     nb = -float(float(m - float(log2 448)) + tau): the error of           */
+/*     float(log2 448) and half an ulp per rounding;                        */
+/*   - rounds the exponent S*c + nb once: half an ulp of it;                */
+/*   - evaluates 2^x with a relative error of at most ORC_EXP2_REL, two     */
+/*     units in the last place of a float32 result (the documented bound of */
+/*     the GPU's approximate base-2 exponential);                           */
+/* plus the oracle's own rounding of the scaled P~ to float32 before it is  */
+/* encoded (2^-24).  With the smooth-Q correction the score and the running */
+/* maximum carry further roundings, passed in as `extra` (log2 units).      */
+/* orc_e4m3_alt_step / orc_h16_alt_step return |other - chosen| for a value */
+/* within `rel` of a midpoint, else 0; orc_attn_quant_head turns these into */
+/* a per-output allowance.                                                  */
 /* ------------------------------------------------------------------------ */
-#define ORC_AMBIG 0x1p-16
+#define ORC_EXP2_REL 0x1p-22
 
-static double e4m3_alt_step(double y) {
+/* Half an ulp of a float32 of magnitude |x| (rounded up to the next binade
+ * when |x| is within 2^-20 of its top, so that a rounding that carries into
+ * the next binade is covered). */
+static double hulp32(double x) {
+    double a = fabs(x) * (1.0 + 0x1p-20);
+    if (!(a >= 0x1p-126)) return 0x1p-150;               /* subnormal spacing / 2; also 0 */
+    int e;
+    frexp(a, &e);                                        /* a in [2^(e-1), 2^e) */
+    return ldexp(1.0, e - 25);                           /* ulp 2^(e-24), halved */
+}
+
+static double log2_448(void) { return 6.0 + log2(7.0); }  /* 448 = 7 * 2^6 */
+
+ORC_EXPORT double orc_p_band(double s, double m, int fold, int tau, double extra) {
+    const double L = log2_448(), Lf = (double)(float)L;
+    double arg = s - m + (fold ? L - tau : 0.0);
+    double bl = hulp32(s) + hulp32(arg) + extra;
+    if (fold) {
+        bl += fabs(Lf - L) + hulp32(m - Lf);
+        if (tau) bl += hulp32(m - Lf + tau);
+    }
+    return (1.0 + ORC_EXP2_REL) * exp2(bl) - 1.0 + 0x1p-24;
+}
+
+static double e4m3_alt_step(double y, double rel) {
     uint8_t c = orc_e4m3_from_float((float)y);
     double v0 = (double)orc_e4m3_to_float(c);
     double v1;
     if (y >= v0) { if ((c & 0x7F) >= 0x7E) return 0.0; v1 = (double)orc_e4m3_to_float((uint8_t)(c + 1)); }
     else { if ((c & 0x7F) == 0) return 0.0; v1 = (double)orc_e4m3_to_float((uint8_t)(c - 1)); }
     double mid = 0.5 * (v0 + v1);
-    return fabs(y - mid) <= ORC_AMBIG * y ? fabs(v1 - v0) : 0.0;
+    return fabs(y - mid) <= rel * y ? fabs(v1 - v0) : 0.0;
 }
-static double h16_alt_step(double p, int bf16) {
+static double h16_alt_step(double p, int bf16, double rel) {
     double h0 = bf16 ? round_to_bf16(p) : round_to_f16((double)(float)p);
-    if (h0 <= 0.0) return 0.0;
+    if (h0 <= 0.0) {                                     /* below half the smallest step */
+        double tiny = bf16 ? 0x1p-133 : 0x1p-24;
+        return fabs(p - 0.5 * tiny) <= rel * p ? tiny : 0.0;
+    }
     int e;
     frexp(h0, &e);                                       /* h0 in [2^(e-1), 2^e) */
     int fb = bf16 ? 7 : 10;
@@ -345,11 +389,20 @@ static double h16_alt_step(double p, int bf16) {
     if (!bf16 && (e - 1) - fb < -24) up = down = ldexp(1.0, -24);
     double h1 = p >= h0 ? h0 + up : h0 - down;
     double mid = 0.5 * (h0 + h1);
-    return fabs(p - mid) <= ORC_AMBIG * p ? fabs(h1 - h0) : 0.0;
+    return fabs(p - mid) <= rel * p ? fabs(h1 - h0) : 0.0;
 }
 
-ORC_EXPORT double orc_e4m3_alt_step(double y) { return e4m3_alt_step(y); }
-ORC_EXPORT double orc_h16_alt_step(double p, int bf16) { return h16_alt_step(p, bf16); }
+ORC_EXPORT double orc_e4m3_alt_step(double y, double rel) { return e4m3_alt_step(y, rel); }
+ORC_EXPORT double orc_h16_alt_step(double p, int bf16, double rel) { return h16_alt_step(p, bf16, rel); }
+
+/* One unit in the last place of an IEEE binary16 value of magnitude |x|.   */
+static double ulp16(double x) {
+    double a = fabs(x);
+    if (a < 0x1p-14) return 0x1p-24;
+    int e;
+    frexp(a, &e);
+    return ldexp(1.0, e - 11);
+}
 
 /* ------------------------------------------------------------------------ */
 /* Quantized attention for one (sequence, head), following the FlashAttention */
@@ -358,8 +411,8 @@ ORC_EXPORT double orc_h16_alt_step(double p, int bf16) { return h16_alt_step(p, 
 /*                                                                          */
 /*  for each query row i, for each 128-key tile in increasing order          */
 /*  (reading: the tile size is the kernel's; the online-softmax state then   */
-/*  matches the kernel's, which matters because P~ is rounded to FP8        */
-/*  relative to the running maximum), skipping tiles with no visible key:   */
+/*  matches the kernel's, which matters because P~ is rounded relative to   */
+/*  the running maximum), skipping tiles with no visible key:               */
 /*    c_ij   = float(float(dQ_i * dK_j) * float(sm_scale * log2 e))          */
 /*    s_ij   = float(S_ij * c_ij)          (+ smooth-Q bias, see below)      */
 /*    m_new  = max(m, max_j s_ij);  alpha = 2^(m - m_new)                    */
@@ -378,7 +431,7 @@ ORC_EXPORT double orc_h16_alt_step(double p, int bf16) { return h16_alt_step(p, 
 /*  out_i = O * dV / (448 * l)  (FP8)      or  O / l  (16-bit)               */
 /*                                                                          */
 /* Causal (reading): top-left aligned, key j visible to query i iff j <= i.  */
-/* Smooth Q: s_ij += bias[i/128][j] * float(sm_scale * log2 e).              */
+/* Smooth Q: s_ij = float(s_ij + bias[i/128][j] * float(sm_scale * log2 e)). */
 /* Conditional (lazy) rescaling, lazy_tau > 0 [reading of the NEXT item     */
 /* "skip the alpha update unless the maximum grows by more than tau"]: the  */
 /* reference r that P~ and O are kept relative to moves to the running      */
@@ -387,76 +440,144 @@ ORC_EXPORT double orc_h16_alt_step(double p, int bf16) { return h16_alt_step(p, 
 /* 448 * 2^-tau (P8 <= 448); the output divides it out again.  lazy_tau = 0 */
 /* is the plain online softmax above.                                       */
 /*                                                                          */
+/* FP16 inner accumulation, acc_mode 1 ("fp32+fp16") [KAI 2.1, sm89 row:    */
+/* fp32fp16 two-level accumulation; GUIDE, 性能调优实战: pv_accum_dtype]: the */
+/* partial sum of each 128-key tile is held in binary16 and added into the  */
+/* fp32 outer accumulator.  Readings: (1) the partial is rounded to binary16 */
+/* after every 32 keys of the tile (one tensor-core instruction's depth),   */
+/* the 32 products themselves summed exactly; (2) one tile's partial must   */
+/* not overflow binary16 (max 65504), and with V codes up to 448 a P~ scale */
+/* of 448 would overflow on a single product; the largest static scale that */
+/* keeps 128 * scale * 448 <= 65504 is 1, so P8 = E4M3(p) and out = O*dV/l.  */
+/* FP8 only, plain online softmax (lazy_tau = 0).                           */
+/*                                                                          */
+/* Identity quantizers, pv_mode 2 (a debug reading that pins the           */
+/* bookkeeping above): scores q_i . k_j * sm_scale * log2 e in fp64 from the */
+/* unquantized qf, kf; P~ and V (v16) unrounded; no float32 step anywhere.  */
+/* The loop is the same one, so with the tiling removed it must equal       */
+/* orc_attn_exact_head to fp64 round-off.                                   */
+/*                                                                          */
 /*   qc [Lq][D] int8, q_rs [Lq] row scales; kc [Lk][D], k_rs [Lk];           */
 /*   pv_mode 0: v8 [Lk][D] E4M3 codes, dv [D];                               */
 /*   pv_mode 1: v16 [Lk][D] 16-bit V values (exact), v_is_bf16 picks the    */
 /*              16-bit type P~ is rounded to;                               */
+/*   pv_mode 2: qf [Lq][D], kf [Lk][D], v16 [Lk][D] fp64 (qc..dv unused);    */
 /*   bias [ceil(Lq/128)][Lk] or NULL; rows [row0, row1) are computed.        */
 /*   out [Lq][D] (only the computed rows are written).                       */
 /*   allow [Lq][D] or NULL: the largest change of each output that ambiguous */
-/*   roundings of P~ (see above) can cause, carried through the same alpha   */
+/*   roundings of P~ (orc_p_band) and, with acc_mode 1, the binary16        */
+/*   roundings of the partial sums (one ulp per rounding: covers rounding to */
+/*   nearest and toward zero) can cause, carried through the same alpha    */
 /*   rescaling and normalization as O.                                       */
 /* ------------------------------------------------------------------------ */
+enum { ORC_PV_FP8 = 0, ORC_PV_16 = 1, ORC_PV_IDENTITY = 2 };
+
 ORC_EXPORT void orc_attn_quant_head(const int8_t* qc, const float* q_rs, const int8_t* kc,
                                     const float* k_rs, const uint8_t* v8, const float* dv,
-                                    const double* v16, int pv_mode, int v_is_bf16,
+                                    const double* v16, const double* qf, const double* kf,
+                                    int pv_mode, int acc_mode, int v_is_bf16,
                                     const double* bias, int64_t Lq, int64_t Lk, int D,
                                     int causal, float sm_scale, int64_t row0, int64_t row1,
                                     double* out, double* allow, int lazy_tau) {
+    const int ident = pv_mode == ORC_PV_IDENTITY;
+    const int acc16 = pv_mode == ORC_PV_FP8 && acc_mode == 1;
     const float sl2 = sm_scale * 1.44269504f;             /* float(log2 e) */
-    const double pscale = 448.0 * ldexp(1.0, -lazy_tau);  /* FP8 static P~ scale */
+    const double sl2d = (double)sm_scale * 1.4426950408889634;
+    const int fold = pv_mode == ORC_PV_FP8 && !acc16;     /* 448 folded into the maximum */
+    const double pscale = !fold ? 1.0 : 448.0 * ldexp(1.0, -lazy_tau);   /* FP8 static P~ scale */
+    const double taud = (double)lazy_tau;
     int64_t ntile = (Lk + 127) / 128;
     #pragma omp parallel
     {
         double* O = (double*)malloc(sizeof(double) * D);
         double* Op = (double*)malloc(sizeof(double) * D);
+        double* Cp = (double*)malloc(sizeof(double) * D);
         double* A = (double*)malloc(sizeof(double) * D);
         double* Ap = (double*)malloc(sizeof(double) * D);
-        float* s = (float*)malloc(sizeof(float) * 128);
+        double* s = (double*)malloc(sizeof(double) * 128);
+        double* ds = (double*)malloc(sizeof(double) * 128);
         double* v8f = NULL;
-        if (pv_mode == 0) v8f = (double*)malloc(sizeof(double) * 256);
+        if (pv_mode == ORC_PV_FP8) v8f = (double*)malloc(sizeof(double) * 256);
         if (v8f) for (int c = 0; c < 256; ++c) v8f[c] = (double)orc_e4m3_to_float((uint8_t)c);
         #pragma omp for schedule(dynamic, 4)
         for (int64_t i = row0; i < row1; ++i) {
-            float m = -INFINITY;
-            double l = 0.0;
+            double m = -INFINITY, l = 0.0;
+            double dm = 0.0;                               /* smooth Q: bound on the kernel's maximum's offset */
             for (int c = 0; c < D; ++c) O[c] = A[c] = 0.0;
             for (int64_t t = 0; t < ntile; ++t) {
                 int64_t j0 = t * 128, j1 = j0 + 128 < Lk ? j0 + 128 : Lk;
                 if (causal && j1 > i + 1) j1 = i + 1;
                 if (j1 <= j0) continue;                    /* fully masked tile */
-                float mt = -INFINITY;
+                double mt = -INFINITY;
                 for (int64_t j = j0; j < j1; ++j) {
-                    int32_t S = 0;
-                    for (int c = 0; c < D; ++c) S += (int32_t)qc[i * D + c] * (int32_t)kc[j * D + c];
-                    float cij = (q_rs[i] * k_rs[j]) * sl2;
-                    float sj = (float)S * cij;
-                    if (bias) sj = (float)((double)sj + bias[(i / 128) * Lk + j] * (double)sl2);
-                    s[j - j0] = sj;
-                    if (sj > mt) mt = sj;
+                    double sc, e = 0.0;
+                    if (ident) {
+                        double d = 0.0;
+                        for (int c = 0; c < D; ++c) d += qf[i * D + c] * kf[j * D + c];
+                        sc = d * sl2d;
+                    } else {
+                        int32_t S = 0;
+                        for (int c = 0; c < D; ++c) S += (int32_t)qc[i * D + c] * (int32_t)kc[j * D + c];
+                        float cij = (q_rs[i] * k_rs[j]) * sl2;
+                        float sf = (float)S * cij;
+                        sc = sf;
+                        if (bias) {
+                            double b64 = bias[(i / 128) * Lk + j];
+                            float b32 = (float)b64;
+                            sc = (double)(float)((double)sf + b64 * (double)sl2);
+                            /* a kernel holding the correction as float32 b32 and
+                             * adding float(b32 * sl2) to the exact S*c in one
+                             * fused multiply-add differs from sc by at most: */
+                            e = 2.0 * hulp32(sc) + hulp32(b64) * (double)sl2
+                              + hulp32((double)b32 * (double)sl2) + hulp32(sf);
+                        }
+                    }
+                    s[j - j0] = sc;
+                    ds[j - j0] = e;
+                    if (sc > mt) mt = sc;
+                    if (e > dm) dm = e;                    /* the running maximum's score may be off by e */
                 }
-                const int move = (m == -INFINITY) || (mt > m + (float)lazy_tau);
-                float mn = move ? (m > mt ? m : mt) : m;
-                double alpha = (m == -INFINITY) ? 0.0 : exp2((double)m - (double)mn);
+                const double lim = ident ? m + taud : (double)(float)(m + taud);
+                const int move = (m == -INFINITY) || (mt > lim);
+                double mn = move ? (m > mt ? m : mt) : m;
+                double alpha = (m == -INFINITY) ? 0.0 : exp2(m - mn);
                 double lt = 0.0;
                 for (int c = 0; c < D; ++c) Op[c] = Ap[c] = 0.0;
-                for (int64_t j = j0; j < j1; ++j) {
-                    double p = exp2((double)s[j - j0] - (double)mn);
-                    lt += p;
-                    if (pv_mode == 0) {
-                        double p8 = v8f[orc_e4m3_from_float((float)(p * pscale))];
-                        const uint8_t* vr = v8 + j * D;
-                        for (int c = 0; c < D; ++c) Op[c] += p8 * v8f[vr[c]];
-                        double st = allow ? e4m3_alt_step(p * pscale) : 0.0;
-                        if (st > 0.0)
-                            for (int c = 0; c < D; ++c) Ap[c] += st * fabs(v8f[vr[c]]);
-                    } else {
-                        double ph = v_is_bf16 ? round_to_bf16(p) : round_to_f16((double)(float)p);
-                        const double* vr = v16 + j * D;
-                        for (int c = 0; c < D; ++c) Op[c] += ph * vr[c];
-                        double st = allow ? h16_alt_step(p, v_is_bf16) : 0.0;
-                        if (st > 0.0)
-                            for (int c = 0; c < D; ++c) Ap[c] += st * fabs(vr[c]);
+                for (int64_t c0 = j0; c0 < j0 + 128; c0 += 32) {          /* 32-key chunks */
+                    int64_t c1 = c0 + 32 < j1 ? c0 + 32 : j1;
+                    for (int c = 0; c < D; ++c) Cp[c] = 0.0;
+                    for (int64_t j = c0; j < c1; ++j) {
+                        double p = exp2(s[j - j0] - mn);
+                        lt += p;
+                        if (ident) {
+                            const double* vr = v16 + j * D;
+                            for (int c = 0; c < D; ++c) Cp[c] += p * vr[c];
+                        } else if (pv_mode == ORC_PV_FP8) {
+                            double y = p * pscale;
+                            double p8 = v8f[orc_e4m3_from_float((float)y)];
+                            const uint8_t* vr = v8 + j * D;
+                            for (int c = 0; c < D; ++c) Cp[c] += p8 * v8f[vr[c]];
+                            double st = allow ? e4m3_alt_step(y, orc_p_band(s[j - j0], mn, fold, fold ? lazy_tau : 0,
+                                                                            ds[j - j0] + dm)) : 0.0;
+                            if (st > 0.0)
+                                for (int c = 0; c < D; ++c) Ap[c] += st * fabs(v8f[vr[c]]);
+                        } else {
+                            double ph = v_is_bf16 ? round_to_bf16(p) : round_to_f16((double)(float)p);
+                            const double* vr = v16 + j * D;
+                            for (int c = 0; c < D; ++c) Cp[c] += ph * vr[c];
+                            double st = allow ? h16_alt_step(p, v_is_bf16, orc_p_band(s[j - j0], mn, 0, 0,
+                                                                                      ds[j - j0] + dm)) : 0.0;
+                            if (st > 0.0)
+                                for (int c = 0; c < D; ++c) Ap[c] += st * fabs(vr[c]);
+                        }
+                    }
+                    for (int c = 0; c < D; ++c) {
+                        if (acc16) {
+                            Op[c] = round_to_f16(Op[c] + Cp[c]);
+                            if (c1 > c0) Ap[c] += ulp16(Op[c]);   /* a chunk of masked keys adds 0 exactly */
+                        } else {
+                            Op[c] += Cp[c];
+                        }
                     }
                 }
                 l = alpha * l + lt;
@@ -467,70 +588,22 @@ ORC_EXPORT void orc_attn_quant_head(const int8_t* qc, const float* q_rs, const i
                 m = mn;
             }
             for (int c = 0; c < D; ++c) {
-                double o;
-                if (l <= 0.0) o = 0.0;                     /* no visible key at all */
-                else if (pv_mode == 0) o = O[c] * (double)dv[c] / (pscale * l);
-                else o = O[c] / l;
+                double o, a;
+                if (l <= 0.0) o = a = 0.0;                 /* no visible key at all */
+                else if (pv_mode == ORC_PV_FP8) {
+                    o = O[c] * (double)dv[c] / (pscale * l);
+                    a = A[c] * (double)dv[c] / (pscale * l);
+                } else {
+                    o = O[c] / l;
+                    a = A[c] / l;
+                }
                 out[i * D + c] = o;
-                if (allow)
-                    allow[i * D + c] = l <= 0.0 ? 0.0
-                                     : pv_mode == 0 ? A[c] * (double)dv[c] / (pscale * l) : A[c] / l;
+                if (allow) allow[i * D + c] = a;
             }
         }
-        free(O); free(Op); free(A); free(Ap); free(s); free(v8f);
+        free(O); free(Op); free(Cp); free(A); free(Ap); free(s); free(ds); free(v8f);
     }
 }
-
-/* ------------------------------------------------------------------------ */
-/* The same tiled online softmax with quantization switched off (debug      */
-/* reading used only to pin the FlashAttention bookkeeping): fp64 scores    */
-/* q_i . k_j * sm_scale * log2 e, unrounded P~ and V.  With the tiling       */
-/* removed it is exactly softmax attention, so it must agree with           */
-/* orc_attn_exact_head to fp64 round-off.                                   */
-/*   q [Lq][D], k [Lk][D], v [Lk][D] fp64.                                    */
-/* ------------------------------------------------------------------------ */
-ORC_EXPORT void orc_attn_tiled_fp64_head(const double* q, const double* k, const double* v,
-                                         int64_t Lq, int64_t Lk, int D, int causal,
-                                         double sm_scale, double* out, int lazy_tau) {
-    const double sl2 = sm_scale * 1.4426950408889634;
-    int64_t ntile = (Lk + 127) / 128;
-    #pragma omp parallel
-    {
-        double* O = (double*)malloc(sizeof(double) * D);
-        double* s = (double*)malloc(sizeof(double) * 128);
-        #pragma omp for schedule(dynamic, 4)
-        for (int64_t i = 0; i < Lq; ++i) {
-            double m = -INFINITY, l = 0.0;
-            for (int c = 0; c < D; ++c) O[c] = 0.0;
-            for (int64_t t = 0; t < ntile; ++t) {
-                int64_t j0 = t * 128, j1 = j0 + 128 < Lk ? j0 + 128 : Lk;
-                if (causal && j1 > i + 1) j1 = i + 1;
-                if (j1 <= j0) continue;
-                double mt = -INFINITY;
-                for (int64_t j = j0; j < j1; ++j) {
-                    double d = 0.0;
-                    for (int c = 0; c < D; ++c) d += q[i * D + c] * k[j * D + c];
-                    s[j - j0] = d * sl2;
-                    if (s[j - j0] > mt) mt = s[j - j0];
-                }
-                const int move = (m == -INFINITY) || (mt > m + (double)lazy_tau);
-                double mn = move ? (m > mt ? m : mt) : m;
-                double alpha = (m == -INFINITY) ? 0.0 : exp2(m - mn);
-                for (int c = 0; c < D; ++c) O[c] *= alpha;
-                l *= alpha;
-                for (int64_t j = j0; j < j1; ++j) {
-                    double p = exp2(s[j - j0] - mn);
-                    l += p;
-                    for (int c = 0; c < D; ++c) O[c] += p * v[j * D + c];
-                }
-                m = mn;
-            }
-            for (int c = 0; c < D; ++c) out[i * D + c] = l > 0.0 ? O[c] / l : 0.0;
-        }
-        free(O); free(s);
-    }
-}
-
 /* ------------------------------------------------------------------------ */
 /* Exact attention, the quantity the method approximates: softmax(q k^T *    */
 /* sm_scale [+ causal mask]) v, in fp64, one pass with the true row maximum. */
