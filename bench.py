@@ -37,8 +37,10 @@ import synth  # noqa: E402
 
 WORKLOAD = "b2_h32_s4096_d128"
 METRIC = "attention TOPS (4BHS²D/t) at D=128, S=4K–32K; % of B200 INT8/FP8 peak"
-FALLBACK_BF16_SUSTAINED = 1400.0   # TFLOP/s, used only without the measured peaks file
+FALLBACK_BF16 = 1590.0             # TFLOP/s burst, used only without the measured peaks file
+FALLBACK_BF16_SUSTAINED = 1400.0   # TFLOP/s sustained, likewise
 FP8_OVER_BF16 = 2.0                # nominal dense ratio (4.5 / 2.25 PFLOP/s); INT8 = FP8 on B200
+SUSTAINED_AFTER_S = 2.0            # timed regions longer than this are compared with the sustained peak
 
 
 def parse():
@@ -49,11 +51,12 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--config", default=WORKLOAD)
     ap.add_argument("--pv", default="fp8", choices=["fp8", "fp16"])
-    ap.add_argument("--pv-accum", default="fp32", choices=["fp32", "fp32+fp32", "fp32_lazy"])
+    ap.add_argument("--pv-accum", default="fp32", choices=["fp32", "fp32+fp32", "fp32_lazy", "fp32+fp16"])
     ap.add_argument("--gran", default="per_block", choices=["per_block", "per_warp", "per_thread", "per_token"])
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-sweep", action="store_true", help="skip the attention-kernel sweep over S")
     return ap.parse_args()
 
 
@@ -64,11 +67,73 @@ def peaks():
         d = json.load(open(path))
         return d, "measured"
     except Exception:
-        return {"bf16_tflops_sustained": FALLBACK_BF16_SUSTAINED, "hbm_gbs": 6650.0}, "fallback"
+        return {"bf16_tflops": FALLBACK_BF16, "bf16_tflops_sustained": FALLBACK_BF16_SUSTAINED,
+                "hbm_gbs": 6650.0}, "fallback"
+
+
+def tensor_peak(pk: dict, region_s: float):
+    """Dense INT8/FP8 peak (TOPS) for a kernel timed over a region of
+    region_s seconds: 2 x the measured bf16 burst figure for short regions,
+    2 x the sustained (power-capped) figure for regions of seconds."""
+    if region_s > SUSTAINED_AFTER_S:
+        return FP8_OVER_BF16 * float(pk.get("bf16_tflops_sustained", FALLBACK_BF16_SUSTAINED)), "sustained"
+    return FP8_OVER_BF16 * float(pk.get("bf16_tflops", FALLBACK_BF16)), "burst"
+
+
+class NvmlClocks:
+    """In-process NVML sampling (read-only queries) of the SM clock and the
+    clock-event reasons every ~1 ms, so that even a region of ~10 ms has a
+    clock record of its own."""
+
+    REASONS = {"hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40, "sw_power_cap": 0x4}
+
+    def __init__(self, gpu_index: int, period_s: float = 0.001):
+        self.idx, self.period = gpu_index, period_s
+        self.samples, self.reasons, self.max_mhz, self.ok = [], set(), None, False
+        self.stop = threading.Event()
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(self.idx)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        except Exception:
+            self.ok = False
+        return self
+
+    def _run(self):
+        nv = self.nv
+        while not self.stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __exit__(self, *a):
+        self.stop.set()
+        if self.ok:
+            self.t.join(timeout=5)
+
+    def summary(self):
+        if not self.samples:
+            return None
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples), "source": "nvml, in-process, ~1 ms"}
 
 
 class Clocks:
-    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed
+    region (used when NVML cannot be opened in-process)."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -144,6 +209,16 @@ def recorded_traffic(workload: str):
     return e.get("dram_bytes_per_launch")
 
 
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
 def max_over_ranks(x: float, device) -> float:
     """The maximum of x over the ranks of the default process group (x itself
     without one): a multi-GPU time is the slowest rank's."""
@@ -190,9 +265,49 @@ def cpu_baseline(spec: synth.Spec, q, k, v, pv: str, budget_s: float):
     dt = time.perf_counter() - t0
     ops = 4.0 * done_rows * spec.S * spec.D * (0.5 if spec.causal else 1.0)
     cores = int(os.environ.get("OMP_NUM_THREADS", os.cpu_count() or 1))
-    return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": cores, "kind": "oracle",
+    return {"value": ops / dt / 1e12, "unit": "TOPS", "cores": cores, "kind": "oracle", "cpu_model": cpu_model(),
             "sample": f"{len(sample)} query tiles x 128 rows x all {spec.S} keys (+ their K/V/Q pre-pass) of "
                       f"{spec.name}, {dt:.1f} s, scaled by the ops of the rows computed"}
+
+
+# ----------------------------------------------------------------------------- S sweep
+def sweep_s(sage, dev, gran, n=20):
+    """The attention kernel alone over the metric's sequence axis: S in
+    1K..32K with B = 32768 / S, H = 32, D = 128, FP8 and 16-bit P~V, causal
+    and not (one-level accumulation), on seeded iid N(0,1) fp16 inputs drawn
+    on the device.  TOPS from CUDA events over n launches, and the fraction
+    of the burst dense FP8/INT8 peak."""
+    pk, _ = peaks()
+    peak, _ = tensor_peak(pk, 0.0)
+    g = torch.Generator(device=dev)
+    res = {}
+    for S in (1024, 2048, 4096, 8192, 16384, 32768):
+        Bs, H, D = 32768 // S, 32, 128
+        g.manual_seed(S)
+        q, k, v = (torch.randn(Bs, H, S, D, generator=g, device=dev, dtype=torch.float32).half() for _ in range(3))
+        o = torch.empty_like(q)
+        w = torch.empty(sage.sage_workspace_bytes(Bs, H, H, S, D, 1, 0), dtype=torch.uint8, device=dev)
+        for pv in ("fp8", "fp16"):
+            sage.quant_qkv(q, k, v, w, "HND", gran, pv)
+            for causal in (False, True):
+                def f():
+                    sage.attn_quantized(o, w, Bs, H, H, S, D, "HND", causal, None, gran, pv, "fp32")
+                for _ in range(3):
+                    f()
+                e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+                torch.cuda.synchronize()
+                e0.record()
+                for _ in range(n):
+                    f()
+                e1.record()
+                torch.cuda.synchronize()
+                ms = e0.elapsed_time(e1) / n
+                tops = 4.0 * Bs * H * S * S * D * (0.5 if causal else 1.0) / (ms * 1e-3) / 1e12
+                res[f"S{S}/{pv}/{'causal' if causal else 'full'}"] = {"tops": round(tops, 1),
+                                                                       "frac": round(tops / peak, 4)}
+        del q, k, v, o, w
+    return {"workload": "B=32768/S, H=32, D=128, fp16 iid N(0,1), HND, one-level accumulation", "gran": gran,
+            "peak": peak, "points": res}
 
 
 # ----------------------------------------------------------------------------- main
@@ -266,7 +381,7 @@ def main():
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
-    with Clocks(local) as clk:
+    with NvmlClocks(local) as nclk, Clocks(local) as clk:
         start.record(stream)
         for i in range(args.steps):
             step(evs[i])
@@ -287,7 +402,7 @@ def main():
 
     # the attention kernel alone in the other modes the workload names (and
     # the conditional-rescaling mode), inputs resident, CUDA events
-    def kernel_tops(pv, acc, n=100):
+    def kernel_ms(pv, acc, n=100):
         sage.quant_qkv(q, k, v, ws, layout, args.gran, pv)
 
         def f():
@@ -302,11 +417,13 @@ def main():
             f()
         m1.record(stream)
         torch.cuda.synchronize()
-        return ops / (m0.elapsed_time(m1) / n * 1e-3) / 1e12
+        return m0.elapsed_time(m1) / n
 
-    other_modes = {f"{pv}/{acc}": kernel_tops(pv, acc)
-                   for pv, acc in [("fp8", "fp32+fp32"), ("fp8", "fp32_lazy"), ("fp16", "fp32"), ("fp16", "fp32+fp32"),
-                                   ("fp16", "fp32_lazy")] if (pv, acc) != (args.pv, args.pv_accum)}
+    other_ms = {(pv, acc): kernel_ms(pv, acc)
+                for pv, acc in [("fp8", "fp32+fp32"), ("fp8", "fp32_lazy"), ("fp8", "fp32+fp16"), ("fp16", "fp32"),
+                                ("fp16", "fp32+fp32"), ("fp16", "fp32_lazy")] if (pv, acc) != (args.pv, args.pv_accum)}
+    other_modes = {f"{pv}/{acc}": ops / (ms * 1e-3) / 1e12 for (pv, acc), ms in other_ms.items()}
+    sweep = None if args.no_sweep or world > 1 else sweep_s(sage, dev, args.gran)
 
     # end to end through the public API with host buffers: every step copies
     # q, k, v in from pinned host memory, runs sageattn and copies the output
@@ -365,9 +482,11 @@ def main():
         return
 
     pk, pk_kind = peaks()
-    peak = FP8_OVER_BF16 * float(pk.get("bf16_tflops_sustained", FALLBACK_BF16_SUSTAINED))
+    peak, peak_kind = tensor_peak(pk, elapsed_ms * 1e-3)
     attn_avg = float(np.mean(attn_ms))
     achieved = ops / (attn_avg * 1e-3) / 1e12
+    two = ("fp8", "fp32+fp32") if args.pv == "fp8" else ("fp16", "fp32+fp32")
+    two_ms = other_ms.get(two)
     pre_avg = float(np.mean(pre_ms))
     elem = spec.total_tokens * D
     pre_bytes = elem * (2 * spec.Hq + 4 * spec.Hkv) + elem * (spec.Hq + 2 * spec.Hkv)   # 9 B/elem at Hq=Hkv
@@ -383,8 +502,14 @@ def main():
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": recorded_traffic(spec.name),
                      "kernel": "attn_fwd_kernel", "kernel_ms": attn_avg,
-                     "peak_source": f"2 x bf16_tflops_sustained ({pk_kind}); burst figure "
-                                    f"{FP8_OVER_BF16 * float(pk.get('bf16_tflops', 0)):.0f}"},
+                     "mode": f"{args.pv}/{args.pv_accum}",
+                     "peak_source": f"2 x bf16_tflops {peak_kind} ({pk_kind}: the dense FP8/INT8 rate is twice "
+                                    f"bf16's); timed region {elapsed_ms:.1f} ms"},
+        "roofline_two_level": None if two_ms is None else {
+            "bound": "tensor", "achieved": ops / (two_ms * 1e-3) / 1e12, "peak": peak, "unit": "TFLOP/s",
+            "frac": ops / (two_ms * 1e-3) / 1e12 / peak, "traffic": None, "kernel": "attn_fwd_kernel",
+            "kernel_ms": two_ms, "mode": f"{two[0]}/{two[1]}",
+            "note": "the two-level accumulation (the API default), attention kernel alone, 100 launches"},
         "prepass": {"ms": pre_avg, "achieved_gbs": pre_bytes / (pre_avg * 1e-3) / 1e9,
                     "peak_gbs": float(pk.get("hbm_gbs", 0)),
                     "frac": pre_bytes / (pre_avg * 1e-3) / 1e9 / float(pk.get("hbm_gbs", 1))},
@@ -392,8 +517,10 @@ def main():
                 "h2d_bytes_per_step": int(sum(t.numel() * t.element_size() for t in (q_h, k_h, v_h))),
                 "d2h_bytes_per_step": int(q_h.numel() * q_h.element_size())},
         "attention_modes_tops": other_modes,   # attention kernel alone, other P~V / accumulation modes
+        "attention_modes_frac": {m: t / peak for m, t in other_modes.items()},
+        "sweep": sweep,
         "gpu_launches": 3 * args.steps,     # pre-pass launches A and B + the attention kernel
-        "clocks": clk.summary(),
+        "clocks": nclk.summary() or clk.summary(),
     }
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(spec, q_h, k_h, v_h, args.pv, args.cpu_seconds)

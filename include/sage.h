@@ -96,8 +96,17 @@ typedef enum { SAGE_PV_FP8 = 0, SAGE_PV_FP16 = 1, SAGE_PV_FP8_SMOOTH_V = 2 } sag
  * FP32_LAZY = FP32 with conditional rescaling: P~ and O stay relative to a
  * reference maximum that moves only when a tile's maximum exceeds it by more
  * than tau (tau = 2 with FP8 P~V, whose static P~ scale becomes 448 * 2^-2;
- * tau = 8 with 16-bit P~V), so most tiles skip the rescale of O. */
-typedef enum { SAGE_ACC_FP32 = 0, SAGE_ACC_FP32_FP32 = 1, SAGE_ACC_FP32_LAZY = 2 } sage_acc_t;
+ * tau = 8 with 16-bit P~V), so most tiles skip the rescale of O.
+ * FP32_FP16 = two-level with a binary16 inner level [Kairos page, section 二
+ * 2.1, sm89 row: fp32fp16 two-level accumulation; install/tuning guide,
+ * 性能调优实战: pv_accum_dtype]: each 128-key tile's partial sum is held in
+ * binary16 by the tensor core and added into the FP32 register accumulator.
+ * FP8 P~V only (SAGE_PV_FP16 gives SAGE_ERR_UNSUPPORTED).  P~ is encoded
+ * with the static scale 1 instead of 448, the largest that keeps one tile's
+ * partial sums (128 keys x P~ <= 1 x V codes <= 448 = 57344) inside
+ * binary16's range. */
+typedef enum { SAGE_ACC_FP32 = 0, SAGE_ACC_FP32_FP32 = 1, SAGE_ACC_FP32_LAZY = 2,
+               SAGE_ACC_FP32_FP16 = 3 } sage_acc_t;
 
 /* ------------------------------------------------------------------------ */
 /* Workspace.                                                               */
@@ -180,9 +189,8 @@ sage_status_t sage_quant_v(const void* v, sage_dtype_t dtype, sage_layout_t layo
 /* ------------------------------------------------------------------------ */
 /* The attention kernel runs a persistent grid of one CTA per SM over the
  * problem's work items (two 128-row query tiles, or one in two-level mode,
- * of one sequence and head).  The environment variable SAGE_MAX_CTAS, when set
- * to a positive number below the SM count, caps that grid; results do not
- * depend on it (the tests use it to make few CTAs walk many items). */
+ * of one sequence and head).  sage_debug_set_max_ctas caps that grid;
+ * results do not depend on it. */
 
 /* The whole forward pass: sage_quant_qkv + the attention kernel.  out has q's shape, layout and dtype.  [Install/tuning guide,
  * 五分钟跑通 and 性能调优实战] */
@@ -261,6 +269,23 @@ sage_status_t sage_attn_fwd_noalloc(const void* q, const void* k, const void* v,
  * device-side argument check failed, e.g. a varlen length above max_seqlen)
  * or SAGE_ERR_CUDA.  *bits (optional) receives the raw error word. */
 sage_status_t sage_get_device_error(void* ws, void* stream, uint32_t* bits);
+
+/* Debug: cap the attention kernel's persistent grid at max_ctas CTAs (0: one
+ * CTA per SM, the default).  Process-wide; applies to the attention launches
+ * that follow.  Results do not depend on it: the tests use it to make a few
+ * CTAs walk many work items.  max_ctas < 0 gives SAGE_ERR_INVALID_ARG. */
+sage_status_t sage_debug_set_max_ctas(int max_ctas);
+
+/* Debug: make the attention launches that follow lose one K tile.  The
+ * loader of CTA 0 skips the copy of the ring_index-th K tile it would load
+ * (counted from 0 over that CTA's work items); the wait for that tile runs
+ * out after about 2 s, the kernel tears down and the workspace's error word
+ * reports a timeout, which sage_get_device_error returns as
+ * SAGE_ERR_TIMEOUT.  This exercises the timeout path without a GPU fault:
+ * no copy is left in flight and the CUDA context stays usable.  The output
+ * rows of the aborted CTA's work items are undefined.  -1 (the default)
+ * switches it off; values below -1 give SAGE_ERR_INVALID_ARG. */
+sage_status_t sage_debug_withhold_k_tile(int ring_index);
 
 /* Debug: the int32 scores of one 128x128 tile, S = Q_codes(q tile) *
  * K_codes(k tile)^T, computed by the same tensor-core MMA path as the

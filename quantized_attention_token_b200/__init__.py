@@ -19,7 +19,8 @@ from typing import Optional
 
 __all__ = [
     "sageattn", "sageattn_varlen", "quant_qk", "quant_qkv", "quant_v", "attn_quantized", "workspace_layout",
-    "get_device_error", "debug_qk_tile", "Workspace", "SageError", "lib", "LIB_PATH",
+    "get_device_error", "debug_qk_tile", "debug_set_max_ctas", "debug_withhold_k_tile", "Workspace", "SageError",
+    "lib", "LIB_PATH",
 ]
 
 HERE = os.path.dirname(os.path.abspath(__file__))
@@ -29,7 +30,8 @@ OK, ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE, ERR_CUDA, ERR_TIMEOUT = ran
 LAYOUT = {"HND": 0, "NHD": 1}
 GRAN = {"per_block": 0, "per_warp": 1, "per_thread": 2, "per_token": 3}
 PV = {"fp8": 0, "fp16": 1, "fp8_smooth_v": 2}   # fp8_smooth_v: FP8 with V smoothed by its channel mean
-ACC = {"fp32": 0, "fp32+fp32": 1, "fp32fp32": 1, "fp32_lazy": 2}   # fp32_lazy: one-level, conditional rescaling
+# fp32_lazy: one-level, conditional rescaling; fp32+fp16: two-level with a binary16 inner level (FP8 P~V)
+ACC = {"fp32": 0, "fp32+fp32": 1, "fp32fp32": 1, "fp32_lazy": 2, "fp32+fp16": 3, "fp32fp16": 3}
 
 
 class SageError(RuntimeError):
@@ -71,6 +73,8 @@ def lib():
         "sage_get_device_error": (I, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
         "sage_debug_qk_tile": (I, [P, I, I, I, I, I, I, I, I, I, I, I, P, P]),
         "sage_status_string": (ctypes.c_char_p, [I]),
+        "sage_debug_set_max_ctas": (I, [I]),
+        "sage_debug_withhold_k_tile": (I, [I]),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -288,3 +292,15 @@ def debug_qk_tile(ws, B, Hq, Hkv, S, D, b, h, q_tile, k_tile, pv_dtype="fp8"):
                                   out.data_ptr(), _stream(ws.device))
     _check("sage_debug_qk_tile", st)
     return out
+
+
+def debug_set_max_ctas(n: int):
+    """Cap the attention kernel's persistent grid at n CTAs (0: one per SM).
+    Process-wide; results do not depend on it."""
+    _check("sage_debug_set_max_ctas", lib().sage_debug_set_max_ctas(int(n)))
+
+
+def debug_withhold_k_tile(ring_index: int):
+    """Make CTA 0 of the following attention launches skip one K tile copy, so
+    that its bounded wait runs out (-1: off).  Tests the timeout path."""
+    _check("sage_debug_withhold_k_tile", lib().sage_debug_withhold_k_tile(int(ring_index)))

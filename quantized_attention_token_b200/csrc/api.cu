@@ -3,6 +3,7 @@
 // Host side only: argument validation, the workspace planner, and the order
 // of launches on the caller's stream.  No device memory is allocated here and
 // no call synchronizes except sage_get_device_error.
+#include <atomic>
 #include <climits>
 #include <cmath>
 #include <cstring>
@@ -14,6 +15,11 @@
 
 namespace sage {
 namespace {
+
+// Debug settings (sage_debug_set_max_ctas, sage_debug_withhold_k_tile):
+// process-wide, read at each attention launch.
+std::atomic<int> g_max_ctas{0};
+std::atomic<int> g_withhold_k{-1};
 
 // ---------------------------------------------------------------- device check
 sage_status_t check_device() {
@@ -97,8 +103,12 @@ sage_status_t check_common(sage_dtype_t dtype, int D, sage_gran_t gran, sage_pv_
   if (gran != SAGE_PER_BLOCK && gran != SAGE_PER_WARP && gran != SAGE_PER_THREAD && gran != SAGE_PER_TOKEN)
     return SAGE_ERR_INVALID_ARG;
   if (pv != SAGE_PV_FP8 && pv != SAGE_PV_FP16 && pv != SAGE_PV_FP8_SMOOTH_V) return SAGE_ERR_INVALID_ARG;
-  if (acc != SAGE_ACC_FP32 && acc != SAGE_ACC_FP32_FP32 && acc != SAGE_ACC_FP32_LAZY) return SAGE_ERR_INVALID_ARG;
+  if (acc != SAGE_ACC_FP32 && acc != SAGE_ACC_FP32_FP32 && acc != SAGE_ACC_FP32_LAZY && acc != SAGE_ACC_FP32_FP16)
+    return SAGE_ERR_INVALID_ARG;
   if (D != 64 && D != 128) return SAGE_ERR_UNSUPPORTED;
+  // the binary16 inner accumulation is defined for FP8 P~V (its P~ scale keeps
+  // one tile's partial sums inside binary16's range)
+  if (acc == SAGE_ACC_FP32_FP16 && pv == SAGE_PV_FP16) return SAGE_ERR_UNSUPPORTED;
   return SAGE_OK;
 }
 
@@ -195,7 +205,10 @@ sage_status_t run_attn(void* out, int bf16, Strides so, const Seqs& seqs, int ns
   p.causal = causal ? 1 : 0;
   p.out_bf16 = bf16;
   p.v_mean = pv == SAGE_PV_FP8_SMOOTH_V ? at<float>(w, L.v_mean) : nullptr;
-  return cuda_status(attn_forward(p, D, pv != SAGE_PV_FP16, acc == SAGE_ACC_FP32_FP32, seqs.max_seqlen, nseq, s));
+  p.max_ctas = g_max_ctas.load();
+  p.dbg_withhold_k = g_withhold_k.load();
+  const int mode = acc == SAGE_ACC_FP32_FP32 ? kAccTwo : acc == SAGE_ACC_FP32_FP16 ? kAccTwoF16 : kAccOne;
+  return cuda_status(attn_forward(p, D, pv != SAGE_PV_FP16, mode, seqs.max_seqlen, nseq, s));
 }
 
 Seqs dense_seqs(int S) {
@@ -402,6 +415,18 @@ SAGE_EXPORT sage_status_t sage_debug_qk_tile(const void* ws, int B, int Hq, int 
   const int8_t* qt = at<int8_t>(w, L.q_codes) + ((size_t)h * L.tiles_q + (size_t)b * tps + q_tile) * kTile * D;
   const int8_t* kt = at<int8_t>(w, L.k_codes) + ((size_t)hk * L.tiles_k + (size_t)b * tps + k_tile) * kTile * D;
   return cuda_status(debug_qk_tile(qt, kt, D, s_out, at<uint32_t>(w, L.err), static_cast<cudaStream_t>(stream)));
+}
+
+SAGE_EXPORT sage_status_t sage_debug_set_max_ctas(int max_ctas) {
+  if (max_ctas < 0) return SAGE_ERR_INVALID_ARG;
+  g_max_ctas.store(max_ctas);
+  return SAGE_OK;
+}
+
+SAGE_EXPORT sage_status_t sage_debug_withhold_k_tile(int ring_index) {
+  if (ring_index < -1) return SAGE_ERR_INVALID_ARG;
+  g_withhold_k.store(ring_index);
+  return SAGE_OK;
 }
 
 SAGE_EXPORT const char* sage_status_string(sage_status_t s) {

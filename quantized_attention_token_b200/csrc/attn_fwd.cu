@@ -25,14 +25,13 @@
 //                 tile's QK^T runs while it works; P~ goes to shared memory in
 //                 the swizzled K-major operand layout; in one-level mode it
 //                 also rescales O in TMEM and writes the epilogue;
-//   WG 2 (two-level mode, NQ = 1) correction: adds each tile's fresh FP32
-//                 partial O into an FP32 register accumulator; epilogue.
+//   WG 2 (two-level mode, NQ = 1) correction: adds each tile's fresh partial
+//                 O (FP32, or binary16 in fp32+fp16 mode) into an FP32
+//                 register accumulator; epilogue.
 // Warpgroup 0 (loader, MMA, allocator) hands registers to WG 1..2 with
 // setmaxnreg (56 / 224 / 224 per thread).
 // Every mbarrier wait is bounded (sage_common.cuh): a wait that never ends sets
 // the device error word and the CTA tears down instead of hanging.
-#include <cstdlib>
-
 #include "sage_launch.cuh"
 
 namespace sage {
@@ -410,7 +409,7 @@ __device__ __forceinline__ bool next_busy_item(const AttnParams& p, int idx, Ite
 
 // One softmax warpgroup: for each item, the online softmax of query tile q
 // over its KV tiles; in one-level mode also the O rescale and the epilogue.
-template <int D, bool PV8, bool ACC2, bool KPT, bool BF16P, bool SMQ>
+template <int D, bool PV8, bool ACC2, bool A16, bool KPT, bool BF16P, bool SMQ>
 __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, uint32_t tmem, int warp, int tid) {
   using C = AttnCfg<D, PV8, ACC2>;
   constexpr int NQ = C::NQ;
@@ -532,7 +531,10 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
           alpha_s[(q * 2 + ab) * 128 + t] = alpha;
           mbar_arrive(bar(C::B_AFULL + 2 * q + ab));
         }
-        const float nb = -(PV8 ? (m_new - kLog2Fp8Max + (float)p.lazy_tau) : m_new);
+        // FP8 P~ carries the static scale 448 (folded into the exponent); with
+        // the binary16 inner accumulation its scale is 1, so that one tile's
+        // partial sums (<= 128 * 448) stay inside binary16's range
+        const float nb = -((PV8 && !A16) ? (m_new - kLog2Fp8Max + (float)p.lazy_tau) : m_new);
         // FP8 P~V, two query tiles: their exponential phases take turns (tile
         // 0's of KV tile j, then tile 1's, then tile 0's of j+1, ...; over the
         // items of the CTA one after the other), so that each runs at the
@@ -663,7 +665,7 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
 }
 
 // ---------------------------------------------------------------- kernel
-template <int D, bool PV8, bool ACC2>
+template <int D, bool PV8, bool ACC2, bool A16>
 __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
   using C = AttnCfg<D, PV8, ACC2>;
   constexpr int NQ = C::NQ, NST = C::NST;
@@ -748,8 +750,12 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
           const int st = kv % NST, u = kv / NST;
           if (u > 0 && !(ok = mbar_wait_poll(bar(C::B_KEMPTY + st), (u - 1) & 1, abort_flag, p.err, kErrTimeoutLoad)))
             break;
-          mbar_expect_tx(bar(C::B_KFULL + st), C::QT);
-          bulk_g2s(sb + C::OFF_K + st * C::QT, kb + (size_t)t * C::QT, C::QT, bar(C::B_KFULL + st));
+          // (debug, host-selected) CTA 0 withholds one K tile: the MMA's wait
+          // for it runs out and the CTA aborts -- the test of the timeout path
+          if (!(blockIdx.x == 0 && kv == p.dbg_withhold_k)) {
+            mbar_expect_tx(bar(C::B_KFULL + st), C::QT);
+            bulk_g2s(sb + C::OFF_K + st * C::QT, kb + (size_t)t * C::QT, C::QT, bar(C::B_KFULL + st));
+          }
           issued_k = kv + 1;
           if (u > 0 && !(ok = mbar_wait_poll(bar(C::B_VEMPTY + st), (u - 1) & 1, abort_flag, p.err, kErrTimeoutLoad)))
             break;
@@ -764,6 +770,7 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
       if (*abort_flag) {
         // let copies in flight land before the CTA's shared memory is released
         for (int t = max(0, issued_k - NST); t < issued_k; ++t) {
+          if (blockIdx.x == 0 && t == p.dbg_withhold_k) continue;   // never issued
           const uint64_t t0 = global_timer_ns();
           while (!mbar_try_wait(bar(C::B_KFULL + t % NST), (t / NST) & 1) && global_timer_ns() - t0 < kWaitLimitNs) {}
         }
@@ -789,7 +796,8 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
     // epilogue.
     if (lane == 0) {
       constexpr uint32_t ID_QK = idesc_i8(128, 128);
-      const uint32_t ID_PV = PV8 ? idesc_e4m3(128, D) : idesc_f16(128, D, p.out_bf16 != 0);
+      const uint32_t ID_PV = PV8 ? (A16 ? idesc_e4m3_acc16(128, D) : idesc_e4m3(128, D))
+                                 : idesc_f16(128, D, p.out_bf16 != 0);
       bool ok = true;
       int kvs = 0, kvp = 0;                  // ring index of the next K tile (QK^T) and V tile (PV)
       uint32_t s_ph = 0, q_ph = 0, p_ph = 0;  // bit q: parity of S_j seeds, Q loads, P~ tiles consumed
@@ -910,7 +918,7 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
     // ------------------------------------------------------------ softmax
     const bool bf16p = !PV8 && p.out_bf16;
     const int variant = (p.gran == 2 ? 4 : 0) + (bf16p ? 2 : 0) + (p.q_bias ? 1 : 0);
-#define SAGE_SOFTMAX(KPT, BF16P, SMQ) softmax_role<D, PV8, ACC2, KPT, BF16P, SMQ>(p, sb, tmem, warp, tid)
+#define SAGE_SOFTMAX(KPT, BF16P, SMQ) softmax_role<D, PV8, ACC2, A16, KPT, BF16P, SMQ>(p, sb, tmem, warp, tid)
     switch (variant) {
       case 0: SAGE_SOFTMAX(false, false, false); break;
       case 1: SAGE_SOFTMAX(false, false, true); break;
@@ -954,15 +962,32 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
         if (!(ok = mbar_wait(bar(C::B_OFULL), o_ph, abort_flag, p.err, kErrTimeoutCorr))) break;
         o_ph ^= 1;
         tc_fence_after();
+        if (A16) {
+          // binary16 partial sums, one per TMEM column; the load packs two
+          // adjacent columns into one register
 #pragma unroll
-        for (int ch = 0; ch < D / 16; ++ch) {
-          uint32_t r[16];
-          tmem_ld16(ob + ch * 16, r);
-          tmem_wait_ld(r);
+          for (int ch = 0; ch < D / 32; ++ch) {
+            uint32_t r[16];
+            tmem_ld32_pack16(ob + ch * 32, r);
+            tmem_wait_ld(r);
 #pragma unroll
-          for (int u = 0; u < 16; u += 2)
-            fma2(oacc[ch * 16 + u], oacc[ch * 16 + u + 1], alpha, alpha, oacc[ch * 16 + u], oacc[ch * 16 + u + 1],
-                 __uint_as_float(r[u]), __uint_as_float(r[u + 1]));
+            for (int u = 0; u < 16; ++u) {
+              const float2 f = h16x2_to_f32x2(r[u]);
+              fma2(oacc[ch * 32 + 2 * u], oacc[ch * 32 + 2 * u + 1], alpha, alpha, oacc[ch * 32 + 2 * u],
+                   oacc[ch * 32 + 2 * u + 1], f.x, f.y);
+            }
+          }
+        } else {
+#pragma unroll
+          for (int ch = 0; ch < D / 16; ++ch) {
+            uint32_t r[16];
+            tmem_ld16(ob + ch * 16, r);
+            tmem_wait_ld(r);
+#pragma unroll
+            for (int u = 0; u < 16; u += 2)
+              fma2(oacc[ch * 16 + u], oacc[ch * 16 + u + 1], alpha, alpha, oacc[ch * 16 + u], oacc[ch * 16 + u + 1],
+                   __uint_as_float(r[u]), __uint_as_float(r[u + 1]));
+          }
         }
         tc_fence_before();
         mbar_arrive(bar(C::B_OREADY));
@@ -1022,7 +1047,7 @@ __global__ void __launch_bounds__(128, 1) qk_tile_kernel(const int8_t* qt, const
     mbar_expect_tx(smem_u32(&bars[0]), 2 * bytes);
     bulk_g2s(smem_u32(sq), qt, bytes, smem_u32(&bars[0]));
     bulk_g2s(smem_u32(sk), kt, bytes, smem_u32(&bars[0]));
-    if (mbar_wait(smem_u32(&bars[0]), 0, &abort_flag, err, kErrTimeoutMma)) {
+    if (mbar_wait_poll(smem_u32(&bars[0]), 0, &abort_flag, err, kErrTimeoutMma)) {
       tc_fence_after();
       for (int kk = 0; kk < D / 32; ++kk)
         mma_i8_ss(tmem, smem_desc(smem_u32(sq) + kk * 32, D), smem_desc(smem_u32(sk) + kk * 32, D),
@@ -1055,11 +1080,12 @@ __global__ void __launch_bounds__(128, 1) qk_tile_kernel(const int8_t* qt, const
 
 // ---------------------------------------------------------------- launchers
 // Persistent grid: one CTA per SM (each holds all of an SM's tensor memory),
-// fewer when there are fewer items.
-template <int D, bool PV8, bool ACC2>
+// fewer when there are fewer items, or p.max_ctas when that is set (a debug
+// cap: results do not depend on the grid).
+template <int D, bool PV8, bool ACC2, bool A16>
 static cudaError_t launch_attn(const AttnParams& p, cudaStream_t s) {
   using C = AttnCfg<D, PV8, ACC2>;
-  auto k = attn_fwd_kernel<D, PV8, ACC2>;
+  auto k = attn_fwd_kernel<D, PV8, ACC2, A16>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // the register split needs the launch allocation it was sized for: with
@@ -1070,12 +1096,7 @@ static cudaError_t launch_attn(const AttnParams& p, cudaStream_t s) {
   int dev = 0, sms = 0;
   if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-  // SAGE_MAX_CTAS caps the persistent grid (tests use it to make a few CTAs
-  // walk many items; results do not depend on it)
-  if (const char* cap = getenv("SAGE_MAX_CTAS")) {
-    const int c = atoi(cap);
-    if (c > 0 && c < sms) sms = c;
-  }
+  if (p.max_ctas > 0 && p.max_ctas < sms) sms = p.max_ctas;
   const int grid = p.n_items < sms ? p.n_items : sms;
   k<<<grid, C::NTHREADS, C::SMEM_BYTES, s>>>(p);
   return cudaGetLastError();
@@ -1087,23 +1108,31 @@ int attn_tiles_per_cta(int D, bool pv8, bool acc2) {
   return acc2 ? 1 : 2;
 }
 
-cudaError_t attn_forward(const AttnParams& p0, int D, bool pv8, bool acc2, int max_len_q, int nseq,
+cudaError_t attn_forward(const AttnParams& p0, int D, bool pv8, int acc, int max_len_q, int nseq,
                          cudaStream_t s) {
+  const bool acc2 = acc != kAccOne;
   const int per = attn_tiles_per_cta(D, pv8, acc2) * kTile;
   const long long nx = (max_len_q + per - 1) / per;
   const long long items = nx * p0.Hq * nseq;
   if (items == 0) return cudaSuccess;
   if (items > 0x7fffffffLL) return cudaErrorInvalidValue;
+  if (acc == kAccTwoF16 && !pv8) return cudaErrorInvalidValue;
   AttnParams p = p0;
   p.n_pairs = (int)nx;
   p.nseq = nseq;
   p.n_items = (int)items;
   if (D == 128) {
-    if (pv8) return acc2 ? launch_attn<128, true, true>(p, s) : launch_attn<128, true, false>(p, s);
-    return acc2 ? launch_attn<128, false, true>(p, s) : launch_attn<128, false, false>(p, s);
+    if (pv8) {
+      if (acc == kAccTwoF16) return launch_attn<128, true, true, true>(p, s);
+      return acc2 ? launch_attn<128, true, true, false>(p, s) : launch_attn<128, true, false, false>(p, s);
+    }
+    return acc2 ? launch_attn<128, false, true, false>(p, s) : launch_attn<128, false, false, false>(p, s);
   }
-  if (pv8) return acc2 ? launch_attn<64, true, true>(p, s) : launch_attn<64, true, false>(p, s);
-  return acc2 ? launch_attn<64, false, true>(p, s) : launch_attn<64, false, false>(p, s);
+  if (pv8) {
+    if (acc == kAccTwoF16) return launch_attn<64, true, true, true>(p, s);
+    return acc2 ? launch_attn<64, true, true, false>(p, s) : launch_attn<64, true, false, false>(p, s);
+  }
+  return acc2 ? launch_attn<64, false, true, false>(p, s) : launch_attn<64, false, false, false>(p, s);
 }
 
 cudaError_t debug_qk_tile(const int8_t* qt, const int8_t* kt, int D, int32_t* out, uint32_t* err,

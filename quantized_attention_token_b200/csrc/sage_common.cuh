@@ -149,21 +149,38 @@ __device__ __forceinline__ uint32_t mbar_try_wait_sleep(uint32_t bar, uint32_t p
   return ok;
 }
 
-// Bounded wait: sleeps in try_wait (20 us hints); between tries it checks the
-// CTA's abort flag and a wall-clock limit.  On timeout it sets the abort flag
-// and the given bit in the device error word and returns false; the caller
-// then leaves its loop so that the CTA tears down cleanly.
+// Bounded wait of a whole warp (all 32 lanes call it at the same place): it
+// sleeps in try_wait (20 us hints); between tries it checks the CTA's abort
+// flag and a wall-clock limit.  On timeout it sets the abort flag and the
+// given bit in the device error word and returns false; the caller then
+// leaves its loop so that the CTA tears down cleanly.  Every decision is
+// taken for the warp as a whole (vote), so its lanes leave together and the
+// warp-collective tcgen05 instructions that follow never see a split warp.
+// Once one lane has seen the phase complete, the others see it too: the
+// barriers waited on here cannot complete their next phase before this warp
+// has moved on (each next phase needs an arrival that follows this wait).
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                           uint32_t* err, uint32_t bit) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (__all_sync(0xffffffffu, mbar_try_wait(bar, parity))) return true;
   const uint64_t t0 = global_timer_ns();
   for (;;) {
-    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
-    if (*abort_flag) return false;
-    if (global_timer_ns() - t0 > kWaitLimitNs) {
-      *abort_flag = 1;
+    const bool done = mbar_try_wait_sleep(bar, parity, 20000u);
+    if (__any_sync(0xffffffffu, done)) {
+      bool seen = done;
+      for (uint32_t i = 0; !seen && i < (1u << 20); ++i) seen = mbar_try_wait(bar, parity);
+      if (__all_sync(0xffffffffu, seen)) return true;
+      *abort_flag = 1;                     // not reached (see above); leave together all the same
       atomicOr(err, bit);
+      return false;
+    }
+    const uint32_t aborted = __ballot_sync(0xffffffffu, *abort_flag != 0);
+    const uint32_t late = __ballot_sync(0xffffffffu, global_timer_ns() - t0 > kWaitLimitNs);
+    if (aborted | late) {
+      if (!aborted) {                      // this warp's wait is the one that ran out
+        *abort_flag = 1;
+        atomicOr(err, bit);
+      }
       return false;
     }
   }
@@ -293,6 +310,10 @@ __host__ __device__ constexpr uint32_t idesc_i8(int M, int N) {
 __host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N) {
   return (1u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
 }
+// E4M3 x E4M3 with a binary16 accumulator (format 0).
+__host__ __device__ constexpr uint32_t idesc_e4m3_acc16(int M, int N) {
+  return (0u << 4) | (0u << 7) | (0u << 10) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
 __host__ __device__ constexpr uint32_t idesc_f16(int M, int N, bool bf16) {
   return (1u << 4) | ((bf16 ? 1u : 0u) << 7) | ((bf16 ? 1u : 0u) << 10) | ((uint32_t)(N >> 3) << 17) |
          ((uint32_t)(M >> 4) << 24);
@@ -328,6 +349,18 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+        "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
+// 32 columns of 16-bit values (one per column, as a binary16 accumulator
+// holds them), two adjacent columns packed per register (lower column in the
+// lower half).
+__device__ __forceinline__ void tmem_ld32_pack16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.pack::16b.b32 "
       "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
       : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
         "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
@@ -464,6 +497,10 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %2, %1;" : "=r"(r) : "f"(lo), "f"(hi));
   return r;
+}
+// Two binary16 values (lower half first) to two floats (exact).
+__device__ __forceinline__ float2 h16x2_to_f32x2(uint32_t v) {
+  return __half22float2(*reinterpret_cast<const __half2*>(&v));
 }
 __device__ __forceinline__ float h16_to_f32(uint16_t bits, bool bf16) {
   return bf16 ? __uint_as_float((uint32_t)bits << 16) : __half2float(__ushort_as_half(bits));

@@ -6,8 +6,8 @@
 
 namespace sage {
 
-// One launch of the persistent pre-pass: which tensors to quantize, where
-// they are, and the workspace regions it fills.
+// One pre-pass job (its launches): which tensors to quantize, where they
+// are, and the workspace regions it fills.
 struct PrepassJob {
   const uint16_t* q = nullptr;
   const uint16_t* k = nullptr;
@@ -27,7 +27,7 @@ struct PrepassJob {
   float* k_mean = nullptr;                // [nseq][Hkv][D]
   float* v_scale = nullptr;               // [nseq][Hkv][D]
   int8_t* q_codes = nullptr;
-  float* q_scale = nullptr;               // [Hq][tiles_q][32]
+  float* q_scale = nullptr;               // [Hq][tiles_q][128] (group g of a tile at [g])
   int8_t* k_codes = nullptr;
   float* k_scale = nullptr;               // [Hkv][tiles_k][16]
   uint8_t* v_codes = nullptr;
@@ -57,7 +57,14 @@ struct AttnParams {
   int causal;
   int out_bf16;
   int n_pairs, nseq, n_items;  // work items: n_pairs query-tile groups x Hq heads x nseq sequences (set by attn_forward)
+  int max_ctas;              // debug: cap on the persistent grid (0: one CTA per SM)
+  int dbg_withhold_k;        // debug: CTA 0 skips the copy of this K tile of its ring (-1: none)
 };
+
+// P~V accumulation of the attention kernel: one FP32 TMEM accumulator across
+// all KV tiles, or a fresh per-tile partial (FP32 or binary16) added into an
+// FP32 register accumulator.
+enum { kAccOne = 0, kAccTwo = 1, kAccTwoF16 = 2 };
 
 // prepass.cu
 cudaError_t prepass_run(const PrepassJob& j, int D, cudaStream_t s);
@@ -66,7 +73,7 @@ cudaError_t prepass_varlen_offsets(const int* cu_q, const int* cu_k, int n, int 
 
 // attn_fwd.cu
 int attn_tiles_per_cta(int D, bool pv8, bool acc2);
-cudaError_t attn_forward(const AttnParams& p, int D, bool pv8, bool acc2, int max_len_q, int nseq,
+cudaError_t attn_forward(const AttnParams& p, int D, bool pv8, int acc, int max_len_q, int nseq,
                          cudaStream_t s);
 cudaError_t debug_qk_tile(const int8_t* qt, const int8_t* kt, int D, int32_t* out, uint32_t* err,
                           cudaStream_t s);

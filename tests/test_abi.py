@@ -64,7 +64,8 @@ def test_workspace_planner(L):
     (dict(ws=0x1010), sage.ERR_INVALID_ARG),         # ws must be 256-byte aligned
     (dict(gran=7), sage.ERR_INVALID_ARG),
     (dict(pv=3), sage.ERR_INVALID_ARG),
-    (dict(acc=3), sage.ERR_INVALID_ARG),
+    (dict(acc=4), sage.ERR_INVALID_ARG),
+    (dict(acc=3, pv=1), sage.ERR_UNSUPPORTED),       # binary16 inner accumulation needs FP8 P~V
     (dict(layout=2), sage.ERR_INVALID_ARG),
     (dict(dtype=2), sage.ERR_INVALID_ARG),
     (dict(ws_bytes=1000), sage.ERR_WORKSPACE),
@@ -101,6 +102,22 @@ def test_varlen_rejects_bad_arguments(L):
     assert L.sage_attn_varlen_fwd(*bad) == sage.ERR_UNSUPPORTED
     bad = list(base); bad[21] = 4096
     assert L.sage_attn_varlen_fwd(*bad) == sage.ERR_WORKSPACE
+
+
+def test_debug_settings_validate_and_reset(L):
+    assert L.sage_debug_set_max_ctas(-1) == sage.ERR_INVALID_ARG
+    assert L.sage_debug_withhold_k_tile(-2) == sage.ERR_INVALID_ARG
+    assert L.sage_debug_set_max_ctas(3) == sage.OK and L.sage_debug_set_max_ctas(0) == sage.OK
+    assert L.sage_debug_withhold_k_tile(5) == sage.OK and L.sage_debug_withhold_k_tile(-1) == sage.OK
+
+
+def test_library_reads_no_environment():
+    """Behaviour is selected through arguments and the debug entry points
+    only: no source of the library reads the process environment."""
+    csrc = os.path.join(ROOT, "quantized_attention_token_b200", "csrc")
+    for f in os.listdir(csrc):
+        src = open(os.path.join(csrc, f)).read()
+        assert "getenv" not in src, f
 
 
 def test_status_strings(L):

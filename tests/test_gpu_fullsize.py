@@ -1,6 +1,17 @@
 """Parity at the full sizes of the workloads, in the launch configuration the
 benchmark times: the GPU computes the whole problem, the oracle recomputes
-sampled query tiles (all keys) of sampled heads one by one."""
+sampled query tiles (all keys) of sampled heads one by one.
+
+Besides the element-wise comparison (2e-3 + the oracle's allowance for
+ambiguous P~ roundings), each test holds the allowance itself down: it must
+never exceed 1e-3 (half the gate) and must be above 1e-4 (5 % of the gate)
+on fewer than 2 % of the sampled outputs, so that the 2e-3 gate is what the
+comparison actually enforces.  The share of outputs with any allowance at all
+is printed: it grows with the row length (one ambiguous P~ among a row's
+keys gives the whole row a small allowance -- about 4-7 % of rows at 4096
+keys, most rows at 32768 keys, each then of order 1e-6 to 1e-5).  Accuracy against exact fp64
+attention: cosine >= 0.999; relative L1 <= 0.02 (16-bit P~V) or <= the
+oracle's own + 0.002 (FP8 P~V, whose E4M3 rounding alone costs 0.034-0.038)."""
 import numpy as np
 import pytest
 import torch
@@ -8,12 +19,12 @@ import torch
 import oracle
 import synth
 import quantized_attention_token_b200 as sage
-from tests.test_gpu_parity import _assert_close
+from tests.test_gpu_parity import _accuracy, _assert_close
 
 pytestmark = pytest.mark.gpu
 
 
-def _oracle_rows(spec, q, k, v, b, h, rows, gran, pv, smooth_q=False, smooth_v=False, lazy_tau=0):
+def _oracle_rows(spec, q, k, v, b, h, rows, gran, pv, smooth_q=False, smooth_v=False, lazy_tau=0, acc="fp32"):
     """Oracle output and allowance for rows [r0, r1) of (sequence b, head h),
     computed on that sequence / head alone."""
     grp = spec.Hq // spec.Hkv
@@ -30,7 +41,8 @@ def _oracle_rows(spec, q, k, v, b, h, rows, gran, pv, smooth_q=False, smooth_v=F
         qs, ks, vs = q[b:b + 1, :, h:h + 1], k[b:b + 1, :, hk:hk + 1], v[b:b + 1, :, hk:hk + 1]
         lay = "NHD"
     out, allow = oracle.attention(qs, ks, vs, lay, spec.causal, gran=gran, pv=pv, q_rows={(0, 0): rows},
-                                  smooth_q=smooth_q, smooth_v=smooth_v, lazy_tau=lazy_tau, with_allowance=True)
+                                  smooth_q=smooth_q, smooth_v=smooth_v, lazy_tau=lazy_tau, with_allowance=True,
+                                  acc=acc)
     sel = (slice(0, 1), slice(0, 1), slice(*rows)) if lay == "HND" else (slice(0, 1), slice(*rows), slice(0, 1))
     pb = oracle.problem(qs, ks, vs, lay)
     ex = oracle.attn_exact_head(pb.q[0][0][rows[0]:rows[1]], pb.k[0][0], pb.v[0][0], spec.causal,
@@ -65,14 +77,28 @@ def _run(spec, gran="per_block", pv="fp8", acc="fp32+fp32", smooth_q=False, smoo
 
 def _check(spec, samples, gran="per_block", pv="fp8", acc="fp32+fp32", smooth_q=False, smooth_v=False):
     q, k, v, out = _run(spec, gran, pv, acc, smooth_q, smooth_v)
+    allows, gots, exs, refs = [], [], [], []
     for b, h, rows in samples:
         tau = (2 if pv == "fp8" else 8) if acc == "fp32_lazy" else 0
-        ref, allow, ex = _oracle_rows(spec, q, k, v, b, h, rows, gran, pv, smooth_q, smooth_v, tau)
+        ref, allow, ex = _oracle_rows(spec, q, k, v, b, h, rows, gran, pv, smooth_q, smooth_v, tau,
+                                      acc if acc == "fp32+fp16" else "fp32")
         got = _gpu_rows(spec, out, b, h, rows)
         _assert_close(got, (ref, allow), spec.dtype, f"{spec.name} b{b} h{h} rows{rows}")
-        o = got.double().numpy().ravel()
-        cos = o @ ex.ravel() / (np.linalg.norm(o) * np.linalg.norm(ex))
-        assert cos >= 0.999, (spec.name, b, h, rows, cos)
+        allows.append(allow.ravel())
+        gots.append(got.double().numpy().ravel())
+        exs.append(ex.ravel())
+        refs.append(ref.ravel())
+    a = np.concatenate(allows)
+    o, e, r = np.concatenate(gots), np.concatenate(exs), np.concatenate(refs)
+    cos, rl1 = _accuracy(o, e)
+    bound = 0.02 if pv == "fp16" else _accuracy(r, e)[1] + 0.002
+    print(f"{spec.name} {pv}/{acc}: allowance max {a.max():.2e}, non-zero {np.mean(a > 0):.3%}, "
+          f"> 1e-4 {np.mean(a > 1e-4):.3%}; cos {cos:.5f}, rel-L1 {rl1:.4f} (bound {bound:.4f})")
+    assert cos >= 0.999, (spec.name, cos)
+    assert rl1 <= bound, (spec.name, rl1, bound)
+    if acc != "fp32+fp16":          # there the allowance also carries the binary16 partial sums' roundings
+        assert a.max() <= 1e-3, a.max()
+        assert np.mean(a > 1e-4) < 0.02, np.mean(a > 1e-4)
 
 
 @pytest.mark.parametrize("pv,acc", [("fp8", "fp32+fp32"), ("fp8", "fp32"), ("fp16", "fp32+fp32")])
@@ -119,3 +145,24 @@ def test_varlen_gqa_smooth_v():
 def test_b2_h32_s4096_d128_lazy_rescale():
     spec = synth.CONFIGS["b2_h32_s4096_d128"]
     _check(spec, [(0, 5, (0, 128)), (1, 27, (3968, 4096))], acc="fp32_lazy")
+
+
+@pytest.mark.parametrize("name,gran", [("sweep_S4096_D64", "per_block"), ("sweep_S16384_D64", "per_thread"),
+                                       ("sweep_S16384_D128", "per_warp")])
+def test_sweep_points_more(name, gran):
+    """Further points of the metric's sequence axis: D = 64 at S = 4096 and
+    16384, per-warp granularity at S = 16384."""
+    spec = synth.CONFIGS[name]
+    last = spec.S - 128
+    _check(spec, [(0, 0, (0, 128)), (spec.B - 1, 31, (last, spec.S)), (spec.B // 2, 13, (spec.S // 2, spec.S // 2 + 128))],
+           gran=gran, acc="fp32")
+
+
+def test_varlen_gqa_causal_two_level():
+    spec = synth.CONFIGS["varlen_gqa"]
+    _check(spec, [(3, 1, (16256, 16384)), (2, 30, (0, 128)), (1, 12, (1024, 1152))], acc="fp32+fp32")
+
+
+def test_b2_h32_s4096_d128_fp16_accumulation():
+    spec = synth.CONFIGS["b2_h32_s4096_d128"]
+    _check(spec, [(0, 2, (0, 128)), (1, 29, (3968, 4096)), (0, 15, (2048, 2176))], acc="fp32+fp16")

@@ -2,9 +2,15 @@
 
 Integer / byte work (INT8 codes, E4M3 codes, int32 scores) must match bit for
 bit; outputs within max-abs 2e-3 of the oracle (plus half an ulp of the
-output's 16-bit type, which the rounded output carries on top); accuracy
-against exact fp64 attention: cosine >= 0.999.
+output's 16-bit type, which the rounded output carries on top, plus the
+oracle's per-output allowance for P~ values whose rounding is ambiguous within
+the derived exp2 error band); accuracy against exact fp64 attention: cosine >=
+0.999 and relative L1 <= 0.02 with 16-bit P~V.  With FP8 P~V the method itself
+(the oracle, computed exactly) lands at 0.034-0.038 relative L1 on zero-mean
+iid inputs -- E4M3 keeps three fraction bits -- so the GPU output is held to
+the oracle's own relative L1 + 0.002 there.
 """
+import contextlib
 import math
 
 import numpy as np
@@ -40,6 +46,34 @@ def _assert_close(out: torch.Tensor, ref, dtype: str, what=""):
     err = np.abs(o - ref)
     bad = ~(err <= _tol(ref, dtype, allow))          # a NaN anywhere counts as outside
     assert not bad.any(), f"{what}: {bad.sum()} of {bad.size} outside tolerance, max err {np.nanmax(err):.3e}"
+
+
+def _accuracy(o: np.ndarray, ex: np.ndarray):
+    o, ex = np.asarray(o, np.float64).ravel(), np.asarray(ex, np.float64).ravel()
+    cos = float(o @ ex / (np.linalg.norm(o) * np.linalg.norm(ex)))
+    rl1 = float(np.abs(o - ex).sum() / np.abs(ex).sum())
+    return cos, rl1
+
+
+def _check_accuracy(out, ex: np.ndarray, ref: np.ndarray, pv: str, what=""):
+    """cosine >= 0.999 against exact fp64 attention, and relative L1 <= 0.02
+    (16-bit P~V) or <= the oracle's own relative L1 + 0.002 (FP8 P~V)."""
+    o = out.double().cpu().numpy() if isinstance(out, torch.Tensor) else out
+    cos, rl1 = _accuracy(o, ex)
+    assert cos >= 0.999, (what, cos)
+    bound = 0.02 if pv == "fp16" else _accuracy(ref, ex)[1] + 0.002
+    assert rl1 <= bound, (what, rl1, bound)
+    return cos, rl1
+
+
+@contextlib.contextmanager
+def max_ctas(n):
+    """Cap the attention kernel's persistent grid for the duration."""
+    sage.debug_set_max_ctas(int(n or 0))
+    try:
+        yield
+    finally:
+        sage.debug_set_max_ctas(0)
 
 
 def _ws_bytes(ws: torch.Tensor) -> np.ndarray:
@@ -211,6 +245,9 @@ CASES = [
     (128, 127, 2, 2, True, "per_block", "fp8", "fp32+fp32", "fp16", "HND"),
     (128, 400, 4, 2, True, "per_token", "fp8", "fp32", "fp16", "HND"),
     (64, 300, 2, 2, False, "per_token", "fp16", "fp32+fp32", "bf16", "NHD"),
+    (64, 256, 2, 2, False, "per_block", "fp8", "fp32+fp16", "fp16", "HND"),
+    (128, 300, 4, 2, True, "per_thread", "fp8", "fp32+fp16", "bf16", "NHD"),
+    (128, 520, 2, 1, False, "per_warp", "fp8", "fp32+fp16", "fp16", "HND"),
 ]
 
 
@@ -222,12 +259,9 @@ def test_attention_matches_oracle(D, S, Hq, Hkv, causal, gran, pv, acc, dtype, l
     out = sage.sageattn(_dev(q), _dev(k), _dev(v), layout, causal, qk_quant_gran=gran, pv_dtype=pv,
                         pv_accum_dtype=acc)
     torch.cuda.synchronize()
-    ref = oracle.attention(q, k, v, layout, causal, gran=gran, pv=pv, with_allowance=True)
+    ref = oracle.attention(q, k, v, layout, causal, gran=gran, pv=pv, with_allowance=True, acc=acc)
     _assert_close(out, ref, dtype, "vs oracle")
-    ex = oracle.attention_exact(q, k, v, layout, causal)
-    o = out.double().cpu().numpy().ravel()
-    cos = o @ ex.ravel() / (np.linalg.norm(o) * np.linalg.norm(ex))
-    assert cos >= 0.999, cos
+    _check_accuracy(out, oracle.attention_exact(q, k, v, layout, causal), ref[0], pv, "vs fp64")
 
 
 @pytest.mark.parametrize("D,S,causal,gran,pv,acc,dtype,layout", [
@@ -247,10 +281,7 @@ def test_attention_smooth_q_matches_oracle(D, S, causal, gran, pv, acc, dtype, l
     torch.cuda.synchronize()
     ref = oracle.attention(q, k, v, layout, causal, gran=gran, pv=pv, smooth_q=True, with_allowance=True)
     _assert_close(out, ref, dtype, "smooth Q vs oracle")
-    ex = oracle.attention_exact(q, k, v, layout, causal)
-    o = out.double().cpu().numpy().ravel()
-    cos = o @ ex.ravel() / (np.linalg.norm(o) * np.linalg.norm(ex))
-    assert cos >= 0.999, cos
+    _check_accuracy(out, oracle.attention_exact(q, k, v, layout, causal), ref[0], pv, "smooth Q vs fp64")
 
 
 @pytest.mark.parametrize("D,S,causal,acc,dtype,layout", [
@@ -269,10 +300,7 @@ def test_attention_smooth_v_matches_oracle(D, S, causal, acc, dtype, layout):
     torch.cuda.synchronize()
     ref = oracle.attention(q, k, v, layout, causal, pv="fp8", smooth_v=True, with_allowance=True)
     _assert_close(out, ref, dtype, "smooth V vs oracle")
-    ex = oracle.attention_exact(q, k, v, layout, causal)
-    o = out.double().cpu().numpy().ravel()
-    cos = o @ ex.ravel() / (np.linalg.norm(o) * np.linalg.norm(ex))
-    assert cos >= 0.999, cos
+    _check_accuracy(out, oracle.attention_exact(q, k, v, layout, causal), ref[0], "fp8", "smooth V vs fp64")
 
 
 def test_varlen_smooth_v_matches_oracle():
@@ -305,10 +333,7 @@ def test_attention_lazy_rescale_matches_oracle(D, S, causal, gran, pv, dtype, la
     ref = oracle.attention(q, k, v, layout, causal, gran=gran, pv=pv, lazy_tau=2 if pv == "fp8" else 8,
                            with_allowance=True)
     _assert_close(out, ref, dtype, "lazy rescale vs oracle")
-    ex = oracle.attention_exact(q, k, v, layout, causal)
-    o = out.double().cpu().numpy().ravel()
-    cos = o @ ex.ravel() / (np.linalg.norm(o) * np.linalg.norm(ex))
-    assert cos >= 0.999, cos
+    _check_accuracy(out, oracle.attention_exact(q, k, v, layout, causal), ref[0], pv, "lazy vs fp64")
 
 
 def test_tiny_config():
@@ -316,7 +341,9 @@ def test_tiny_config():
     q, k, v = synth.make(sp)
     out = sage.sageattn(_dev(q), _dev(k), _dev(v), "HND", False)
     torch.cuda.synchronize()
-    _assert_close(out, oracle.attention(q, k, v, with_allowance=True), "fp16", "tiny")
+    ref = oracle.attention(q, k, v, with_allowance=True)
+    _assert_close(out, ref, "fp16", "tiny")
+    _check_accuracy(out, oracle.attention_exact(q, k, v), ref[0], "fp8", "tiny vs fp64")
 
 
 @pytest.mark.parametrize("causal", [True, False])
@@ -382,71 +409,70 @@ def test_one_level_accumulation_as_accurate_as_two_level(pv):
 
 
 # ----------------------------------------------------------------------------- persistent grid
-@pytest.mark.parametrize("max_ctas", ["1", "3"])
+@pytest.mark.parametrize("n_ctas", [1, 3])
 @pytest.mark.parametrize("D,S,causal,pv,acc,gran,dtype,layout", [
     (128, 600, False, "fp8", "fp32", "per_block", "fp16", "HND"),
     (128, 600, True, "fp8", "fp32", "per_warp", "bf16", "NHD"),
     (64, 520, True, "fp16", "fp32", "per_block", "fp16", "HND"),
     (128, 300, True, "fp8", "fp32+fp32", "per_thread", "fp16", "HND"),
     (64, 700, False, "fp16", "fp32+fp32", "per_token", "bf16", "NHD"),
+    (128, 600, True, "fp8", "fp32+fp16", "per_block", "fp16", "HND"),
 ])
-def test_persistent_items_match_oracle(monkeypatch, max_ctas, D, S, causal, pv, acc, gran, dtype, layout):
+def test_persistent_items_match_oracle(n_ctas, D, S, causal, pv, acc, gran, dtype, layout):
     """A capped grid, so that each CTA walks many items one after the other:
     the mbarrier phases, the K/V ring, the Q reloads and the FP8 token run on
     across items, including tail items whose second query tile is empty."""
-    monkeypatch.setenv("SAGE_MAX_CTAS", max_ctas)
     sp = synth.Spec("t", Hq=4, Hkv=2, D=D, B=2, S=S, dtype=dtype, layout=layout, causal=causal, k_bias_std=3.0,
                     seed=120 + S)
     q, k, v = synth.make(sp)
-    out = sage.sageattn(_dev(q), _dev(k), _dev(v), layout, causal, qk_quant_gran=gran, pv_dtype=pv,
-                        pv_accum_dtype=acc)
-    torch.cuda.synchronize()
-    ref = oracle.attention(q, k, v, layout, causal, gran=gran, pv=pv, with_allowance=True)
-    _assert_close(out, ref, dtype, f"{max_ctas} CTAs vs oracle")
+    with max_ctas(n_ctas):
+        out = sage.sageattn(_dev(q), _dev(k), _dev(v), layout, causal, qk_quant_gran=gran, pv_dtype=pv,
+                            pv_accum_dtype=acc)
+        torch.cuda.synchronize()
+    ref = oracle.attention(q, k, v, layout, causal, gran=gran, pv=pv, with_allowance=True, acc=acc)
+    _assert_close(out, ref, dtype, f"{n_ctas} CTAs vs oracle")
 
 
-@pytest.mark.parametrize("pv,acc", [("fp8", "fp32"), ("fp16", "fp32"), ("fp8", "fp32+fp32")])
-def test_persistent_varlen_gqa_matches_oracle(monkeypatch, pv, acc):
+@pytest.mark.parametrize("pv,acc", [("fp8", "fp32"), ("fp16", "fp32"), ("fp8", "fp32+fp32"), ("fp8", "fp32+fp16")])
+def test_persistent_varlen_gqa_matches_oracle(pv, acc):
     """Two CTAs over the items of six sequences (one empty, one of a single
     token), causal, grouped heads."""
-    monkeypatch.setenv("SAGE_MAX_CTAS", "2")
     sp = synth.Spec("t", Hq=4, Hkv=2, D=128, seqlens=[200, 1, 0, 129, 384, 77], causal=True, seed=52)
     q, k, v = synth.make(sp)
     cu = sp.cu_seqlens()
     cu_d = torch.from_numpy(cu).cuda()
-    out = sage.sageattn_varlen(_dev(q), _dev(k), _dev(v), cu_d, cu_d, max(sp.seqlens), True, pv_dtype=pv,
-                               pv_accum_dtype=acc)
-    torch.cuda.synchronize()
-    ref = oracle.attention(q, k, v, causal=True, pv=pv, cu_seqlens=cu, with_allowance=True)
+    with max_ctas(2):
+        out = sage.sageattn_varlen(_dev(q), _dev(k), _dev(v), cu_d, cu_d, max(sp.seqlens), True, pv_dtype=pv,
+                                   pv_accum_dtype=acc)
+        torch.cuda.synchronize()
+    ref = oracle.attention(q, k, v, causal=True, pv=pv, cu_seqlens=cu, with_allowance=True, acc=acc)
     _assert_close(out, ref, "fp16", "varlen, 2 CTAs")
 
 
-@pytest.mark.parametrize("acc", ["fp32", "fp32+fp32", "fp32_lazy"])
-def test_persistent_smooth_qv_matches_oracle(monkeypatch, acc):
+@pytest.mark.parametrize("acc", ["fp32", "fp32+fp32", "fp32_lazy", "fp32+fp16"])
+def test_persistent_smooth_qv_matches_oracle(acc):
     """Smooth Q (its per-key corrections ride with each V tile through the
     ring) and smooth V with one CTA walking all items."""
-    monkeypatch.setenv("SAGE_MAX_CTAS", "1")
     sp = synth.Spec("t", Hq=4, Hkv=2, D=128, B=2, S=400, dtype="fp16", layout="HND", causal=False, k_bias_std=3.0,
                     q_block_offset_std=1.0, seed=130)
     q, k, v = synth.make(sp)
     v = v + torch.from_numpy(np.random.default_rng(13).normal(0, 8, 128).astype(np.float32)).to(v.dtype)
-    out = sage.sageattn(_dev(q), _dev(k), _dev(v), "HND", False, pv_dtype="fp8", pv_accum_dtype=acc,
-                        smooth_q=True, smooth_v=True)
-    torch.cuda.synchronize()
+    with max_ctas(1):
+        out = sage.sageattn(_dev(q), _dev(k), _dev(v), "HND", False, pv_dtype="fp8", pv_accum_dtype=acc,
+                            smooth_q=True, smooth_v=True)
+        torch.cuda.synchronize()
     ref = oracle.attention(q, k, v, "HND", False, pv="fp8", smooth_q=True, smooth_v=True,
-                           lazy_tau=2 if acc == "fp32_lazy" else 0, with_allowance=True)
+                           lazy_tau=2 if acc == "fp32_lazy" else 0, with_allowance=True, acc=acc)
     _assert_close(out, ref, "fp16", "smooth Q+V, 1 CTA")
 
 
-@pytest.mark.parametrize("max_ctas", [None, "2"])
+@pytest.mark.parametrize("n_ctas", [0, 2])
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("pv,acc", [("fp8", "fp32"), ("fp16", "fp32"), ("fp8", "fp32+fp32")])
-def test_varlen_cross_length_matches_oracle(monkeypatch, max_ctas, causal, pv, acc):
+def test_varlen_cross_length_matches_oracle(n_ctas, causal, pv, acc):
     """Queries and keys with their own sequence boundaries (more keys, fewer
     keys, no queries, no keys), grouped heads; a sequence without keys gives
     zero rows."""
-    if max_ctas:
-        monkeypatch.setenv("SAGE_MAX_CTAS", max_ctas)
     rng = np.random.default_rng(7)
     H, Hk, D = 4, 2, 128
     lq, lk = [150, 40, 0, 200, 17, 300], [90, 300, 10, 0, 17, 260]
@@ -455,10 +481,76 @@ def test_varlen_cross_length_matches_oracle(monkeypatch, max_ctas, causal, pv, a
     q = torch.from_numpy(rng.normal(size=(cq[-1], H, D)).astype(np.float16))
     k = torch.from_numpy((rng.normal(size=(ck[-1], Hk, D)) + rng.normal(0, 3, size=(1, Hk, D))).astype(np.float16))
     v = torch.from_numpy(rng.normal(size=(ck[-1], Hk, D)).astype(np.float16))
-    out = sage.sageattn_varlen(_dev(q), _dev(k), _dev(v), torch.from_numpy(cq).cuda(), torch.from_numpy(ck).cuda(),
-                               max(max(lq), max(lk)), causal, pv_dtype=pv, pv_accum_dtype=acc)
-    torch.cuda.synchronize()
+    with max_ctas(n_ctas):
+        out = sage.sageattn_varlen(_dev(q), _dev(k), _dev(v), torch.from_numpy(cq).cuda(),
+                                   torch.from_numpy(ck).cuda(), max(max(lq), max(lk)), causal, pv_dtype=pv,
+                                   pv_accum_dtype=acc)
+        torch.cuda.synchronize()
     ref = oracle.attention(q, k, v, causal=causal, pv=pv, cu_seqlens=cq, cu_seqlens_k=ck, with_allowance=True)
     _assert_close(out, ref, "fp16", "cross-length varlen vs oracle")
     b = lk.index(0)
     assert torch.count_nonzero(out[cq[b]:cq[b + 1]]).item() == 0
+
+
+# ----------------------------------------------------------------------------- fp32+fp16 accumulation
+def test_fp16_accumulation_partials_round_like_the_oracle():
+    """Q = 0 makes every P~ exactly 1 (the scale-1 code); V of E4M3 integers
+    with channel maximum 448 makes V's codes V itself.  Each 32-key chunk's
+    sum is an integer and the tile's binary16 partial is the chain of
+    roundings the oracle computes: the GPU must agree within one binary16
+    ulp per rounding (the oracle's allowance), and the rounding must show."""
+    S, D = 512, 128
+    rng = np.random.default_rng(42)
+    vals = np.array([448, 416, 352, 320, 13, 11, 9, 7, 3, 1, 0, -1, -5, -15, -448], np.float64)
+    vv = vals[rng.integers(0, len(vals), (S, D))]
+    vv[0, :] = 448.0
+    q = torch.zeros(1, 1, S, D, dtype=torch.float16)
+    k = torch.randn(1, 1, S, D, generator=torch.Generator().manual_seed(2)).half()
+    v = torch.from_numpy(vv.astype(np.float16)).view(1, 1, S, D)
+    out = sage.sageattn(_dev(q), _dev(k), _dev(v), "HND", False, pv_dtype="fp8", pv_accum_dtype="fp32+fp16")
+    torch.cuda.synchronize()
+    ref = oracle.attention(q, k, v, pv="fp8", acc="fp32+fp16", with_allowance=True)
+    _assert_close(out, ref, "fp16", "fp16 partials")
+    exact_mean = vv.mean(axis=0)
+    assert np.max(np.abs(ref[0][0, 0, 0] - exact_mean)) > 1e-3          # the binary16 rounding is visible
+
+
+def test_fp16_accumulation_unsupported_with_16bit_pv():
+    sp = synth.Spec("t", Hq=2, Hkv=2, D=64, B=1, S=128, seed=5)
+    q, k, v = (_dev(t) for t in synth.make(sp))
+    with pytest.raises(ValueError):
+        sage.sageattn(q, k, v, pv_dtype="fp16", pv_accum_dtype="fp32+fp16")
+
+
+# ----------------------------------------------------------------------------- device timeout path
+@pytest.mark.parametrize("acc", ["fp32", "fp32+fp32"])
+def test_device_timeout_is_reported_and_the_context_recovers(acc):
+    """CTA 0 withholds one K tile (host-selected debug switch): the MMA's
+    bounded wait for it runs out after about 2 s, the CTA tears down through
+    the abort path (copies in flight drained, MMAs committed, tensor memory
+    freed), and the error word reports the timeout.  No GPU fault is
+    involved.  The next normal call, on the same workspace after the error
+    word was read and on a fresh one, must match the oracle."""
+    sp = synth.Spec("t", Hq=2, Hkv=2, D=128, B=1, S=1024, k_bias_std=3.0, seed=140)
+    q, k, v = synth.make(sp)
+    qd, kd, vd = _dev(q), _dev(k), _dev(v)
+    ws = torch.zeros(sage.sage_workspace_bytes(1, 2, 2, 1024, 128, 0, 0), dtype=torch.uint8, device="cuda")
+    sage.debug_set_max_ctas(1)
+    sage.debug_withhold_k_tile(3)
+    try:
+        sage.sageattn(qd, kd, vd, "HND", False, pv_accum_dtype=acc, workspace=ws)
+        st, bits = sage.get_device_error(ws)
+    finally:
+        sage.debug_withhold_k_tile(-1)
+        sage.debug_set_max_ctas(0)
+    assert st == sage.ERR_TIMEOUT, (st, hex(bits))
+    # the first of the attention kernel's waits to run out: the MMA issuer's
+    # (for the K tile) or the loader's (for the ring slot that tile holds)
+    assert bits & 0xF and not bits & ~0xF, hex(bits)
+    assert sage.get_device_error(ws) == (0, 0)           # reading cleared it
+    ref = oracle.attention(q, k, v, with_allowance=True)
+    for w in (ws, torch.zeros_like(ws)):
+        out = sage.sageattn(qd, kd, vd, "HND", False, pv_accum_dtype=acc, workspace=w)
+        torch.cuda.synchronize()
+        assert sage.get_device_error(w) == (0, 0)
+        _assert_close(out, ref, "fp16", "after a timeout")
