@@ -138,7 +138,8 @@ class Workspace:
         key = torch.device(device).index or 0
         buf = cls._cache.get(key)
         if buf is None or buf.numel() < nbytes:
-            buf = torch.empty(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
+            # zeroed: the device error word at its start must begin at 0
+            buf = torch.zeros(max(nbytes, 1 << 20), dtype=torch.uint8, device=device)
             cls._cache[key] = buf
         return buf
 
