@@ -270,6 +270,13 @@ sage_status_t sage_attn_fwd_noalloc(const void* q, const void* k, const void* v,
  * or SAGE_ERR_CUDA.  *bits (optional) receives the raw error word. */
 sage_status_t sage_get_device_error(void* ws, void* stream, uint32_t* bits);
 
+/* The CUDA runtime error (a cudaError_t value) behind the calling thread's
+ * most recent SAGE_ERR_CUDA, and its name (e.g. "cudaErrorInvalidValue");
+ * 0 / "cudaSuccess" before any.  Not reset by later successful calls.  The
+ * name is a static string owned by the CUDA runtime. */
+int sage_last_cuda_error(void);
+const char* sage_last_cuda_error_name(void);
+
 /* Debug: cap the attention kernel's persistent grid at max_ctas CTAs (0: one
  * CTA per SM, the default).  Process-wide; applies to the attention launches
  * that follow.  Results do not depend on it: the tests use it to make a few

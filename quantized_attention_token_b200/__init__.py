@@ -73,6 +73,8 @@ def lib():
         "sage_get_device_error": (I, [P, P, ctypes.POINTER(ctypes.c_uint32)]),
         "sage_debug_qk_tile": (I, [P, I, I, I, I, I, I, I, I, I, I, I, P, P]),
         "sage_status_string": (ctypes.c_char_p, [I]),
+        "sage_last_cuda_error": (I, []),
+        "sage_last_cuda_error_name": (ctypes.c_char_p, []),
         "sage_debug_set_max_ctas": (I, [I]),
         "sage_debug_withhold_k_tile": (I, [I]),
     }
@@ -88,6 +90,8 @@ def _check(fn: str, status: int):
         msg = lib().sage_status_string(status).decode()
         if status in (ERR_INVALID_ARG, ERR_UNSUPPORTED, ERR_WORKSPACE):
             raise ValueError(f"{fn}: {msg} (status {status})")
+        if status == ERR_CUDA:
+            msg += f" ({lib().sage_last_cuda_error_name().decode()})"
         raise SageError(fn, status, msg)
 
 

@@ -14,6 +14,16 @@
 #define SAGE_EXPORT extern "C" __attribute__((visibility("default")))
 
 namespace sage {
+
+// The CUDA error behind the calling thread's last SAGE_ERR_CUDA.
+thread_local int g_last_cuda_error = 0;
+
+sage_status_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return SAGE_OK;
+  g_last_cuda_error = (int)e;
+  return SAGE_ERR_CUDA;
+}
+
 namespace {
 
 // Debug settings (sage_debug_set_max_ctas, sage_debug_withhold_k_tile):
@@ -25,13 +35,12 @@ std::atomic<int> g_withhold_k{-1};
 sage_status_t check_device() {
   static int cache[128] = {0};   // 0 unknown, 1 sm_100, -1 other
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (sage_status_t st = cuda_status(cudaGetDevice(&dev))) return st;
   if (dev < 0 || dev >= 128) return SAGE_ERR_UNSUPPORTED;
   if (cache[dev] == 0) {
     int maj = 0, mnr = 0;
-    if (cudaDeviceGetAttribute(&maj, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&mnr, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess)
-      return SAGE_ERR_CUDA;
+    if (sage_status_t st = cuda_status(cudaDeviceGetAttribute(&maj, cudaDevAttrComputeCapabilityMajor, dev))) return st;
+    if (sage_status_t st = cuda_status(cudaDeviceGetAttribute(&mnr, cudaDevAttrComputeCapabilityMinor, dev))) return st;
     cache[dev] = (maj == 10 && mnr == 0) ? 1 : -1;
   }
   return cache[dev] == 1 ? SAGE_OK : SAGE_ERR_UNSUPPORTED;
@@ -96,7 +105,6 @@ Strides dense_strides(sage_layout_t layout, int H, int S, int D) {
   return Strides{(long long)S * H * D, (long long)D, (long long)H * D};
 }
 
-sage_status_t cuda_status(cudaError_t e) { return e == cudaSuccess ? SAGE_OK : SAGE_ERR_CUDA; }
 
 sage_status_t check_common(sage_dtype_t dtype, int D, sage_gran_t gran, sage_pv_t pv, sage_acc_t acc) {
   if (dtype != SAGE_F16 && dtype != SAGE_BF16) return SAGE_ERR_INVALID_ARG;
@@ -121,16 +129,18 @@ size_t stats_zero_bytes(const sage_ws_layout_t& L, int nseq, int Hkv, int D) {
 sage_status_t run_prepass(const void* q, const void* k, const void* v, int bf16, Strides sq, Strides sk,
                           Strides sv, const Seqs& seqs, int nseq, int Hq, int Hkv, int D, int gran, int pv,
                           int smooth_k, int smooth_q, void* ws, const sage_ws_layout_t& L, cudaStream_t s) {
-  if (cudaMemsetAsync(at<char>(ws, L.k_stat), 0, stats_zero_bytes(L, nseq, Hkv, D), s) != cudaSuccess)
-    return SAGE_ERR_CUDA;
+  if (sage_status_t st = cuda_status(cudaMemsetAsync(at<char>(ws, L.k_stat), 0, stats_zero_bytes(L, nseq, Hkv, D), s)))
+    return st;
   if (seqs.cu_k) {
     // A varlen sequence without keys gets no K / V tile, so nothing else
     // writes its K means and V scales / means: zero them, so that its queries
     // (no visible key: output 0) read zeros rather than stale workspace bytes.
     const size_t nd = (size_t)nseq * Hkv * D;
-    if (k && cudaMemsetAsync(at<char>(ws, L.k_mean), 0, nd * 4, s) != cudaSuccess) return SAGE_ERR_CUDA;
-    if (v && cudaMemsetAsync(at<char>(ws, L.v_scale), 0, L.v_mean + nd * 4 - L.v_scale, s) != cudaSuccess)
-      return SAGE_ERR_CUDA;
+    if (k)
+      if (sage_status_t st = cuda_status(cudaMemsetAsync(at<char>(ws, L.k_mean), 0, nd * 4, s))) return st;
+    if (v)
+      if (sage_status_t st = cuda_status(cudaMemsetAsync(at<char>(ws, L.v_scale), 0, L.v_mean + nd * 4 - L.v_scale, s)))
+        return st;
   }
   PrepassJob j;
   j.q = static_cast<const uint16_t*>(q);
@@ -169,10 +179,11 @@ sage_status_t run_prepass(const void* q, const void* k, const void* v, int bf16,
   j.v_codes = at<uint8_t>(ws, L.v_codes);
   j.q_mean = smooth_q ? at<float>(ws, L.q_mean) : nullptr;
   j.q_bias = smooth_q ? at<float>(ws, L.q_bias) : nullptr;
-  if (seqs.cu_k &&
-      prepass_varlen_offsets(seqs.cu_q, seqs.cu_k, nseq, seqs.max_seqlen, L.tiles_q, L.tiles_k,
-                             const_cast<int*>(seqs.toff_q), const_cast<int*>(seqs.toff_k), j.err, s) != cudaSuccess)
-    return SAGE_ERR_CUDA;
+  if (seqs.cu_k)
+    if (sage_status_t st = cuda_status(prepass_varlen_offsets(seqs.cu_q, seqs.cu_k, nseq, seqs.max_seqlen, L.tiles_q,
+                                                              L.tiles_k, const_cast<int*>(seqs.toff_q),
+                                                              const_cast<int*>(seqs.toff_k), j.err, s)))
+      return st;
   return cuda_status(prepass_run(j, D, s));
 }
 
@@ -389,9 +400,10 @@ SAGE_EXPORT sage_status_t sage_get_device_error(void* ws, void* stream, uint32_t
   if (!ws || !aligned(ws, 256)) return SAGE_ERR_INVALID_ARG;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t w = 0;
-  if (cudaStreamSynchronize(s) != cudaSuccess) return SAGE_ERR_CUDA;
-  if (cudaMemcpy(&w, ws, sizeof(w), cudaMemcpyDeviceToHost) != cudaSuccess) return SAGE_ERR_CUDA;
-  if (w && cudaMemset(ws, 0, sizeof(w)) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (sage_status_t st = cuda_status(cudaStreamSynchronize(s))) return st;
+  if (sage_status_t st = cuda_status(cudaMemcpy(&w, ws, sizeof(w), cudaMemcpyDeviceToHost))) return st;
+  if (w)
+    if (sage_status_t st = cuda_status(cudaMemset(ws, 0, sizeof(w)))) return st;
   if (bits) *bits = w;
   if (w & (kErrTimeoutLoad | kErrTimeoutMma | kErrTimeoutSoftmax | kErrTimeoutCorr)) return SAGE_ERR_TIMEOUT;
   if (w) return SAGE_ERR_INVALID_ARG;
@@ -427,6 +439,12 @@ SAGE_EXPORT sage_status_t sage_debug_withhold_k_tile(int ring_index) {
   if (ring_index < -1) return SAGE_ERR_INVALID_ARG;
   g_withhold_k.store(ring_index);
   return SAGE_OK;
+}
+
+SAGE_EXPORT int sage_last_cuda_error(void) { return sage::g_last_cuda_error; }
+
+SAGE_EXPORT const char* sage_last_cuda_error_name(void) {
+  return cudaGetErrorName(static_cast<cudaError_t>(sage::g_last_cuda_error));
 }
 
 SAGE_EXPORT const char* sage_status_string(sage_status_t s) {

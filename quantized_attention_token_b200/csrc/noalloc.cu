@@ -33,12 +33,13 @@ void* g_scratch_ptr[kMaxDevices] = {};
 // first call for that device (with the device current).
 sage_status_t scratch_for_current_device(void** ptr) {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (sage_status_t st = sage::cuda_status(cudaGetDevice(&dev))) return st;
   if (dev < 0 || dev >= kMaxDevices) return SAGE_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_mu);
   if (!g_scratch_ptr[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return SAGE_ERR_CUDA;
+    if (sage_status_t st = sage::cuda_status(cudaGetSymbolAddress(&p, g_noalloc_scratch))) return st;
+    if (!p) return SAGE_ERR_CUDA;
     g_scratch_ptr[dev] = p;
   }
   *ptr = g_scratch_ptr[dev];
@@ -60,7 +61,7 @@ SAGE_EXPORT sage_status_t sage_attn_fwd_noalloc(const void* q, const void* k, co
   if (st != SAGE_OK) return st;
   // The array keeps the previous call's contents.  The pre-pass zeroes its own
   // accumulators; the device error word must start at zero too.
-  if (cudaMemsetAsync(ws, 0, 256, static_cast<cudaStream_t>(stream)) != cudaSuccess) return SAGE_ERR_CUDA;
+  if (sage_status_t st = sage::cuda_status(cudaMemsetAsync(ws, 0, 256, static_cast<cudaStream_t>(stream)))) return st;
   return sage_attn_fwd(q, k, v, out, dtype, B, Hq, Hkv, S, D, layout, is_causal, sm_scale, gran, pv, pv_accum,
                        smooth_k, 0, ws, SAGE_NOALLOC_SCRATCH_BYTES, stream);
 }

@@ -2,6 +2,7 @@
 // libsage CUDA translation units (pre-pass, attention, C ABI).
 #pragma once
 
+#include "sage.h"
 #include "sage_common.cuh"
 
 namespace sage {
@@ -68,6 +69,10 @@ enum { kAccOne = 0, kAccTwo = 1, kAccTwoF16 = 2 };
 
 // prepass.cu
 cudaError_t prepass_run(const PrepassJob& j, int D, cudaStream_t s);
+
+// SAGE_OK for cudaSuccess; otherwise records e as the calling thread's last
+// CUDA error (sage_last_cuda_error) and returns SAGE_ERR_CUDA.  (api.cu)
+sage_status_t cuda_status(cudaError_t e);
 cudaError_t prepass_varlen_offsets(const int* cu_q, const int* cu_k, int n, int max_seqlen, int cap_q, int cap_k,
                                    int* toff_q, int* toff_k, uint32_t* err, cudaStream_t s);
 

@@ -90,6 +90,9 @@ def test_valid_arguments_without_a_gpu_report_cuda_error(L):
     st = L.sage_attn_fwd(0x10000, 0x20000, 0x30000, 0x40000, 0, 1, 4, 2, 256, 128, 0, 0, 0.0, 0, 0, 1, 1, 0,
                          0x100000, 1 << 30, None)
     assert st in (sage.ERR_CUDA, sage.ERR_UNSUPPORTED)
+    if st == sage.ERR_CUDA:        # the runtime's reason is kept for the caller
+        assert L.sage_last_cuda_error() != 0
+        assert L.sage_last_cuda_error_name().decode().startswith("cudaError")
 
 
 def test_varlen_rejects_bad_arguments(L):
