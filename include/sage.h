@@ -294,6 +294,20 @@ sage_status_t sage_debug_set_max_ctas(int max_ctas);
  * switches it off; values below -1 give SAGE_ERR_INVALID_ARG. */
 sage_status_t sage_debug_withhold_k_tile(int ring_index);
 
+/* Debug: on = 1 sends K and V of the pre-passes that follow through the
+ * one-pass cluster path wherever a head's keys fit the shared memory of one
+ * thread-block cluster (up to 16 CTAs x 128 KB): K and V are read from HBM
+ * once instead of twice.  0 (the default) keeps the two-launch path
+ * (statistics launch, then quantize launch), which measured faster on B200
+ * for every workload tried.  Both paths write identical bytes.  Process-wide.
+ * Other values give SAGE_ERR_INVALID_ARG. */
+sage_status_t sage_debug_set_prepass_one_pass(int on);
+
+/* Debug: the K / V path the calling thread's last pre-pass took: 1 the
+ * one-pass cluster path, 2 the two-launch path, 0 none (no K or V, or no
+ * pre-pass yet). */
+int sage_debug_last_prepass_path(void);
+
 /* Debug: the int32 scores of one 128x128 tile, S = Q_codes(q tile) *
  * K_codes(k tile)^T, computed by the same tensor-core MMA path as the
  * attention kernel from a workspace filled by sage_quant_qk.  s_out: device

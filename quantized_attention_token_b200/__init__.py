@@ -19,7 +19,8 @@ from typing import Optional
 
 __all__ = [
     "sageattn", "sageattn_varlen", "quant_qk", "quant_qkv", "quant_v", "attn_quantized", "workspace_layout",
-    "get_device_error", "debug_qk_tile", "debug_set_max_ctas", "debug_withhold_k_tile", "Workspace", "SageError",
+    "get_device_error", "debug_qk_tile", "debug_set_max_ctas", "debug_withhold_k_tile",
+    "debug_set_prepass_one_pass", "debug_last_prepass_path", "Workspace", "SageError",
     "lib", "LIB_PATH",
 ]
 
@@ -77,6 +78,8 @@ def lib():
         "sage_last_cuda_error_name": (ctypes.c_char_p, []),
         "sage_debug_set_max_ctas": (I, [I]),
         "sage_debug_withhold_k_tile": (I, [I]),
+        "sage_debug_set_prepass_one_pass": (I, [I]),
+        "sage_debug_last_prepass_path": (I, []),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -309,3 +312,19 @@ def debug_withhold_k_tile(ring_index: int):
     """Make CTA 0 of the following attention launches skip one K tile copy, so
     that its bounded wait runs out (-1: off).  Tests the timeout path."""
     _check("sage_debug_withhold_k_tile", lib().sage_debug_withhold_k_tile(int(ring_index)))
+
+
+PREPASS_PATH = {0: None, 1: "one_pass", 2: "two_launch"}
+
+
+def debug_set_prepass_one_pass(on: bool):
+    """Send K / V of the following pre-passes through the one-pass cluster
+    path wherever a head fits it (default: the two-launch path).
+    Process-wide; both paths write identical bytes."""
+    _check("sage_debug_set_prepass_one_pass", lib().sage_debug_set_prepass_one_pass(int(bool(on))))
+
+
+def debug_last_prepass_path():
+    """"one_pass", "two_launch" or None: the K / V path of this thread's last
+    pre-pass."""
+    return PREPASS_PATH[lib().sage_debug_last_prepass_path()]

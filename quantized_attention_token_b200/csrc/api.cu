@@ -26,10 +26,14 @@ sage_status_t cuda_status(cudaError_t e) {
 
 namespace {
 
-// Debug settings (sage_debug_set_max_ctas, sage_debug_withhold_k_tile):
-// process-wide, read at each attention launch.
+// Debug settings (sage_debug_set_max_ctas, sage_debug_withhold_k_tile,
+// sage_debug_set_prepass_one_pass): process-wide, read at each launch.
 std::atomic<int> g_max_ctas{0};
 std::atomic<int> g_withhold_k{-1};
+std::atomic<int> g_prepass_one_pass{0};
+// The K / V path of the calling thread's last pre-pass (kPrepassOnePass /
+// kPrepassTwoLaunch, 0 none).
+thread_local int g_last_prepass_path = 0;
 
 // ---------------------------------------------------------------- device check
 sage_status_t check_device() {
@@ -184,7 +188,8 @@ sage_status_t run_prepass(const void* q, const void* k, const void* v, int bf16,
                                                               L.tiles_k, const_cast<int*>(seqs.toff_q),
                                                               const_cast<int*>(seqs.toff_k), j.err, s)))
       return st;
-  return cuda_status(prepass_run(j, D, s));
+  j.one_pass = g_prepass_one_pass.load();
+  return cuda_status(prepass_run(j, D, s, &g_last_prepass_path));
 }
 
 sage_status_t run_attn(void* out, int bf16, Strides so, const Seqs& seqs, int nseq, int Hq, int Hkv, int D,
@@ -440,6 +445,14 @@ SAGE_EXPORT sage_status_t sage_debug_withhold_k_tile(int ring_index) {
   g_withhold_k.store(ring_index);
   return SAGE_OK;
 }
+
+SAGE_EXPORT sage_status_t sage_debug_set_prepass_one_pass(int on) {
+  if (on != 0 && on != 1) return SAGE_ERR_INVALID_ARG;
+  g_prepass_one_pass.store(on);
+  return SAGE_OK;
+}
+
+SAGE_EXPORT int sage_debug_last_prepass_path(void) { return g_last_prepass_path; }
 
 SAGE_EXPORT int sage_last_cuda_error(void) { return sage::g_last_cuda_error; }
 

@@ -27,6 +27,11 @@
 // Each thread loads its whole share of a tile (eight or four 16-byte loads)
 // before any arithmetic, and several CTAs share an SM, so one CTA's barrier
 // waits overlap the others' loads.
+//
+// A one-pass alternative for K and V (debug-selected, see
+// prepass_kv_cluster_kernel) reads them from HBM once: one thread-block
+// cluster per (tensor, sequence, KV head) holds the head in shared memory.
+// It writes the same bytes; on B200 it measured slower than the two launches.
 #include "sage_launch.cuh"
 
 namespace sage {
@@ -145,9 +150,13 @@ __device__ __forceinline__ uint16_t unkey16(uint32_t k) {
 }
 template <int D>
 struct VSmem {
-  uint32_t tile[kTile * D / 2];   // the 16-bit tile, row-major, two values per word
   float inv[D];                   // 448 / channel amax (FP8 mode)
   float mu[D];                    // channel mean (smooth V), else 0
+};
+template <int D>
+struct VTileSmem {
+  VSmem<D> v;
+  uint32_t tile[kTile * D / 2];   // the 16-bit tile, row-major, two values per word
 };
 
 // Sum or max of a per-lane value over the lanes of a warp that own the same
@@ -162,16 +171,14 @@ __device__ __forceinline__ T reduce_same_chunk(T x, Op op) {
 // ---------------------------------------------------------------- Q / K tile
 // INT8 codes and group scales of one Q tile (launch A) or K tile (launch B);
 // for K also the channel mean (written once per sequence and head).
+// v: the thread's NR chunks of the tile (zeros past the sequence).
 template <int D, bool IS_Q, bool BF16>
-__device__ void quant_tile(const PrepassJob& j, int h, int t, const TileLoc& L, QuantSmem<D>& sm) {
+__device__ void quant_tile(const PrepassJob& j, int h, int t, const TileLoc& L, QuantSmem<D>& sm,
+                           const uint4 (&v)[Map<D>::NR]) {
   using M = Map<D>;
   const int tid = threadIdx.x, cc = tid % M::TPR, rg = tid / M::TPR, warp = tid >> 5, lane = tid & 31;
   const int H = IS_Q ? j.Hq : j.Hkv;
   const int tiles = IS_Q ? j.tiles_q : j.tiles_k;
-  const Strides& st = IS_Q ? j.sq : j.sk;
-  const uint16_t* head = (IS_Q ? j.q : j.k) + (long long)L.b * st.sb + (long long)h * st.sh;
-  uint4 v[M::NR];
-  load_tile<D, true>(head, st.ss, L, v);
 
   const bool smooth = IS_Q ? j.smooth_q : j.smooth_k;
   if (smooth) {
@@ -286,12 +293,10 @@ __device__ void quant_tile(const PrepassJob& j, int h, int t, const TileLoc& L, 
 // is a multiple of 2^-24 below 2^23 in magnitude, so fp64 holds it exactly and
 // it is added as a 2^-24 fixed-point int64 (bf16: added as fp64).
 template <int D, bool BF16>
-__device__ void kstat_tile(const PrepassJob& j, int h, const TileLoc& L, StatSmem<D>& sm) {
+__device__ void kstat_tile(const PrepassJob& j, int h, const TileLoc& L, StatSmem<D>& sm,
+                           const uint4 (&v)[Map<D>::NR]) {
   using M = Map<D>;
   const int tid = threadIdx.x, cc = tid % M::TPR, warp = tid >> 5, lane = tid & 31;
-  const uint16_t* head = j.k + (long long)L.b * j.sk.sb + (long long)h * j.sk.sh;
-  uint4 v[M::NR];
-  load_tile<D, false>(head, j.sk.ss, L, v);
 #pragma unroll
   for (int u = 0; u < 8; ++u) {
     double a = 0.0;
@@ -317,12 +322,10 @@ __device__ void kstat_tile(const PrepassJob& j, int h, const TileLoc& L, StatSme
 // mean and |max| of V - mean: float32 subtraction of a fixed mean is monotone,
 // so that |max| comes from the two extremes.
 template <int D, bool BF16, bool SMOOTH>
-__device__ void vstat_tile(const PrepassJob& j, int h, const TileLoc& L, StatSmem<D>& sm) {
+__device__ void vstat_tile(const PrepassJob& j, int h, const TileLoc& L, StatSmem<D>& sm,
+                           const uint4 (&v)[Map<D>::NR]) {
   using M = Map<D>;
   const int tid = threadIdx.x, cc = tid % M::TPR, rg = tid / M::TPR, warp = tid >> 5, lane = tid & 31;
-  const uint16_t* head = j.v + (long long)L.b * j.sv.sb + (long long)h * j.sv.sh;
-  uint4 v[M::NR];
-  load_tile<D, false>(head, j.sv.ss, L, v);
   const size_t o = ((size_t)L.b * j.Hkv + h) * D;
   if constexpr (!SMOOTH) {
 #pragma unroll
@@ -384,15 +387,13 @@ __device__ void vstat_tile(const PrepassJob& j, int h, const TileLoc& L, StatSme
 
 // ---------------------------------------------------------------- V tile
 // V written transposed: FP8 rows of 128 keys, or 16-bit rows split in two
-// 64-key halves.  The tile is staged in shared memory; each output unit
+// 64-key halves.  `tile` is the 16-bit tile in shared memory, row-major, two
+// values per 32-bit word, rows past the sequence zero; the caller makes it
+// visible to the whole CTA before the first barrier below.  Each output unit
 // gathers two adjacent channels (one 32-bit word per key).
 template <int D, bool BF16, bool SMOOTH>
-__device__ void v_tile(const PrepassJob& j, int h, int t, const TileLoc& L, VSmem<D>& sm) {
-  using M = Map<D>;
-  const int tid = threadIdx.x, cc = tid % M::TPR, rg = tid / M::TPR;
-  const uint16_t* head = j.v + (long long)L.b * j.sv.sb + (long long)h * j.sv.sh;
-  uint4 v[M::NR];
-  load_tile<D, true>(head, j.sv.ss, L, v);
+__device__ void v_tile(const PrepassJob& j, int h, int t, const TileLoc& L, VSmem<D>& sm, const uint32_t* tile) {
+  const int tid = threadIdx.x;
   if (j.pv8 && tid < D) {
     const size_t o = ((size_t)L.b * j.Hkv + h) * D + tid;
     float am, mu = 0.f;
@@ -412,9 +413,6 @@ __device__ void v_tile(const PrepassJob& j, int h, int t, const TileLoc& L, VSme
     sm.inv[tid] = am > 0.f ? __fdiv_rn(kFp8Max, am) : 0.f;
     if (L.tile == 0) j.v_scale[o] = __fdiv_rn(am, kFp8Max);
   }
-#pragma unroll
-  for (int i = 0; i < M::NR; ++i)
-    *reinterpret_cast<uint4*>(&sm.tile[(rg * M::NR + i) * (D / 2) + cc * 4]) = v[i];
   __syncthreads();
   uint8_t* tb = j.v_codes + ((size_t)h * j.tiles_k + t) * (size_t)(D * kTile * (j.pv8 ? 1 : 2));
   if (j.pv8) {
@@ -430,7 +428,7 @@ __device__ void v_tile(const PrepassJob& j, int h, int t, const TileLoc& L, VSme
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int key = 16 * k + 4 * q4 + e;
-          const uint32_t x = sm.tile[key * (D / 2) + p];
+          const uint32_t x = tile[key * (D / 2) + p];
           const float x0 = h16_to_f32((uint16_t)(x & 0xFFFF), BF16), x1 = h16_to_f32((uint16_t)(x >> 16), BF16);
           if (SMOOTH) {        // (V - mean) * 448 / |max|; keys past the sequence stay 0
             const bool in = key < L.nvalid;
@@ -453,7 +451,7 @@ __device__ void v_tile(const PrepassJob& j, int h, int t, const TileLoc& L, VSme
       const int p = w % (D / 2), o = w / (D / 2), hf = o >> 3, kk = o & 7;
       uint32_t x[8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] = sm.tile[(8 * o + e) * (D / 2) + p];
+      for (int e = 0; e < 8; ++e) x[e] = tile[(8 * o + e) * (D / 2) + p];
       uint32_t a[4], b[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
@@ -481,13 +479,23 @@ __global__ void __launch_bounds__(kPrepassThreads, 3) prepass_a_kernel(const Pre
   const int nq = j.do_q ? j.Hq : 0;
   const int nks = (j.do_k && j.smooth_k) ? j.Hkv : 0;
   TileLoc L;
+  uint4 v[Map<D>::NR];
   if (y < nq) {
-    if (t < j.tiles_q && locate(j, true, t, L)) quant_tile<D, true, BF16>(j, y, t, L, sm.q);
+    if (t < j.tiles_q && locate(j, true, t, L)) {
+      load_tile<D, true>(j.q + (long long)L.b * j.sq.sb + (long long)y * j.sq.sh, j.sq.ss, L, v);
+      quant_tile<D, true, BF16>(j, y, t, L, sm.q, v);
+    }
   } else if ((y -= nq) < nks) {
-    if (t < j.tiles_k && locate(j, false, t, L)) kstat_tile<D, BF16>(j, y, L, sm.s);
+    if (t < j.tiles_k && locate(j, false, t, L)) {
+      load_tile<D, false>(j.k + (long long)L.b * j.sk.sb + (long long)y * j.sk.sh, j.sk.ss, L, v);
+      kstat_tile<D, BF16>(j, y, L, sm.s, v);
+    }
   } else {
     y -= nks;
-    if (t < j.tiles_k && locate(j, false, t, L)) vstat_tile<D, BF16, SV>(j, y, L, sm.s);
+    if (t < j.tiles_k && locate(j, false, t, L)) {
+      load_tile<D, false>(j.v + (long long)L.b * j.sv.sb + (long long)y * j.sv.sh, j.sv.ss, L, v);
+      vstat_tile<D, BF16, SV>(j, y, L, sm.s, v);
+    }
   }
 }
 
@@ -497,15 +505,191 @@ template <int D, bool BF16, bool SV>
 __global__ void __launch_bounds__(kPrepassThreads, 3) prepass_b_kernel(const PrepassJob j) {
   __shared__ union {
     QuantSmem<D> q;
-    VSmem<D> v;
+    VTileSmem<D> vt;
   } sm;
   const int t = gridDim.x - 1 - blockIdx.x;
   const int y = gridDim.y - 1 - blockIdx.y;
   const int nk = j.do_k ? j.Hkv : 0;
   TileLoc L;
   if (!locate(j, false, t, L)) return;
-  if (y < nk) quant_tile<D, false, BF16>(j, y, t, L, sm.q);
-  else v_tile<D, BF16, SV>(j, y - nk, t, L, sm.v);
+  uint4 v[Map<D>::NR];
+  if (y < nk) {
+    load_tile<D, true>(j.k + (long long)L.b * j.sk.sb + (long long)y * j.sk.sh, j.sk.ss, L, v);
+    quant_tile<D, false, BF16>(j, y, t, L, sm.q, v);
+  } else {
+    const int h = y - nk;
+    load_tile<D, true>(j.v + (long long)L.b * j.sv.sb + (long long)h * j.sv.sh, j.sv.ss, L, v);
+    using M = Map<D>;
+    const int cc = threadIdx.x % M::TPR, rg = threadIdx.x / M::TPR;
+#pragma unroll
+    for (int i = 0; i < M::NR; ++i)
+      *reinterpret_cast<uint4*>(&sm.vt.tile[(rg * M::NR + i) * (D / 2) + cc * 4]) = v[i];
+    v_tile<D, BF16, SV>(j, h, t, L, sm.vt.v, sm.vt.tile);
+  }
+}
+
+// ---------------------------------------------------------------- K / V in one pass
+// When every sequence's K (or V) of one head fits in the shared memory of a
+// thread-block cluster, one cluster per (tensor, sequence, KV head) reads it
+// from HBM once: CTA `rank` copies tiles rank*TMAX .. rank*TMAX + TMAX-1 into
+// its own shared memory, adds their statistics into the per-(sequence, head)
+// accumulators (as launch A does), waits at the cluster barrier for the other
+// CTAs' contributions, and then quantizes its tiles from shared memory (as
+// launch B does).  The statistics meet in global memory: the accumulators are
+// exact integer / max reductions, so their order does not matter, and the
+// cluster barrier's release / acquire makes every CTA's atomics visible to
+// the others.  No CTA reads another's shared memory.
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ uint32_t cluster_index() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// 16-byte asynchronous global -> shared copy (plain form: whole source, no
+// cache hint) and its group bookkeeping.
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+// Wait until at most n (0..7) of this thread's groups are pending.
+__device__ __forceinline__ void cp_async_wait_upto(int n) {
+  switch (n) {
+    case 0: cp_async_wait<0>(); break;
+    case 1: cp_async_wait<1>(); break;
+    case 2: cp_async_wait<2>(); break;
+    case 3: cp_async_wait<3>(); break;
+    case 4: cp_async_wait<4>(); break;
+    case 5: cp_async_wait<5>(); break;
+    case 6: cp_async_wait<6>(); break;
+    default: cp_async_wait<7>(); break;
+  }
+}
+
+// Start copying the thread's NR chunks of a tile into shared memory (rows of
+// D 16-bit values, the layout load_staged and v_tile read); chunks past the
+// sequence are zeroed with plain stores.
+template <int D>
+__device__ __forceinline__ void stage_tile(const uint16_t* head, long long ss, const TileLoc& L, uint32_t stage,
+                                           uint8_t* stage_ptr) {
+  using M = Map<D>;
+  const int cc = threadIdx.x % M::TPR, rg = threadIdx.x / M::TPR;
+  const uint16_t* p = head + (long long)(L.start + L.tile * kTile + rg * M::NR) * ss + cc * 8;
+#pragma unroll
+  for (int i = 0; i < M::NR; ++i) {
+    const uint32_t off = (uint32_t)((rg * M::NR + i) * (D * 2) + cc * 16);
+    if (rg * M::NR + i < L.nvalid) cp_async16(stage + off, p + i * ss);
+    else *reinterpret_cast<uint4*>(stage_ptr + off) = make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+// The thread's NR chunks of a tile staged in shared memory.
+template <int D>
+__device__ __forceinline__ void load_staged(const uint8_t* stage, uint4 (&v)[Map<D>::NR]) {
+  using M = Map<D>;
+  const int cc = threadIdx.x % M::TPR, rg = threadIdx.x / M::TPR;
+#pragma unroll
+  for (int i = 0; i < M::NR; ++i)
+    v[i] = *reinterpret_cast<const uint4*>(stage + (size_t)(rg * M::NR + i) * (D * 2) + cc * 16);
+}
+
+// Tile ti of sequence b's keys: its token range and workspace slot t.  False
+// when it holds no tokens, when the sequence's length is invalid (flagged by
+// the offsets kernel) or when its slot lies past the workspace's tiles.
+__device__ __forceinline__ bool locate_kv(const PrepassJob& j, int b, int ti, int& t, TileLoc& L) {
+  const Seqs& s = j.seqs;
+  L.b = b;
+  L.tile = ti;
+  if (!s.cu_k) {
+    L.start = 0;
+    L.len = s.S;
+    t = b * s.tps + ti;
+  } else {
+    L.start = s.cu_k[b];
+    L.len = s.cu_k[b + 1] - L.start;
+    if (L.len < 0 || L.len > s.max_seqlen) return false;
+    t = s.toff_k[b] + ti;
+  }
+  L.nvalid = min(kTile, L.len - ti * kTile);
+  return L.nvalid > 0 && t < j.tiles_k;
+}
+
+template <int D>
+__host__ __device__ constexpr int kv_tile_bytes() { return kTile * D * 2; }
+
+// Cluster c (clusterid.x) is job c: jobs [0, n_k_jobs) are the K heads
+// (sequence-major), the rest the V heads.  Dynamic shared memory: TMAX tiles.
+template <int D, bool BF16, bool SV, int TMAX>
+__global__ void __launch_bounds__(kPrepassThreads, 2) prepass_kv_cluster_kernel(const PrepassJob j, int n_k_jobs) {
+  extern __shared__ __align__(128) uint8_t stage_mem[];
+  __shared__ union {
+    QuantSmem<D> q;
+    StatSmem<D> s;
+    VSmem<D> v;
+  } sm;
+  constexpr int SB = kv_tile_bytes<D>();
+  const int rank = (int)cluster_rank(), job = (int)cluster_index();
+  const bool is_k = job < n_k_jobs;
+  const int jb = is_k ? job : job - n_k_jobs;
+  const int b = jb / j.Hkv, h = jb - b * j.Hkv;
+  const Strides& st = is_k ? j.sk : j.sv;
+  const uint16_t* head = (is_k ? j.k : j.v) + (long long)b * st.sb + (long long)h * st.sh;
+  const uint32_t stage0 = (uint32_t)__cvta_generic_to_shared(stage_mem);
+  // 1. all of this CTA's copies in flight, one group per tile
+#pragma unroll
+  for (int i = 0; i < TMAX; ++i) {
+    TileLoc L;
+    int t;
+    if (locate_kv(j, b, rank * TMAX + i, t, L)) stage_tile<D>(head, st.ss, L, stage0 + i * SB, stage_mem + i * SB);
+    cp_async_commit();
+  }
+  // 2. statistics of each tile as its copy lands: smooth K needs the channel
+  //    sums, FP8 V the channel |max| (and, smooth V, sums and extremes)
+  const bool stats = is_k ? (j.smooth_k != 0) : (j.pv8 != 0);
+#pragma unroll
+  for (int i = 0; i < TMAX; ++i) {
+    cp_async_wait_upto(TMAX - 1 - i);
+    TileLoc L;
+    int t;
+    if (stats && locate_kv(j, b, rank * TMAX + i, t, L)) {
+      uint4 v[Map<D>::NR];
+      load_staged<D>(stage_mem + i * SB, v);
+      if (is_k) kstat_tile<D, BF16>(j, h, L, sm.s, v);
+      else vstat_tile<D, BF16, SV>(j, h, L, sm.s, v);
+      __syncthreads();             // sm.s is reused by the next tile
+    }
+  }
+  cp_async_wait<0>();
+  __syncthreads();                 // every staged tile visible to the whole CTA
+  // 3. every CTA of the cluster has added its contributions
+  cluster_sync_all();
+  // 4. quantize from shared memory
+#pragma unroll 1
+  for (int i = 0; i < TMAX; ++i) {
+    TileLoc L;
+    int t;
+    if (!locate_kv(j, b, rank * TMAX + i, t, L)) continue;
+    if (is_k) {
+      uint4 v[Map<D>::NR];
+      load_staged<D>(stage_mem + i * SB, v);
+      quant_tile<D, false, BF16>(j, h, t, L, sm.q, v);
+    } else {
+      v_tile<D, BF16, SV>(j, h, t, L, sm.v, reinterpret_cast<const uint32_t*>(stage_mem + i * SB));
+    }
+    __syncthreads();               // sm is reused by the next tile
+  }
 }
 
 // ---------------------------------------------------------------- smooth-Q bias
@@ -565,8 +749,95 @@ __global__ void varlen_offsets_kernel(const int* cu_q, const int* cu_k, int n, i
 }
 
 // ---------------------------------------------------------------- launchers
+// Largest cluster the one-pass K / V path uses (16 needs the non-portable
+// cluster-size opt-in) and the largest staged share of a CTA.
+constexpr int kKvMaxCluster = 16;
+template <int D>
+constexpr int kv_max_tiles_per_cta() { return D == 128 ? 4 : 8; }   // 128 KB of shared memory
+
+// The one-pass K / V launch with TMAX tiles per CTA and `cl` CTAs per
+// cluster.  `done` stays false (and nothing is launched) when the device
+// cannot place such a cluster.
+template <int D, bool BF16, bool SV, int TMAX>
+static cudaError_t launch_kv_cluster(const PrepassJob& j, int cl, cudaStream_t s, bool& done) {
+  done = false;
+  auto k = prepass_kv_cluster_kernel<D, BF16, SV, TMAX>;
+  const int dyn = TMAX * kv_tile_bytes<D>();
+  const int n_k = j.do_k ? j.nseq * j.Hkv : 0;
+  const long long jobs = (long long)n_k + (j.do_v ? (long long)j.nseq * j.Hkv : 0);
+  if (jobs == 0) {
+    done = true;
+    return cudaSuccess;
+  }
+  if (jobs * cl > 0x7fffffffLL) return cudaSuccess;
+  cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, dyn);
+  if (e != cudaSuccess) return e;
+  if (cl > 8 && (e = cudaFuncSetAttribute(k, cudaFuncAttributeNonPortableClusterSizeAllowed, 1)) != cudaSuccess)
+    return e;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3((unsigned)(jobs * cl), 1, 1);
+  cfg.blockDim = dim3(kPrepassThreads, 1, 1);
+  cfg.dynamicSmemBytes = dyn;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = cl;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  int fit = 0;
+  if (cudaOccupancyMaxActiveClusters(&fit, k, &cfg) != cudaSuccess || fit < 1) {
+    (void)cudaGetLastError();      // not placeable: the caller takes the two-launch path
+    return cudaSuccess;
+  }
+  e = cudaLaunchKernelEx(&cfg, k, j, n_k);
+  done = e == cudaSuccess;
+  return e;
+}
+
+// Tiles of the longest sequence's keys -> (TMAX, cluster size) of the
+// one-pass path, or false when a head does not fit a cluster.
+template <int D>
+static bool kv_cluster_shape(const PrepassJob& j, int& tmax, int& cl) {
+  const long long tiles = j.seqs.cu_k ? ((long long)j.seqs.max_seqlen + kTile - 1) / kTile : j.seqs.tps;
+  if (tiles <= 0) return false;
+  for (tmax = 2; tmax <= kv_max_tiles_per_cta<D>(); tmax *= 2)
+    if ((long long)kKvMaxCluster * tmax >= tiles) break;
+  if (tmax > kv_max_tiles_per_cta<D>()) return false;
+  const int need = (int)((tiles + tmax - 1) / tmax);
+  for (cl = 1; cl < need; cl *= 2) {}
+  return true;
+}
+
 template <int D, bool BF16, bool SV>
-static cudaError_t launch_prepass(const PrepassJob& j, cudaStream_t s) {
+static cudaError_t launch_kv_one_pass(const PrepassJob& j, cudaStream_t s, bool& done) {
+  done = false;
+  int tmax = 0, cl = 0;
+  if (!kv_cluster_shape<D>(j, tmax, cl)) return cudaSuccess;
+  if (tmax == 2) return launch_kv_cluster<D, BF16, SV, 2>(j, cl, s, done);
+  if (tmax == 4) return launch_kv_cluster<D, BF16, SV, 4>(j, cl, s, done);
+  if constexpr (kv_max_tiles_per_cta<D>() >= 8) return launch_kv_cluster<D, BF16, SV, 8>(j, cl, s, done);
+  return cudaSuccess;
+}
+
+template <int D, bool BF16, bool SV>
+static cudaError_t launch_prepass(const PrepassJob& j0, cudaStream_t s, int* path) {
+  // Launches A / B; with j0.one_pass K and V go through the cluster kernel
+  // where a head fits one (it reads them once, but each CTA loads, waits at
+  // the cluster barrier and then computes, and on B200 that measured slower
+  // than the two launches for every workload tried).
+  PrepassJob j = j0;
+  if (path) *path = 0;
+  if ((j0.do_k || j0.do_v) && j0.tiles_k > 0) {
+    bool done = false;
+    if (j0.one_pass) {
+      const cudaError_t e = launch_kv_one_pass<D, BF16, SV>(j0, s, done);
+      if (e != cudaSuccess) return e;
+    }
+    if (done) j.do_k = j.do_v = 0;
+    if (path) *path = done ? kPrepassOnePass : kPrepassTwoLaunch;
+  }
   const int nq = j.do_q ? j.Hq : 0;
   const int nks = (j.do_k && j.smooth_k) ? j.Hkv : 0;
   const int nvs = (j.do_v && j.pv8) ? j.Hkv : 0;
@@ -582,19 +853,20 @@ static cudaError_t launch_prepass(const PrepassJob& j, cudaStream_t s) {
     const cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
   }
-  if (j.q_bias && j.do_q && j.do_k && j.tiles_q > 0)
-    qbias_kernel<D><<<dim3(j.tiles_q, j.seqs.tps, j.Hq), kTile, 0, s>>>(j, j.q_bias);
+  if (j0.q_bias && j0.do_q && j0.do_k && j0.tiles_q > 0)
+    qbias_kernel<D><<<dim3(j0.tiles_q, j0.seqs.tps, j0.Hq), kTile, 0, s>>>(j0, j0.q_bias);
   return cudaGetLastError();
 }
 
 template <bool SV>
-static cudaError_t prepass_dispatch(const PrepassJob& j, int D, cudaStream_t s) {
-  if (D == 128) return j.bf16 ? launch_prepass<128, true, SV>(j, s) : launch_prepass<128, false, SV>(j, s);
-  return j.bf16 ? launch_prepass<64, true, SV>(j, s) : launch_prepass<64, false, SV>(j, s);
+static cudaError_t prepass_dispatch(const PrepassJob& j, int D, cudaStream_t s, int* path) {
+  if (D == 128)
+    return j.bf16 ? launch_prepass<128, true, SV>(j, s, path) : launch_prepass<128, false, SV>(j, s, path);
+  return j.bf16 ? launch_prepass<64, true, SV>(j, s, path) : launch_prepass<64, false, SV>(j, s, path);
 }
 
-cudaError_t prepass_run(const PrepassJob& j, int D, cudaStream_t s) {
-  return j.smooth_v ? prepass_dispatch<true>(j, D, s) : prepass_dispatch<false>(j, D, s);
+cudaError_t prepass_run(const PrepassJob& j, int D, cudaStream_t s, int* path) {
+  return j.smooth_v ? prepass_dispatch<true>(j, D, s, path) : prepass_dispatch<false>(j, D, s, path);
 }
 
 cudaError_t prepass_varlen_offsets(const int* cu_q, const int* cu_k, int n, int max_seqlen, int cap_q, int cap_k,

@@ -19,6 +19,7 @@ struct PrepassJob {
   int bf16 = 0, gran = 0, smooth_k = 0, smooth_q = 0, pv8 = 1, smooth_v = 0;
   int do_q = 0, do_k = 0, do_v = 0;
   int tiles_q = 0, tiles_k = 0;    // workspace tiles per head
+  int one_pass = 0;                // debug: K / V through the cluster kernel where a head fits one
   uint32_t* err = nullptr;
   unsigned long long* k_stat = nullptr;   // [nseq][Hkv][D] int64 (fp16) / fp64 bits (bf16) channel sums
   uint32_t* v_stat = nullptr;             // [nseq][Hkv][D][2]: float bits of channel |max|;
@@ -68,7 +69,10 @@ struct AttnParams {
 enum { kAccOne = 0, kAccTwo = 1, kAccTwoF16 = 2 };
 
 // prepass.cu
-cudaError_t prepass_run(const PrepassJob& j, int D, cudaStream_t s);
+// *path (optional): kPrepassOnePass when K / V went through the cluster
+// kernel, kPrepassTwoLaunch when through launches A / B, 0 when neither ran.
+enum { kPrepassOnePass = 1, kPrepassTwoLaunch = 2 };
+cudaError_t prepass_run(const PrepassJob& j, int D, cudaStream_t s, int* path);
 
 // SAGE_OK for cudaSuccess; otherwise records e as the calling thread's last
 // CUDA error (sage_last_cuda_error) and returns SAGE_ERR_CUDA.  (api.cu)

@@ -112,6 +112,9 @@ def test_debug_settings_validate_and_reset(L):
     assert L.sage_debug_withhold_k_tile(-2) == sage.ERR_INVALID_ARG
     assert L.sage_debug_set_max_ctas(3) == sage.OK and L.sage_debug_set_max_ctas(0) == sage.OK
     assert L.sage_debug_withhold_k_tile(5) == sage.OK and L.sage_debug_withhold_k_tile(-1) == sage.OK
+    assert L.sage_debug_set_prepass_one_pass(2) == sage.ERR_INVALID_ARG
+    assert L.sage_debug_set_prepass_one_pass(1) == sage.OK and L.sage_debug_set_prepass_one_pass(0) == sage.OK
+    assert L.sage_debug_last_prepass_path() in (0, 1, 2)
 
 
 def test_library_reads_no_environment():

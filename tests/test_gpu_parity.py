@@ -76,6 +76,17 @@ def max_ctas(n):
         sage.debug_set_max_ctas(0)
 
 
+@contextlib.contextmanager
+def prepass_path(path):
+    """Run the block with K / V of the pre-pass on `path`: "two_launch" (the
+    default) or "one_pass" (the cluster path, wherever a head fits it)."""
+    sage.debug_set_prepass_one_pass(path == "one_pass")
+    try:
+        yield
+    finally:
+        sage.debug_set_prepass_one_pass(False)
+
+
 def _ws_bytes(ws: torch.Tensor) -> np.ndarray:
     torch.cuda.synchronize()
     return ws.cpu().numpy()
@@ -92,13 +103,20 @@ def _ws_bytes(ws: torch.Tensor) -> np.ndarray:
     (64, 200, "per_token", "bf16", "NHD"),
 ])
 @pytest.mark.parametrize("smooth_k", [True, False])
-def test_prepass_codes_bit_exact(D, S, gran, dtype, layout, smooth_k):
+@pytest.mark.parametrize("path", ["two_launch", "one_pass"])
+def test_prepass_codes_bit_exact(D, S, gran, dtype, layout, smooth_k, path):
+    """Codes and scales of Q, K and V against the oracle, bit for bit, on both
+    K / V paths of the pre-pass."""
     sp = synth.Spec("t", Hq=4, Hkv=2, D=D, B=2, S=S, dtype=dtype, layout=layout, k_bias_std=3.0, seed=31)
     q, k, v = synth.make(sp)
     nb = sage.sage_workspace_bytes(2, 4, 2, S, D, 0, 0)
     ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
-    sage.quant_qk(_dev(q), _dev(k), ws, layout, gran, smooth_k=smooth_k)
-    sage.quant_v(_dev(v), ws, layout, "fp8")
+    expect = path
+    with prepass_path(path):
+        sage.quant_qk(_dev(q), _dev(k), ws, layout, gran, smooth_k=smooth_k)
+        assert sage.debug_last_prepass_path() == expect
+        sage.quant_v(_dev(v), ws, layout, "fp8")
+        assert sage.debug_last_prepass_path() == expect
     assert sage.get_device_error(ws) == (0, 0)
     L = sage.workspace_layout(2, 2 * S, 2 * S, S, 4, 2, D)
     W = _ws_bytes(ws)
@@ -139,7 +157,8 @@ def test_prepass_codes_bit_exact(D, S, gran, dtype, layout, smooth_k):
     (128, 300, "per_block", "fp16", "HND"),
     (64, 257, "per_thread", "bf16", "NHD"),
 ])
-def test_prepass_smooth_q_bit_exact(D, S, gran, dtype, layout):
+@pytest.mark.parametrize("path", ["two_launch", "one_pass"])
+def test_prepass_smooth_q_bit_exact(D, S, gran, dtype, layout, path):
     """Smooth Q: block means, INT8 codes of Q - mean, and the per-key score
     corrections (fp64 sum in channel order, rounded to float once)."""
     Hq, Hkv, B = 4, 2, 2
@@ -147,7 +166,8 @@ def test_prepass_smooth_q_bit_exact(D, S, gran, dtype, layout):
                     q_block_offset_std=1.0, seed=35)
     q, k, v = synth.make(sp)
     ws = torch.zeros(sage.sage_workspace_bytes(B, Hq, Hkv, S, D, 0, 1), dtype=torch.uint8, device="cuda")
-    sage.quant_qk(_dev(q), _dev(k), ws, layout, gran, smooth_k=True, smooth_q=True)
+    with prepass_path(path):
+        sage.quant_qk(_dev(q), _dev(k), ws, layout, gran, smooth_k=True, smooth_q=True)
     assert sage.get_device_error(ws) == (0, 0)
     L = sage.workspace_layout(B, B * S, B * S, S, Hq, Hkv, D, smooth_q=1)
     W = _ws_bytes(ws)
@@ -172,7 +192,8 @@ def test_prepass_smooth_q_bit_exact(D, S, gran, dtype, layout):
 
 
 @pytest.mark.parametrize("D,S,dtype,layout", [(128, 300, "fp16", "HND"), (64, 517, "bf16", "NHD")])
-def test_prepass_smooth_v_bit_exact(D, S, dtype, layout):
+@pytest.mark.parametrize("path", ["two_launch", "one_pass"])
+def test_prepass_smooth_v_bit_exact(D, S, dtype, layout, path):
     """Smooth V: channel mean (exact sum), E4M3 codes of V - mean and the
     scales, against the oracle; keys past the sequence stay 0."""
     Hq, Hkv, B = 2, 2, 2
@@ -180,7 +201,8 @@ def test_prepass_smooth_v_bit_exact(D, S, dtype, layout):
     q, k, v = synth.make(sp)
     v = v + torch.from_numpy(np.random.default_rng(7).normal(0, 8, D).astype(np.float32)).to(v.dtype)
     ws = torch.zeros(sage.sage_workspace_bytes(B, Hq, Hkv, S, D, 2, 0), dtype=torch.uint8, device="cuda")
-    sage.quant_v(_dev(v), ws, layout, "fp8_smooth_v")
+    with prepass_path(path):
+        sage.quant_v(_dev(v), ws, layout, "fp8_smooth_v")
     assert sage.get_device_error(ws) == (0, 0)
     L = sage.workspace_layout(B, B * S, B * S, S, Hq, Hkv, D, pv=2)
     W = _ws_bytes(ws)
@@ -197,6 +219,61 @@ def test_prepass_smooth_v_bit_exact(D, S, dtype, layout):
             assert np.array_equal(vs[b, h], rv.scales), (b, h)
             assert np.array_equal(g[:S], rv.codes), (b, h)
             assert np.all(g[S:] == 0)
+
+
+def _outputs_region(ws, L) -> np.ndarray:
+    """The workspace bytes the attention kernel reads (means, scales, codes),
+    i.e. everything past the pre-pass accumulators."""
+    return _ws_bytes(ws)[L["k_mean"]:L["total"]]
+
+
+@pytest.mark.parametrize("D,S,B,dtype,layout,pv", [
+    (128, 8000, 1, "fp16", "HND", "fp8"),           # 63 tiles: 16-CTA clusters, 4 tiles per CTA
+    (128, 4096, 2, "bf16", "NHD", "fp8_smooth_v"),  # 32 tiles: 16 x 2, the benchmark's shape class
+    (64, 16000, 1, "bf16", "HND", "fp8"),           # 125 tiles: 16 x 8
+    (64, 1000, 3, "fp16", "NHD", "fp16"),           # 8 tiles: 4 x 2
+    (128, 129, 2, "fp16", "HND", "fp8"),            # 2 tiles: one CTA per head
+])
+def test_prepass_paths_write_identical_bytes(D, S, B, dtype, layout, pv):
+    """Q, K and V through the one-pass cluster path and through the
+    two-launch path: every byte the attention kernel reads is the same, at
+    cluster shapes the CASES sizes do not reach (up to 16 CTAs x 8 tiles)."""
+    Hq, Hkv = 2, 2
+    sp = synth.Spec("t", Hq=Hq, Hkv=Hkv, D=D, B=B, S=S, dtype=dtype, layout=layout, k_bias_std=3.0, seed=37)
+    q, k, v = (_dev(t) for t in synth.make(sp))
+    code = {"fp8": 0, "fp16": 1, "fp8_smooth_v": 2}[pv]
+    L = sage.workspace_layout(B, B * S, B * S, S, Hq, Hkv, D, pv=code)
+    got = {}
+    for path in ("two_launch", "one_pass"):
+        ws = torch.zeros(sage.sage_workspace_bytes(B, Hq, Hkv, S, D, code, 0), dtype=torch.uint8, device="cuda")
+        with prepass_path(path):
+            sage.quant_qkv(q, k, v, ws, layout, "per_thread", pv)
+            taken = sage.debug_last_prepass_path()
+        assert sage.get_device_error(ws) == (0, 0)
+        assert taken == path, (path, taken)
+        got[path] = _outputs_region(ws, L)
+    assert np.array_equal(got["one_pass"], got["two_launch"])
+
+
+@pytest.mark.parametrize("pv,smooth_v", [("fp8", False), ("fp8", True), ("fp16", False)])
+def test_varlen_prepass_paths_agree(pv, smooth_v):
+    """Varlen with empty, one-token and ragged sequences: both K / V paths of
+    the pre-pass give the same attention output, bit for bit, and the
+    one-pass result matches the oracle."""
+    sp = synth.Spec("t", Hq=4, Hkv=2, D=64, seqlens=[200, 1, 0, 129, 1100, 77], causal=True, seed=51)
+    q, k, v = synth.make(sp)
+    cu = sp.cu_seqlens()
+    cu_d = torch.from_numpy(cu).cuda()
+    outs = {}
+    for path in ("two_launch", "one_pass"):
+        with prepass_path(path):
+            outs[path] = sage.sageattn_varlen(_dev(q), _dev(k), _dev(v), cu_d, cu_d, max(sp.seqlens), True,
+                                              pv_dtype=pv, pv_accum_dtype="fp32", smooth_v=smooth_v)
+            assert sage.debug_last_prepass_path() == path
+    torch.cuda.synchronize()
+    assert torch.equal(outs["one_pass"], outs["two_launch"])
+    ref = oracle.attention(q, k, v, causal=True, pv=pv, smooth_v=smooth_v, cu_seqlens=cu, with_allowance=True)
+    _assert_close(outs["one_pass"], ref, "fp16", "varlen one-pass pre-pass vs oracle")
 
 
 def test_prepass_v16_layout():
