@@ -99,9 +99,10 @@ __device__ __forceinline__ constexpr int kgrp(int col) {
   return KPT ? ((col >> 6) << 3) + (col & 7) : (col >> 6);
 }
 
-// Phase 1 of a tile for one query row.  The S accumulator was seeded with
-// the bit pattern of 1.5 * 2^23 before the MMA added the int32 products, so
-// each column holds the float t = 1.5 * 2^23 + S exactly (|S| < 2^22).
+// Phase 1 of a tile for one query row.  Each column of r holds the float
+// t = 1.5 * 2^23 + S exactly (|S| < 2^22): the S accumulator was seeded with
+// that bit pattern before the MMA added the int32 products (one-level), or
+// the pattern was added to the int32 sums in registers (two-level).
 // Masked keys -> -inf; returns the tile maximum m_tile = max_g c_g *
 // max_g(S) (c > 0 keeps the order; t is monotonic in S).
 template <bool KPT>
@@ -438,9 +439,11 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
   uint32_t ph = 3u * PH_LAST0;
   int kvbase = 0;       // K/V ring index of the item's first tile (smooth Q)
 
-  // seed the S columns for the first QK^T (see tile_max)
-  tmem_fill128(taddr, 0x4B400000u);
-  tmem_wait_st();
+  // one-level: seed the S columns for the first QK^T (see tile_max)
+  if (!ACC2) {
+    tmem_fill128(taddr, 0x4B400000u);
+    tmem_wait_st();
+  }
   tc_fence_before();
   mbar_arrive(bar(C::B_SCONS + q));
 
@@ -480,9 +483,18 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
         tc_fence_after();
         uint32_t r[128];
         tmem_ld128_sync(taddr, r);
-        // the S columns are read: re-seed them (the stores complete during the
-        // max below) and then let the next QK^T in -- of this item or the next
-        tmem_fill128(taddr, 0x4B400000u);
+        // The S columns are read.  One-level: re-seed them (the stores
+        // complete during the max below), then let the next QK^T in -- of
+        // this item or the next.  Two-level: S holds the plain int32 sums;
+        // adding the seed's bit pattern in registers gives the same float
+        // bits t = 1.5 * 2^23 + S (|S| < 2^22), and measured faster there
+        // than the tensor-memory stores.
+        if (ACC2) {
+#pragma unroll
+          for (int i = 0; i < 128; ++i) r[i] += 0x4B400000u;
+        } else {
+          tmem_fill128(taddr, 0x4B400000u);
+        }
         // keys past the sequence, or (causal) past this row, are masked
         const int col0 = j * kTile;
         const bool masked = (col0 + kTile > it.Lk) || (p.causal && j == qt);
@@ -808,7 +820,9 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
         for (int kk = 0; kk < D / 32; ++kk) {
           const uint64_t a = smem_desc(sb + C::OFF_Q + q * C::QT + kk * 32, D);
           const uint64_t bd = smem_desc(sb + C::OFF_K + st * C::QT + kk * 32, D);
-          mma_i8_ss(d, a, bd, ID_QK, 1);        // onto the 1.5 * 2^23 seed
+          // one-level: onto the 1.5 * 2^23 seed; two-level: the first K chunk
+          // overwrites S and the softmax adds the seed's bits itself
+          mma_i8_ss(d, a, bd, ID_QK, ACC2 ? (kk > 0) : 1);
         }
         tc_commit(bar(C::B_SFULL + q));
       };

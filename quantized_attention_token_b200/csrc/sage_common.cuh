@@ -186,14 +186,16 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
   }
 }
 
-// Bounded wait for single-thread roles (MMA issuer, loader): try_wait without
-// a suspend hint, so the thread reacts as soon as the phase completes.
+// Bounded wait for single-thread roles (MMA issuer, loader): a first try_wait,
+// then try_wait with a suspend-time hint, so that the waiting thread gives its
+// issue slots to the softmax warps on the same SM sub-partition (measured
+// faster than spinning) and still wakes when the phase completes.
 __device__ __forceinline__ bool mbar_wait_poll(uint32_t bar, uint32_t parity, volatile int* abort_flag,
                                                uint32_t* err, uint32_t bit) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
-    if (mbar_try_wait(bar, parity)) return true;
+    if (mbar_try_wait_sleep(bar, parity, 20000u)) return true;
     if ((it & 63u) == 0) {
       if (*abort_flag) return false;
       if (global_timer_ns() - t0 > kWaitLimitNs) {
