@@ -310,6 +310,17 @@ def sweep_s(sage, dev, gran, n=20):
             "peak": peak, "points": res}
 
 
+def bench_config(spec: synth.Spec, args) -> dict:
+    """The workload description both arms print (the reference arm times the
+    oracle on the same workload)."""
+    elem = spec.total_tokens * spec.D
+    return {"workload": spec.name, "B": spec.B, "H": spec.Hq, "Hkv": spec.Hkv, "S": spec.S, "D": spec.D,
+            "layout": spec.layout, "causal": spec.causal, "input_dtype": spec.dtype, "qk_gran": args.gran,
+            "pv": args.pv, "pv_accum": args.pv_accum,
+            "l2": "inputs larger than L2: Q/K/V %s = %d MiB per GPU, L2 126 MB" % (
+                spec.dtype, (spec.Hq + 2 * spec.Hkv) * elem * 2 >> 20)}
+
+
 # ----------------------------------------------------------------------------- main
 def main():
     args = parse()
@@ -334,7 +345,7 @@ def main():
                 "steps": args.steps, "warmup": args.warmup, "ms_per_step": ops / (val * 1e12) * 1e3,
                 "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "int8+e4m3 (f64 oracle)",
                 "data": "synthetic",
-                "config": {"workload": spec.name, "B": spec.B, "H": spec.Hq, "S": spec.S, "D": spec.D},
+                "config": bench_config(spec, args),
                 "cpu_baseline": cb,
                 "e2e": {"value": val, "unit": "TOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
         print(json.dumps(line), flush=True)
@@ -494,11 +505,7 @@ def main():
         "metric": METRIC, "value": value, "unit": "TOPS", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "int8+e4m3" if args.pv == "fp8" else "int8+f16", "data": "synthetic",
-        "config": {"workload": spec.name, "B": B, "H": spec.Hq, "Hkv": spec.Hkv, "S": S, "D": D,
-                   "layout": layout, "causal": spec.causal, "input_dtype": spec.dtype, "qk_gran": args.gran,
-                   "pv": args.pv, "pv_accum": args.pv_accum,
-                   "l2": "inputs larger than L2: Q/K/V %s = %d MiB per GPU, L2 126 MB" % (
-                       spec.dtype, (spec.Hq + 2 * spec.Hkv) * elem * 2 >> 20)},
+        "config": bench_config(spec, args),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": recorded_traffic(spec.name),
                      "kernel": "attn_fwd_kernel", "kernel_ms": attn_avg,
