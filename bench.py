@@ -195,15 +195,16 @@ def kernel_source_hash():
     return h.hexdigest()[:16]
 
 
-def recorded_traffic(workload: str):
-    """dram bytes per launch of the attention kernel from the committed ncu
-    summary, if it was taken on the current kernel source; else None."""
+def recorded_traffic(workload: str, mode: str):
+    """dram bytes per launch of the attention kernel in `mode` ("pv/accum")
+    from the committed ncu summary, if it was taken on the current kernel
+    source; else None."""
     path = os.path.join(ROOT, "profiles", "attn_fwd_traffic.json")
     try:
         d = json.load(open(path))
     except Exception:
         return None
-    e = d.get(workload)
+    e = d.get(f"{workload} {mode}")
     if not e or e.get("source_hash") != kernel_source_hash():
         return None
     return e.get("dram_bytes_per_launch")
@@ -507,14 +508,15 @@ def main():
         "vs_baseline": None, "dtype": "int8+e4m3" if args.pv == "fp8" else "int8+f16", "data": "synthetic",
         "config": bench_config(spec, args),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": recorded_traffic(spec.name),
+                     "frac": achieved / peak, "traffic": recorded_traffic(spec.name, f"{args.pv}/{args.pv_accum}"),
                      "kernel": "attn_fwd_kernel", "kernel_ms": attn_avg,
                      "mode": f"{args.pv}/{args.pv_accum}",
                      "peak_source": f"2 x bf16_tflops {peak_kind} ({pk_kind}: the dense FP8/INT8 rate is twice "
                                     f"bf16's); timed region {elapsed_ms:.1f} ms"},
         "roofline_two_level": None if two_ms is None else {
             "bound": "tensor", "achieved": ops / (two_ms * 1e-3) / 1e12, "peak": peak, "unit": "TFLOP/s",
-            "frac": ops / (two_ms * 1e-3) / 1e12 / peak, "traffic": None, "kernel": "attn_fwd_kernel",
+            "frac": ops / (two_ms * 1e-3) / 1e12 / peak, "traffic": recorded_traffic(spec.name, f"{two[0]}/{two[1]}"),
+            "kernel": "attn_fwd_kernel",
             "kernel_ms": two_ms, "mode": f"{two[0]}/{two[1]}",
             "note": "the two-level accumulation (the API default), attention kernel alone, 100 launches"},
         "prepass": {"ms": pre_avg, "achieved_gbs": pre_bytes / (pre_avg * 1e-3) / 1e9,
