@@ -20,8 +20,8 @@
  *          (pv_accum_dtype).
  *
  * The pages give no formulas, block sizes or rounding rules.  The readings
- * taken where they are silent are stated at each routine and listed in the
- * design notes: round-to-nearest-even everywhere, symmetric INT8 codes in
+ * taken where they are silent are stated at each routine; the main ones:
+ * round-to-nearest-even everywhere, symmetric INT8 codes in
  * [-127, 127], the group shapes of orc_q_group/orc_k_group, 128-key tiles in
  * increasing order for the online softmax, the row sum taken over the
  * unquantized P~, a static FP8 scale of 448 (the E4M3 maximum) for P~.
