@@ -341,6 +341,50 @@ def test_attention_matches_oracle(D, S, Hq, Hkv, causal, gran, pv, acc, dtype, l
     _check_accuracy(out, oracle.attention_exact(q, k, v, layout, causal), ref[0], pv, "vs fp64")
 
 
+def _random_cases(n=48, seed=2024):
+    """Seeded random configurations across the options the API takes:
+    shapes with ragged S, GQA ratios, layouts, types, granularities, P~V
+    modes, accumulation modes (lazy included), sm_scale and smooth_k."""
+    rng = np.random.default_rng(seed)
+    cases = []
+    for i in range(n):
+        D = int(rng.choice([64, 128]))
+        Hq, Hkv = [(2, 2), (4, 2), (4, 1), (3, 3), (6, 2)][int(rng.integers(5))]
+        pv = str(rng.choice(["fp8", "fp16"]))
+        accs = ["fp32", "fp32+fp32", "fp32_lazy"] + (["fp32+fp16"] if pv == "fp8" else [])
+        cases.append(dict(D=D, S=int(rng.integers(1, 600)), B=int(rng.integers(1, 4)), Hq=Hq, Hkv=Hkv,
+                          causal=bool(rng.integers(2)), gran=str(rng.choice(["per_block", "per_warp", "per_thread",
+                                                                             "per_token"])),
+                          pv=pv, acc=str(rng.choice(accs)), dtype=str(rng.choice(["fp16", "bf16"])),
+                          layout=str(rng.choice(["HND", "NHD"])),
+                          sm_scale=None if rng.integers(2) else float(rng.uniform(0.03, 0.2)),
+                          smooth_k=bool(rng.integers(4) > 0), seed=1000 + i))
+    return cases
+
+
+@pytest.mark.parametrize("c", _random_cases(), ids=lambda c: f"seed{c['seed']}")
+def test_attention_random_configurations_match_oracle(c):
+    """Element-wise parity and accuracy on seeded random configurations, so
+    that option combinations outside the hand-picked cases are covered too."""
+    # outlier K channels only where K is smoothed: without smoothing they are
+    # the error the method's smoothing step exists to remove
+    sp = synth.Spec("t", Hq=c["Hq"], Hkv=c["Hkv"], D=c["D"], B=c["B"], S=c["S"], dtype=c["dtype"],
+                    layout=c["layout"], causal=c["causal"], k_bias_std=3.0 if c["smooth_k"] else 0.0,
+                    seed=c["seed"])
+    q, k, v = synth.make(sp)
+    out = sage.sageattn(_dev(q), _dev(k), _dev(v), c["layout"], c["causal"], sm_scale=c["sm_scale"],
+                        qk_quant_gran=c["gran"], pv_dtype=c["pv"], pv_accum_dtype=c["acc"], smooth_k=c["smooth_k"])
+    torch.cuda.synchronize()
+    lazy = c["acc"] == "fp32_lazy"
+    tau = (2 if c["pv"] == "fp8" else 8) if lazy else 0
+    ref = oracle.attention(q, k, v, c["layout"], c["causal"], sm_scale=c["sm_scale"], gran=c["gran"], pv=c["pv"],
+                           smooth_k=c["smooth_k"], lazy_tau=tau, with_allowance=True,
+                           acc="fp32" if lazy else c["acc"])
+    _assert_close(out, ref, c["dtype"], f"vs oracle {c}")
+    _check_accuracy(out, oracle.attention_exact(q, k, v, c["layout"], c["causal"], sm_scale=c["sm_scale"]), ref[0],
+                    c["pv"], f"vs fp64 {c}")
+
+
 @pytest.mark.parametrize("D,S,causal,gran,pv,acc,dtype,layout", [
     (128, 384, False, "per_block", "fp8", "fp32", "fp16", "HND"),
     (128, 300, True, "per_thread", "fp8", "fp32+fp32", "bf16", "NHD"),
