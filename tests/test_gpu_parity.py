@@ -613,6 +613,48 @@ def test_varlen_cross_length_matches_oracle(n_ctas, causal, pv, acc):
     assert torch.count_nonzero(out[cq[b]:cq[b + 1]]).item() == 0
 
 
+def _random_varlen_cases(n=16, seed=77):
+    rng = np.random.default_rng(seed)
+    cases = []
+    for i in range(n):
+        ns = int(rng.integers(1, 7))
+        same = bool(rng.integers(2))
+        lq = [int(x) for x in rng.choice([0, 1, 17, 128, 129, 300, 513], size=ns)]
+        lk = lq if same else [int(x) for x in rng.choice([0, 1, 40, 128, 255, 400], size=ns)]
+        pv = str(rng.choice(["fp8", "fp16"]))
+        accs = ["fp32", "fp32+fp32"] + (["fp32+fp16"] if pv == "fp8" else [])
+        Hq, Hkv = [(2, 2), (4, 2), (8, 2), (3, 1)][int(rng.integers(4))]
+        cases.append(dict(lq=lq, lk=lk, Hq=Hq, Hkv=Hkv, D=int(rng.choice([64, 128])), causal=bool(rng.integers(2)),
+                          pv=pv, acc=str(rng.choice(accs)), gran=str(rng.choice(["per_block", "per_warp", "per_thread"])),
+                          dtype=str(rng.choice(["fp16", "bf16"])), seed=2000 + i))
+    return cases
+
+
+@pytest.mark.parametrize("c", _random_varlen_cases(), ids=lambda c: f"seed{c['seed']}")
+def test_varlen_random_configurations_match_oracle(c):
+    """Seeded random packed batches: own query and key boundaries (empty,
+    one-token and ragged sequences), grouped heads, both P~V modes, the
+    accumulation modes and granularities, fp16 and bf16."""
+    rng = np.random.default_rng(c["seed"])
+    lq, lk, H, Hk, D = c["lq"], c["lk"], c["Hq"], c["Hkv"], c["D"]
+    cq = np.concatenate([[0], np.cumsum(lq)]).astype(np.int32)
+    ck = np.concatenate([[0], np.cumsum(lk)]).astype(np.int32)
+    tdt = torch.float16 if c["dtype"] == "fp16" else torch.bfloat16
+    q = torch.from_numpy(rng.normal(size=(cq[-1], H, D)).astype(np.float32)).to(tdt)
+    k = torch.from_numpy((rng.normal(size=(ck[-1], Hk, D)) + rng.normal(0, 3, size=(1, Hk, D))).astype(np.float32)).to(tdt)
+    v = torch.from_numpy(rng.normal(size=(ck[-1], Hk, D)).astype(np.float32)).to(tdt)
+    mx = max(max(lq), max(lk), 1)
+    out = sage.sageattn_varlen(_dev(q), _dev(k), _dev(v), torch.from_numpy(cq).cuda(), torch.from_numpy(ck).cuda(),
+                               mx, c["causal"], qk_quant_gran=c["gran"], pv_dtype=c["pv"], pv_accum_dtype=c["acc"])
+    torch.cuda.synchronize()
+    ref = oracle.attention(q, k, v, causal=c["causal"], gran=c["gran"], pv=c["pv"], cu_seqlens=cq, cu_seqlens_k=ck,
+                           with_allowance=True, acc=c["acc"])
+    _assert_close(out, ref, c["dtype"], f"varlen vs oracle {c}")
+    for b in range(len(lq)):                   # a sequence without keys gives zero rows
+        if lk[b] == 0:
+            assert torch.count_nonzero(out[cq[b]:cq[b + 1]].float()).item() == 0
+
+
 # ----------------------------------------------------------------------------- fp32+fp16 accumulation
 def test_fp16_accumulation_partials_round_like_the_oracle():
     """Q = 0 makes every P~ exactly 1 (the scale-1 code); V of E4M3 integers
