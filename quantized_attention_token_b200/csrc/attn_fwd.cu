@@ -58,7 +58,8 @@ struct AttnCfg {
   static constexpr int OFF_ALPHA = OFF_P + NPB * NQ * PT;     // float [NQ][2][128]   (two-level)
   static constexpr int OFF_L = OFF_ALPHA + NQ * 2 * 128 * 4;  // float [NQ][128]      (two-level)
   static constexpr int OFF_BIAS = OFF_L + NQ * 128 * 4;       // float [NST][NQ][128]  (smooth Q)
-  static constexpr int OFF_BAR = OFF_BIAS + NST * NQ * 128 * 4;
+  static constexpr int OFF_KSC = OFF_BIAS + NST * NQ * 128 * 4;  // float [NST][16]: each K tile's group scales
+  static constexpr int OFF_BAR = OFF_KSC + NST * kKGroupsMax * 4;
   enum {
     B_QFULL = 0,
     B_QEMPTY = B_QFULL + NQ,         // MMA -> loader: the item's last QK^T with this Q tile is done
@@ -414,6 +415,7 @@ template <int D, bool PV8, bool ACC2, bool A16, bool KPT, bool BF16P, bool SMQ>
 __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, uint32_t tmem, int warp, int tid) {
   using C = AttnCfg<D, PV8, ACC2>;
   constexpr int NQ = C::NQ;
+  constexpr bool KSC_SMEM = KPT && !ACC2;   // K group scales from shared memory (see the tile loop)
   auto bar = [&](int i) -> uint32_t { return sb + C::OFF_BAR + 8 * i; };
   uint8_t* smem = reinterpret_cast<uint8_t*>(__cvta_shared_to_generic(sb));
   uint32_t* misc = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
@@ -437,7 +439,7 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
   enum : uint32_t { PH_S = 1, PH_PV = 2, PH_PVANY = 4, PH_TOK = 8, PH_GO = 16, PH_L = 32, PH_LANY = 64,
                     PH_A0 = 128 /* 2 bits */, PH_LAST0 = 512 /* 2 bits */ };
   uint32_t ph = 3u * PH_LAST0;
-  int kvbase = 0;       // K/V ring index of the item's first tile (smooth Q)
+  int kvbase = 0;       // K/V ring index of the item's first tile
 
   // one-level: seed the S columns for the first QK^T (see tile_max)
   if (!ACC2) {
@@ -462,21 +464,38 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
     float m = -INFINITY, l = 0.f;
     if (nq > 0) {
       const float qsc = p.q_scale[((size_t)it.h * p.tiles_q + it.tq0 + qt) * kQGroupsMax + q_group(p.gran, t)];
+      // K group scales: one-level per-thread mode reads each tile's 16 from
+      // shared memory, where they arrive with the V tile (16 live registers
+      // less in the tile loop); the other modes keep the next tile's few
+      // scales in registers, fetched one tile ahead (measured faster there)
       const float* ksb = p.k_scale + ((size_t)it.hk * p.tiles_k + it.tk0) * kKGroupsMax;
-      // K group scales of the next tile are fetched one tile ahead
-      float ksn[KPT ? 16 : 2];
+      float ksn[KSC_SMEM ? 1 : (KPT ? 16 : 2)];
+      if constexpr (!KSC_SMEM) {
 #pragma unroll
-      for (int g = 0; g < (KPT ? 16 : 2); ++g) ksn[g] = __ldg(ksb + g);
+        for (int g = 0; g < (KPT ? 16 : 2); ++g) ksn[g] = __ldg(ksb + g);
+      }
       if (!PV8 && NQ == 2 && q == 1 && it.n[0] > 0) {
         if (!(ok = mbar_wait(bar(C::B_GO), (ph / PH_GO) & 1, abort_flag, p.err, kErrTimeoutSoftmax))) break;
       }
       for (int j = 0; j < nq; ++j) {
+        const int kv = kvbase + j;
         float c[16];
+        if constexpr (KSC_SMEM) {
+          // the tile's K group scales (and, smooth Q, its key corrections)
+          // arrive with its V tile
+          if (!(ok = mbar_wait(bar(C::B_VFULL + kv % C::NST), (kv / C::NST) & 1, abort_flag, p.err,
+                               kErrTimeoutSoftmax)))
+            break;
+          const float* ksc = reinterpret_cast<const float*>(smem + C::OFF_KSC + (kv % C::NST) * (kKGroupsMax * 4));
 #pragma unroll
-        for (int g = 0; g < 16; ++g) c[g] = g < (KPT ? 16 : 2) ? fmaxf((qsc * ksn[g]) * p.sl2, 1e-30f) : 1e-30f;
-        if (j + 1 < nq) {
+          for (int g = 0; g < 16; ++g) c[g] = fmaxf((qsc * ksc[g]) * p.sl2, 1e-30f);
+        } else {
 #pragma unroll
-          for (int g = 0; g < (KPT ? 16 : 2); ++g) ksn[g] = __ldg(ksb + (j + 1) * kKGroupsMax + g);
+          for (int g = 0; g < 16; ++g) c[g] = g < (KPT ? 16 : 2) ? fmaxf((qsc * ksn[g]) * p.sl2, 1e-30f) : 1e-30f;
+          if (j + 1 < nq) {
+#pragma unroll
+            for (int g = 0; g < (KPT ? 16 : 2); ++g) ksn[g] = __ldg(ksb + (j + 1) * kKGroupsMax + g);
+          }
         }
         if (!(ok = mbar_wait(bar(C::B_SFULL + q), ph & PH_S, abort_flag, p.err, kErrTimeoutSoftmax))) break;
         ph ^= PH_S;
@@ -501,11 +520,12 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
         const int lim = p.causal ? min(it.Lk, row + 1) : it.Lk;
         float mt;
         if (SMQ) {
-          // the tile's key corrections arrive with its V tile
-          const int kv = kvbase + j;
-          if (!(ok = mbar_wait(bar(C::B_VFULL + kv % C::NST), (kv / C::NST) & 1, abort_flag, p.err,
-                               kErrTimeoutSoftmax)))
-            break;
+          if constexpr (!KSC_SMEM) {
+            // the tile's key corrections arrive with its V tile
+            if (!(ok = mbar_wait(bar(C::B_VFULL + kv % C::NST), (kv / C::NST) & 1, abort_flag, p.err,
+                                 kErrTimeoutSoftmax)))
+              break;
+          }
           const float* bias =
               reinterpret_cast<const float*>(smem + C::OFF_BIAS + ((kv % C::NST) * NQ + q) * 512);
           mt = tile_max_bias<KPT>(r, c, bias, p.sl2, masked, col0, lim);
@@ -632,7 +652,7 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
       Item<NQ> nx;
       if (next_busy_item<NQ>(p, opaque(idx), nx) && item_n<NQ>(nx, q) > 0) {
         prefetch_l1(p.q_scale + ((size_t)nx.h * p.tiles_q + nx.tq0 + nx.pair * NQ + q) * kQGroupsMax + q_group(p.gran, t));
-        prefetch_l1(p.k_scale + ((size_t)nx.hk * p.tiles_k + nx.tk0) * kKGroupsMax);
+        if (!KSC_SMEM) prefetch_l1(p.k_scale + ((size_t)nx.hk * p.tiles_k + nx.tk0) * kKGroupsMax);
       }
     }
     if (it.maxn > 0) {
@@ -751,6 +771,7 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
         if (!ok) break;
         const int8_t* kb = p.k_codes + ((size_t)it.hk * p.tiles_k + it.tk0) * C::QT;
         const uint8_t* vb = p.v_codes + ((size_t)it.hk * p.tiles_k + it.tk0) * (size_t)C::VT;
+        const float* ksc_b = p.k_scale + ((size_t)it.hk * p.tiles_k + it.tk0) * kKGroupsMax;
         // smooth Q: bias rows of the valid query tiles (n[q] > 0 for a prefix of q)
         int nbias = 0;
         if (p.q_bias)
@@ -771,8 +792,14 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
           issued_k = kv + 1;
           if (u > 0 && !(ok = mbar_wait_poll(bar(C::B_VEMPTY + st), (u - 1) & 1, abort_flag, p.err, kErrTimeoutLoad)))
             break;
-          mbar_expect_tx(bar(C::B_VFULL + st), C::VT + nbias * 512);
+          mbar_expect_tx(bar(C::B_VFULL + st), C::VT + nbias * 512 + (ACC2 ? 0 : kKGroupsMax * 4));
           bulk_g2s(sb + C::OFF_V + st * C::VT, vb + (size_t)t * C::VT, C::VT, bar(C::B_VFULL + st));
+          // one-level: the K tile's group scales ride with its V tile (the
+          // per-thread softmax reads them before its P~ of this tile; the
+          // stage is released only after that tile's last P~V)
+          if (!ACC2)
+            bulk_g2s(sb + C::OFF_KSC + st * (kKGroupsMax * 4), ksc_b + (size_t)t * kKGroupsMax, kKGroupsMax * 4,
+                     bar(C::B_VFULL + st));
           for (int q = 0; q < nbias; ++q)   // smooth Q: the query tiles' corrections for key tile t
             bulk_g2s(sb + C::OFF_BIAS + (st * NQ + q) * 512, bias_b + (size_t)q * p.bias_ld + (size_t)t * kTile, 512,
                      bar(C::B_VFULL + st));
