@@ -308,6 +308,18 @@ sage_status_t sage_debug_set_prepass_one_pass(int on);
  * pre-pass yet). */
 int sage_debug_last_prepass_path(void);
 
+/* Debug: on = 1 (the default) lets dense attention with one-level
+ * accumulation (fp32, fp32_lazy) write its output through a tensor map with
+ * asynchronous bulk tensor stores of each warp's staged rows; 0 makes every
+ * launch write the staged rows with per-warp 16-byte stores, the path that
+ * varlen and the two-level modes always take.  Both paths write identical
+ * bytes.  Process-wide.  Other values give SAGE_ERR_INVALID_ARG. */
+sage_status_t sage_debug_set_out_map(int on);
+
+/* Debug: the output store path of the calling thread's last attention launch:
+ * 1 the tensor map, 2 per-warp stores, 0 none yet. */
+int sage_debug_last_out_path(void);
+
 /* Debug: the int32 scores of one 128x128 tile, S = Q_codes(q tile) *
  * K_codes(k tile)^T, computed by the same tensor-core MMA path as the
  * attention kernel from a workspace filled by sage_quant_qk.  s_out: device

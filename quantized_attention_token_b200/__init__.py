@@ -20,7 +20,8 @@ from typing import Optional
 __all__ = [
     "sageattn", "sageattn_varlen", "quant_qk", "quant_qkv", "quant_v", "attn_quantized", "workspace_layout",
     "get_device_error", "debug_qk_tile", "debug_set_max_ctas", "debug_withhold_k_tile",
-    "debug_set_prepass_one_pass", "debug_last_prepass_path", "Workspace", "SageError",
+    "debug_set_prepass_one_pass", "debug_last_prepass_path", "debug_set_out_map", "debug_last_out_path",
+    "Workspace", "SageError",
     "lib", "LIB_PATH",
 ]
 
@@ -80,6 +81,8 @@ def lib():
         "sage_debug_withhold_k_tile": (I, [I]),
         "sage_debug_set_prepass_one_pass": (I, [I]),
         "sage_debug_last_prepass_path": (I, []),
+        "sage_debug_set_out_map": (I, [I]),
+        "sage_debug_last_out_path": (I, []),
     }
     for name, (res, args) in sigs.items():
         fn = getattr(L, name)
@@ -328,3 +331,19 @@ def debug_last_prepass_path():
     """"one_pass", "two_launch" or None: the K / V path of this thread's last
     pre-pass."""
     return PREPASS_PATH[lib().sage_debug_last_prepass_path()]
+
+
+OUT_PATH = {0: None, 1: "tensor_map", 2: "warp_stores"}
+
+
+def debug_set_out_map(on: bool):
+    """Let dense one-level attention store its output through a tensor map
+    (the default) or make every launch use per-warp stores.  Process-wide;
+    both paths write identical bytes."""
+    _check("sage_debug_set_out_map", lib().sage_debug_set_out_map(int(bool(on))))
+
+
+def debug_last_out_path():
+    """"tensor_map", "warp_stores" or None: the output store path of this
+    thread's last attention launch."""
+    return OUT_PATH[lib().sage_debug_last_out_path()]

@@ -27,13 +27,18 @@ sage_status_t cuda_status(cudaError_t e) {
 namespace {
 
 // Debug settings (sage_debug_set_max_ctas, sage_debug_withhold_k_tile,
-// sage_debug_set_prepass_one_pass): process-wide, read at each launch.
+// sage_debug_set_prepass_one_pass, sage_debug_set_out_map): process-wide, read
+// at each launch.
 std::atomic<int> g_max_ctas{0};
 std::atomic<int> g_withhold_k{-1};
 std::atomic<int> g_prepass_one_pass{0};
+std::atomic<int> g_out_map{1};
 // The K / V path of the calling thread's last pre-pass (kPrepassOnePass /
 // kPrepassTwoLaunch, 0 none).
 thread_local int g_last_prepass_path = 0;
+// The output store path of the calling thread's last attention launch
+// (1 tensor map, 2 per-warp stores, 0 none).
+thread_local int g_last_out_path = 0;
 
 // ---------------------------------------------------------------- device check
 sage_status_t check_device() {
@@ -192,6 +197,41 @@ sage_status_t run_prepass(const void* q, const void* k, const void* v, int bf16,
   return cuda_status(prepass_run(j, D, s, &g_last_prepass_path));
 }
 
+// cuTensorMapEncodeTiled, looked up once through the runtime (no link to the
+// driver library); null when the driver does not provide it.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn encode_tiled() {
+  static const EncodeTiledFn fn = [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q{};
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      (void)cudaGetLastError();
+      return (EncodeTiledFn) nullptr;
+    }
+    return reinterpret_cast<EncodeTiledFn>(f);
+  }();
+  return fn;
+}
+
+// The output as a 4-D tensor (D, S, H, B) of 16-bit values (HND and NHD differ
+// only in the strides), boxes of 64 columns x 32 rows, 128-byte swizzle.  Rows
+// past S fall outside the tensor, so the stores clip the last tile.  False
+// (plain stores) when the encoder is missing or refuses the shape.
+bool encode_out_map(CUtensorMap& m, const AttnParams& p, int D, int B, int H, int S) {
+  const EncodeTiledFn enc = encode_tiled();
+  if (!enc || S <= 0) return false;
+  const cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)S, (cuuint64_t)H, (cuuint64_t)B};
+  const cuuint64_t strides[3] = {(cuuint64_t)p.os.ss * 2, (cuuint64_t)p.os.sh * 2, (cuuint64_t)p.os.sb * 2};
+  const cuuint32_t box[4] = {64, 32, 1, 1};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  return enc(&m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 4, p.out, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 sage_status_t run_attn(void* out, int bf16, Strides so, const Seqs& seqs, int nseq, int Hq, int Hkv, int D,
                        int causal, float sm_scale, int gran, int pv, int acc, int smooth_q, const void* ws,
                        const sage_ws_layout_t& L, cudaStream_t s) {
@@ -224,7 +264,12 @@ sage_status_t run_attn(void* out, int bf16, Strides so, const Seqs& seqs, int ns
   p.max_ctas = g_max_ctas.load();
   p.dbg_withhold_k = g_withhold_k.load();
   const int mode = acc == SAGE_ACC_FP32_FP32 ? kAccTwo : acc == SAGE_ACC_FP32_FP16 ? kAccTwoF16 : kAccOne;
-  return cuda_status(attn_forward(p, D, pv != SAGE_PV_FP16, mode, seqs.max_seqlen, nseq, s));
+  // dense one-level: the epilogue stores through a tensor map of the output
+  CUtensorMap out_map{};
+  p.use_out_map =
+      (g_out_map.load() && !seqs.cu_q && mode == kAccOne && encode_out_map(out_map, p, D, nseq, Hq, seqs.S)) ? 1 : 0;
+  g_last_out_path = p.use_out_map ? 1 : 2;
+  return cuda_status(attn_forward(p, out_map, D, pv != SAGE_PV_FP16, mode, seqs.max_seqlen, nseq, s));
 }
 
 Seqs dense_seqs(int S) {
@@ -453,6 +498,14 @@ SAGE_EXPORT sage_status_t sage_debug_set_prepass_one_pass(int on) {
 }
 
 SAGE_EXPORT int sage_debug_last_prepass_path(void) { return g_last_prepass_path; }
+
+SAGE_EXPORT sage_status_t sage_debug_set_out_map(int on) {
+  if (on != 0 && on != 1) return SAGE_ERR_INVALID_ARG;
+  g_out_map.store(on);
+  return SAGE_OK;
+}
+
+SAGE_EXPORT int sage_debug_last_out_path(void) { return g_last_out_path; }
 
 SAGE_EXPORT int sage_last_cuda_error(void) { return sage::g_last_cuda_error; }
 

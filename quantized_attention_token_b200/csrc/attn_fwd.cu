@@ -285,17 +285,24 @@ __device__ __forceinline__ void store_row(uint16_t* orow, uint32_t ob, const flo
 // rounded to 16 bits.  Each thread puts its row in shared memory, in 16-byte
 // chunks XOR-swizzled by row, and then the warp writes whole rows: one store
 // instruction covers 512 contiguous bytes of two (D = 128) or four (D = 64)
-// rows.  Rows 0-15 are staged at stage0, rows 16-31 at stage1, each 16 x 2D
-// bytes: the warp's own rows of the query tile's two P~ halves, which only
-// this warp writes next.
-template <int D, bool PV8>
+// rows.  The staging areas stage0 and stage1 (4 KB each) are the warp's own
+// rows of the query tile's two P~ halves, which only this warp writes next.
+// BOXED: the layout is that of the boxes of the output tensor map (64 columns
+// x 32 rows of 128 bytes, 16-byte chunk c of row r at c ^ (r mod 8): the
+// 128-byte swizzle), columns 0-63 at stage0 and 64-127 at stage1; otherwise
+// rows 0-15 are at stage0 and 16-31 at stage1, chunk c of row r at
+// c ^ (r mod chunks per row).  by_map (BOXED only): the caller stores the
+// boxes with bulk tensor stores; otherwise the warp writes the rows here.
+template <int D, bool PV8, bool BOXED>
 __device__ __forceinline__ void store_tile(uint16_t* orow0, long long ss, int nvalid, uint32_t stage0, uint32_t stage1,
                                            uint32_t ob, float inv_l, const float* vsc, const float* vmu, bool bf16,
-                                           bool have_o, int lane) {
-  constexpr int RB = 2 * D;       // bytes of an output row
-  constexpr int CH = RB / 16;     // 16-byte chunks per row
+                                           bool have_o, int lane, bool by_map) {
+  constexpr int CH = 2 * D / 16;  // 16-byte chunks per row
   constexpr int RPI = 32 / CH;    // rows per warp store instruction
-  const uint32_t my_row = (lane < 16 ? stage0 : stage1) + (lane & 15) * RB;
+  auto chunk_addr = [&](int r, int k) -> uint32_t {
+    if (BOXED) return ((k >> 3) ? stage1 : stage0) + r * 128 + (((k & 7) ^ (r & 7)) << 4);
+    return (r < 16 ? stage0 : stage1) + (r & 15) * (2 * D) + ((k ^ (r & (CH - 1))) << 4);
+  };
 #pragma unroll
   for (int ch = 0; ch < D / 32; ++ch) {
     uint32_t r[32];
@@ -323,14 +330,15 @@ __device__ __forceinline__ void store_tile(uint16_t* orow0, long long ss, int nv
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk) {
       const int k = ch * 4 + kk;
-      st_shared_v4(my_row + ((k ^ (lane & (CH - 1))) << 4), w[4 * kk], w[4 * kk + 1], w[4 * kk + 2], w[4 * kk + 3]);
+      st_shared_v4(chunk_addr(lane, k), w[4 * kk], w[4 * kk + 1], w[4 * kk + 2], w[4 * kk + 3]);
     }
   }
+  if (BOXED && by_map) return;
   __syncwarp();
 #pragma unroll
   for (int i = 0; i < 32 / RPI; ++i) {
     const int rr = i * RPI + lane / CH, k = lane % CH;
-    const uint4 v = ld_shared_v4((rr < 16 ? stage0 : stage1) + (rr & 15) * RB + ((k ^ (rr & (CH - 1))) << 4));
+    const uint4 v = ld_shared_v4(chunk_addr(rr, k));
     if (rr < nvalid) *reinterpret_cast<uint4*>(orow0 + rr * ss + k * 8) = v;
   }
   __syncwarp();
@@ -412,7 +420,8 @@ __device__ __forceinline__ bool next_busy_item(const AttnParams& p, int idx, Ite
 // One softmax warpgroup: for each item, the online softmax of query tile q
 // over its KV tiles; in one-level mode also the O rescale and the epilogue.
 template <int D, bool PV8, bool ACC2, bool A16, bool KPT, bool BF16P, bool SMQ>
-__device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, uint32_t tmem, int warp, int tid) {
+__device__ __forceinline__ void softmax_role(const AttnParams& p, const CUtensorMap* out_map, uint32_t sb,
+                                             uint32_t tmem, int warp, int tid) {
   using C = AttnCfg<D, PV8, ACC2>;
   constexpr int NQ = C::NQ;
   constexpr bool KSC_SMEM = KPT && !ACC2;   // K group scales from shared memory (see the tile loop)
@@ -455,6 +464,12 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
     const int qt = it.pair * NQ + q;
     const int row = qt * kTile + t;
     const int nq = item_n<NQ>(it, q);
+    if (!ACC2 && p.use_out_map) {
+      // the previous item's output stores have read the staging area that
+      // this item's P~ and epilogue overwrite
+      if ((t & 31) == 0) bulk_wait_read0();
+      __syncwarp();
+    }
     // FP8 token: warpgroup of the next busy item's first exponential phase
     int next_first = -1;
     if (PV8 && NQ == 2 && it.maxn > 0) {
@@ -690,15 +705,31 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, uint32_t sb, u
       // 16-bit: the two 64-key halves of the one buffer)
       const uint32_t half = C::NPB == 2 ? (uint32_t)(NQ * C::PT) : (uint32_t)(C::PT / 2);
       const uint32_t stage0 = sb + C::OFF_P + q * C::PT + w * 4096;
-      store_tile<D, PV8>(orow0, p.os.ss, min(32, max(0, io.Lq - row0)), stage0, stage0 + half, ob,
-                         l > 0.f ? 1.0f / l : 0.f, vsc, vmu, bf16, nq > 0, t & 31);
+      const int nvalid = min(32, max(0, io.Lq - row0));
+      const bool by_map = !ACC2 && p.use_out_map != 0;
+      store_tile<D, PV8, !ACC2>(orow0, p.os.ss, nvalid, stage0, stage0 + half, ob, l > 0.f ? 1.0f / l : 0.f, vsc, vmu,
+                         bf16, nq > 0, t & 31, by_map);
+      if (by_map) {
+        // dense: the boxes go out with asynchronous bulk tensor stores; the
+        // staging area is reused only after they have read it (the wait at
+        // the next item's start)
+        fence_proxy_async_smem();
+        __syncwarp();
+        if ((t & 31) == 0 && nvalid > 0) {
+          tma_store_4d(out_map, stage0, 0, row0, io.h, io.b);
+          if (D == 128) tma_store_4d(out_map, stage0 + half, 64, row0, io.h, io.b);
+          bulk_commit();
+        }
+      }
     }
   }
+  // no bulk store still reads this CTA's shared memory when it ends
+  if (!ACC2 && (t & 31) == 0) bulk_wait_read0();
 }
 
 // ---------------------------------------------------------------- kernel
 template <int D, bool PV8, bool ACC2, bool A16>
-__global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p, const __grid_constant__ CUtensorMap out_map) {
   using C = AttnCfg<D, PV8, ACC2>;
   constexpr int NQ = C::NQ, NST = C::NST;
   extern __shared__ uint8_t smem_raw[];
@@ -959,7 +990,7 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p) {
     // ------------------------------------------------------------ softmax
     const bool bf16p = !PV8 && p.out_bf16;
     const int variant = (p.gran == 2 ? 4 : 0) + (bf16p ? 2 : 0) + (p.q_bias ? 1 : 0);
-#define SAGE_SOFTMAX(KPT, BF16P, SMQ) softmax_role<D, PV8, ACC2, A16, KPT, BF16P, SMQ>(p, sb, tmem, warp, tid)
+#define SAGE_SOFTMAX(KPT, BF16P, SMQ) softmax_role<D, PV8, ACC2, A16, KPT, BF16P, SMQ>(p, &out_map, sb, tmem, warp, tid)
     switch (variant) {
       case 0: SAGE_SOFTMAX(false, false, false); break;
       case 1: SAGE_SOFTMAX(false, false, true); break;
@@ -1124,7 +1155,7 @@ __global__ void __launch_bounds__(128, 1) qk_tile_kernel(const int8_t* qt, const
 // fewer when there are fewer items, or p.max_ctas when that is set (a debug
 // cap: results do not depend on the grid).
 template <int D, bool PV8, bool ACC2, bool A16>
-static cudaError_t launch_attn(const AttnParams& p, cudaStream_t s) {
+static cudaError_t launch_attn(const AttnParams& p, const CUtensorMap& out_map, cudaStream_t s) {
   using C = AttnCfg<D, PV8, ACC2>;
   auto k = attn_fwd_kernel<D, PV8, ACC2, A16>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
@@ -1139,7 +1170,7 @@ static cudaError_t launch_attn(const AttnParams& p, cudaStream_t s) {
   if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
   if (p.max_ctas > 0 && p.max_ctas < sms) sms = p.max_ctas;
   const int grid = p.n_items < sms ? p.n_items : sms;
-  k<<<grid, C::NTHREADS, C::SMEM_BYTES, s>>>(p);
+  k<<<grid, C::NTHREADS, C::SMEM_BYTES, s>>>(p, out_map);
   return cudaGetLastError();
 }
 
@@ -1149,8 +1180,8 @@ int attn_tiles_per_cta(int D, bool pv8, bool acc2) {
   return acc2 ? 1 : 2;
 }
 
-cudaError_t attn_forward(const AttnParams& p0, int D, bool pv8, int acc, int max_len_q, int nseq,
-                         cudaStream_t s) {
+cudaError_t attn_forward(const AttnParams& p0, const CUtensorMap& out_map, int D, bool pv8, int acc, int max_len_q,
+                         int nseq, cudaStream_t s) {
   const bool acc2 = acc != kAccOne;
   const int per = attn_tiles_per_cta(D, pv8, acc2) * kTile;
   const long long nx = (max_len_q + per - 1) / per;
@@ -1164,16 +1195,16 @@ cudaError_t attn_forward(const AttnParams& p0, int D, bool pv8, int acc, int max
   p.n_items = (int)items;
   if (D == 128) {
     if (pv8) {
-      if (acc == kAccTwoF16) return launch_attn<128, true, true, true>(p, s);
-      return acc2 ? launch_attn<128, true, true, false>(p, s) : launch_attn<128, true, false, false>(p, s);
+      if (acc == kAccTwoF16) return launch_attn<128, true, true, true>(p, out_map, s);
+      return acc2 ? launch_attn<128, true, true, false>(p, out_map, s) : launch_attn<128, true, false, false>(p, out_map, s);
     }
-    return acc2 ? launch_attn<128, false, true, false>(p, s) : launch_attn<128, false, false, false>(p, s);
+    return acc2 ? launch_attn<128, false, true, false>(p, out_map, s) : launch_attn<128, false, false, false>(p, out_map, s);
   }
   if (pv8) {
-    if (acc == kAccTwoF16) return launch_attn<64, true, true, true>(p, s);
-    return acc2 ? launch_attn<64, true, true, false>(p, s) : launch_attn<64, true, false, false>(p, s);
+    if (acc == kAccTwoF16) return launch_attn<64, true, true, true>(p, out_map, s);
+    return acc2 ? launch_attn<64, true, true, false>(p, out_map, s) : launch_attn<64, true, false, false>(p, out_map, s);
   }
-  return acc2 ? launch_attn<64, false, true, false>(p, s) : launch_attn<64, false, false, false>(p, s);
+  return acc2 ? launch_attn<64, false, true, false>(p, out_map, s) : launch_attn<64, false, false, false>(p, out_map, s);
 }
 
 cudaError_t debug_qk_tile(const int8_t* qt, const int8_t* kt, int D, int32_t* out, uint32_t* err,

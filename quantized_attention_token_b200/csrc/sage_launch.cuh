@@ -2,6 +2,8 @@
 // libsage CUDA translation units (pre-pass, attention, C ABI).
 #pragma once
 
+#include <cuda.h>   // CUtensorMap (encoded through the runtime's driver entry point)
+
 #include "sage.h"
 #include "sage_common.cuh"
 
@@ -38,6 +40,11 @@ struct PrepassJob {
 };
 
 struct AttnParams {
+  // 1: the epilogue stores each warp's staged rows with asynchronous bulk
+  // tensor stores through the output tensor map (a separate kernel parameter:
+  // dense one-level modes); 0: plain stores (varlen, two-level modes, or no
+  // encoder available).
+  int use_out_map;
   const int8_t* q_codes;
   const float* q_scale;
   const int8_t* k_codes;
@@ -82,8 +89,10 @@ cudaError_t prepass_varlen_offsets(const int* cu_q, const int* cu_k, int n, int 
 
 // attn_fwd.cu
 int attn_tiles_per_cta(int D, bool pv8, bool acc2);
-cudaError_t attn_forward(const AttnParams& p, int D, bool pv8, int acc, int max_len_q, int nseq,
-                         cudaStream_t s);
+// out_map: the output as a 4-D tensor map (D, S, H, B) of 16-bit values with
+// 64 x 32 boxes in the 128-byte swizzle, read when p.use_out_map is 1.
+cudaError_t attn_forward(const AttnParams& p, const CUtensorMap& out_map, int D, bool pv8, int acc, int max_len_q,
+                         int nseq, cudaStream_t s);
 cudaError_t debug_qk_tile(const int8_t* qt, const int8_t* kt, int D, int32_t* out, uint32_t* err,
                           cudaStream_t s);
 

@@ -115,6 +115,9 @@ def test_debug_settings_validate_and_reset(L):
     assert L.sage_debug_set_prepass_one_pass(2) == sage.ERR_INVALID_ARG
     assert L.sage_debug_set_prepass_one_pass(1) == sage.OK and L.sage_debug_set_prepass_one_pass(0) == sage.OK
     assert L.sage_debug_last_prepass_path() in (0, 1, 2)
+    assert L.sage_debug_set_out_map(2) == sage.ERR_INVALID_ARG
+    assert L.sage_debug_set_out_map(0) == sage.OK and L.sage_debug_set_out_map(1) == sage.OK
+    assert L.sage_debug_last_out_path() in (0, 1, 2)
 
 
 def test_library_reads_no_environment():

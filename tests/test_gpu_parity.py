@@ -500,6 +500,52 @@ def test_repeated_calls_are_deterministic():
     assert torch.equal(a, b)
 
 
+@contextlib.contextmanager
+def out_map(on):
+    """Run the block with the tensor-map output stores of dense one-level
+    attention on (the default) or off (per-warp stores everywhere)."""
+    sage.debug_set_out_map(on)
+    try:
+        yield
+    finally:
+        sage.debug_set_out_map(True)
+
+
+@pytest.mark.parametrize("D,S,B,Hq,causal,pv,acc,dtype,layout", [
+    (128, 4096, 1, 2, False, "fp8", "fp32", "fp16", "HND"),
+    (128, 1000, 2, 3, True, "fp16", "fp32", "bf16", "NHD"),
+    (64, 777, 2, 2, True, "fp8", "fp32_lazy", "fp16", "NHD"),
+    (64, 160, 1, 4, False, "fp16", "fp32_lazy", "bf16", "HND"),
+    (128, 33, 3, 2, True, "fp8", "fp32", "bf16", "HND"),
+])
+def test_output_store_paths_write_identical_bytes(D, S, B, Hq, causal, pv, acc, dtype, layout):
+    """Dense one-level attention writes its output through the tensor map by
+    default; per-warp stores of the same staged rows give the same bytes, also
+    for ragged last tiles and both layouts."""
+    sp = synth.Spec("t", Hq=Hq, Hkv=Hq, D=D, B=B, S=S, dtype=dtype, layout=layout, seed=61)
+    q, k, v = (_dev(t) for t in synth.make(sp))
+    a = sage.sageattn(q, k, v, layout, causal, pv_dtype=pv, pv_accum_dtype=acc)
+    torch.cuda.synchronize()
+    assert sage.debug_last_out_path() == "tensor_map"
+    with out_map(False):
+        b = sage.sageattn(q, k, v, layout, causal, pv_dtype=pv, pv_accum_dtype=acc)
+        torch.cuda.synchronize()
+        assert sage.debug_last_out_path() == "warp_stores"
+    assert torch.equal(a, b)
+
+
+def test_two_level_and_varlen_use_warp_stores():
+    sp = synth.Spec("t", Hq=2, Hkv=2, D=128, B=1, S=256, layout="NHD", seed=62)
+    q, k, v = (_dev(t) for t in synth.make(sp))
+    sage.sageattn(q, k, v, "NHD", False, pv_dtype="fp8", pv_accum_dtype="fp32+fp32")
+    torch.cuda.synchronize()
+    assert sage.debug_last_out_path() == "warp_stores"
+    cu = torch.tensor([0, 256], dtype=torch.int32, device="cuda")
+    sage.sageattn_varlen(q[0], k[0], v[0], cu, cu, 256, False, pv_accum_dtype="fp32")
+    torch.cuda.synchronize()
+    assert sage.debug_last_out_path() == "warp_stores"
+
+
 @pytest.mark.parametrize("pv", ["fp8", "fp16"])
 def test_one_level_accumulation_as_accurate_as_two_level(pv):
     """The two accumulation modes see the same P~ and V codes; they differ in
