@@ -728,7 +728,13 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, const CUtensor
 }
 
 // ---------------------------------------------------------------- kernel
-template <int D, bool PV8, bool ACC2, bool A16>
+// VAR: the softmax variant, fixed at compile time (0-7: 4 per_thread K
+// scales, 2 bf16 P~, 1 smooth-Q correction; the host picks the kernel), or -1
+// for all variants behind a run-time switch.  The two-level kernels are built
+// per variant: with the eight compiled into one kernel, the smooth-Q ones made
+// it spill and the plain per_block path ran 3-4 % slower.  The one-level
+// kernels keep the switch, which measured 1-3 % faster for them.
+template <int D, bool PV8, bool ACC2, bool A16, int VAR>
 __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p, const __grid_constant__ CUtensorMap out_map) {
   using C = AttnCfg<D, PV8, ACC2>;
   constexpr int NQ = C::NQ, NST = C::NST;
@@ -991,15 +997,20 @@ __global__ void __launch_bounds__(384, 1) attn_fwd_kernel(const AttnParams p, co
     const bool bf16p = !PV8 && p.out_bf16;
     const int variant = (p.gran == 2 ? 4 : 0) + (bf16p ? 2 : 0) + (p.q_bias ? 1 : 0);
 #define SAGE_SOFTMAX(KPT, BF16P, SMQ) softmax_role<D, PV8, ACC2, A16, KPT, BF16P, SMQ>(p, &out_map, sb, tmem, warp, tid)
-    switch (variant) {
-      case 0: SAGE_SOFTMAX(false, false, false); break;
-      case 1: SAGE_SOFTMAX(false, false, true); break;
-      case 2: SAGE_SOFTMAX(false, true, false); break;
-      case 3: SAGE_SOFTMAX(false, true, true); break;
-      case 4: SAGE_SOFTMAX(true, false, false); break;
-      case 5: SAGE_SOFTMAX(true, false, true); break;
-      case 6: SAGE_SOFTMAX(true, true, false); break;
-      default: SAGE_SOFTMAX(true, true, true); break;
+    if constexpr (VAR >= 0) {
+      (void)variant;
+      SAGE_SOFTMAX((VAR & 4) != 0, (VAR & 2) != 0, (VAR & 1) != 0);
+    } else {
+      switch (variant) {
+        case 0: SAGE_SOFTMAX(false, false, false); break;
+        case 1: SAGE_SOFTMAX(false, false, true); break;
+        case 2: SAGE_SOFTMAX(false, true, false); break;
+        case 3: SAGE_SOFTMAX(false, true, true); break;
+        case 4: SAGE_SOFTMAX(true, false, false); break;
+        case 5: SAGE_SOFTMAX(true, false, true); break;
+        case 6: SAGE_SOFTMAX(true, true, false); break;
+        default: SAGE_SOFTMAX(true, true, true); break;
+      }
     }
 #undef SAGE_SOFTMAX
   } else if (ACC2) {
@@ -1154,10 +1165,10 @@ __global__ void __launch_bounds__(128, 1) qk_tile_kernel(const int8_t* qt, const
 // Persistent grid: one CTA per SM (each holds all of an SM's tensor memory),
 // fewer when there are fewer items, or p.max_ctas when that is set (a debug
 // cap: results do not depend on the grid).
-template <int D, bool PV8, bool ACC2, bool A16>
+template <int D, bool PV8, bool ACC2, bool A16, int VAR>
 static cudaError_t launch_attn(const AttnParams& p, const CUtensorMap& out_map, cudaStream_t s) {
   using C = AttnCfg<D, PV8, ACC2>;
-  auto k = attn_fwd_kernel<D, PV8, ACC2, A16>;
+  auto k = attn_fwd_kernel<D, PV8, ACC2, A16, VAR>;
   cudaError_t e = cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES);
   if (e != cudaSuccess) return e;
   // the register split needs the launch allocation it was sized for: with
@@ -1180,6 +1191,32 @@ int attn_tiles_per_cta(int D, bool pv8, bool acc2) {
   return acc2 ? 1 : 2;
 }
 
+// Two-level kernels: the instantiation of softmax variant `var` (the same
+// bits as the kernel's run-time switch); bf16 P~ exists only for 16-bit P~V.
+template <int D, bool PV8, bool A16, int V = 0>
+static cudaError_t launch_two_level(const AttnParams& p, const CUtensorMap& out_map, int var, cudaStream_t s) {
+  if constexpr (V > 7) {
+    return cudaErrorInvalidValue;
+  } else if constexpr (PV8 && (V & 2)) {
+    return launch_two_level<D, PV8, A16, V + 1>(p, out_map, var, s);
+  } else {
+    if (var == V) return launch_attn<D, PV8, true, A16, V>(p, out_map, s);
+    return launch_two_level<D, PV8, A16, V + 1>(p, out_map, var, s);
+  }
+}
+
+template <int D>
+static cudaError_t launch_mode(const AttnParams& p, const CUtensorMap& out_map, bool pv8, int acc, cudaStream_t s) {
+  const int var = (p.gran == 2 ? 4 : 0) + (!pv8 && p.out_bf16 ? 2 : 0) + (p.q_bias ? 1 : 0);
+  if (pv8) {
+    if (acc == kAccTwoF16) return launch_two_level<D, true, true>(p, out_map, var, s);
+    if (acc == kAccTwo) return launch_two_level<D, true, false>(p, out_map, var, s);
+    return launch_attn<D, true, false, false, -1>(p, out_map, s);
+  }
+  if (acc == kAccTwo) return launch_two_level<D, false, false>(p, out_map, var, s);
+  return launch_attn<D, false, false, false, -1>(p, out_map, s);
+}
+
 cudaError_t attn_forward(const AttnParams& p0, const CUtensorMap& out_map, int D, bool pv8, int acc, int max_len_q,
                          int nseq, cudaStream_t s) {
   const bool acc2 = acc != kAccOne;
@@ -1193,18 +1230,8 @@ cudaError_t attn_forward(const AttnParams& p0, const CUtensorMap& out_map, int D
   p.n_pairs = (int)nx;
   p.nseq = nseq;
   p.n_items = (int)items;
-  if (D == 128) {
-    if (pv8) {
-      if (acc == kAccTwoF16) return launch_attn<128, true, true, true>(p, out_map, s);
-      return acc2 ? launch_attn<128, true, true, false>(p, out_map, s) : launch_attn<128, true, false, false>(p, out_map, s);
-    }
-    return acc2 ? launch_attn<128, false, true, false>(p, out_map, s) : launch_attn<128, false, false, false>(p, out_map, s);
-  }
-  if (pv8) {
-    if (acc == kAccTwoF16) return launch_attn<64, true, true, true>(p, out_map, s);
-    return acc2 ? launch_attn<64, true, true, false>(p, out_map, s) : launch_attn<64, true, false, false>(p, out_map, s);
-  }
-  return acc2 ? launch_attn<64, false, true, false>(p, out_map, s) : launch_attn<64, false, false, false>(p, out_map, s);
+  if (D == 128) return launch_mode<128>(p, out_map, pv8, acc, s);
+  return launch_mode<64>(p, out_map, pv8, acc, s);
 }
 
 cudaError_t debug_qk_tile(const int8_t* qt, const int8_t* kt, int D, int32_t* out, uint32_t* err,
