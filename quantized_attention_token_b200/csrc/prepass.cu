@@ -37,6 +37,13 @@
 namespace sage {
 
 constexpr int kPrepassThreads = 256;
+// Resident CTAs per SM the pre-pass launches are built for.  D = 64 threads
+// hold half as many 16-byte chunks of a tile (4), so a fourth CTA keeps more
+// loads in flight: 0.196 vs 0.224 ms at B=8 H=32 S=4096 D=64 on B200, without
+// spills.  At D = 128 a fourth CTA left 64 registers and made the kernels spill
+// (108-228 bytes), for no gain at B=2 H=32 S=4096.
+template <int D>
+constexpr int prepass_min_ctas() { return D == 64 ? 4 : 3; }
 
 // Thread (cc = tid % TPR, rg = tid / TPR) owns 16-byte chunk cc (channels
 // 8cc .. 8cc+7) of the NR consecutive rows rg*NR .. rg*NR + NR-1.
@@ -469,7 +476,7 @@ __device__ void v_tile(const PrepassJob& j, int h, int t, const TileLoc& L, VSme
 // Launch A: blockIdx.x = tile slot, blockIdx.y over [Q heads | K-statistics
 // heads | V-statistics heads] (each part present only when asked for).
 template <int D, bool BF16, bool SV>
-__global__ void __launch_bounds__(kPrepassThreads, 3) prepass_a_kernel(const PrepassJob j) {
+__global__ void __launch_bounds__(kPrepassThreads, prepass_min_ctas<D>()) prepass_a_kernel(const PrepassJob j) {
   __shared__ union {
     QuantSmem<D> q;
     StatSmem<D> s;
@@ -502,7 +509,7 @@ __global__ void __launch_bounds__(kPrepassThreads, 3) prepass_a_kernel(const Pre
 // Launch B: blockIdx.y over [K heads | V heads], both axes walked backwards
 // (the last V head's last tile first).
 template <int D, bool BF16, bool SV>
-__global__ void __launch_bounds__(kPrepassThreads, 3) prepass_b_kernel(const PrepassJob j) {
+__global__ void __launch_bounds__(kPrepassThreads, prepass_min_ctas<D>()) prepass_b_kernel(const PrepassJob j) {
   __shared__ union {
     QuantSmem<D> q;
     VTileSmem<D> vt;
