@@ -283,25 +283,21 @@ __device__ __forceinline__ void store_row(uint16_t* orow, uint32_t ob, const flo
 // One-level epilogue of one warp's 32 rows (its quarter of the TMEM lanes):
 // out = O * 1/l (* delta_V[c] in FP8 mode, + the channel mean with smooth V),
 // rounded to 16 bits.  Each thread puts its row in shared memory, in 16-byte
-// chunks XOR-swizzled by row, and then the warp writes whole rows: one store
-// instruction covers 512 contiguous bytes of two (D = 128) or four (D = 64)
-// rows.  The staging areas stage0 and stage1 (4 KB each) are the warp's own
-// rows of the query tile's two P~ halves, which only this warp writes next.
-// BOXED: the layout is that of the boxes of the output tensor map (64 columns
-// x 32 rows of 128 bytes, 16-byte chunk c of row r at c ^ (r mod 8): the
-// 128-byte swizzle), columns 0-63 at stage0 and 64-127 at stage1; otherwise
-// rows 0-15 are at stage0 and 16-31 at stage1, chunk c of row r at
-// c ^ (r mod chunks per row).  by_map (BOXED only): the caller stores the
-// boxes with bulk tensor stores; otherwise the warp writes the rows here.
-template <int D, bool PV8, bool BOXED>
+// chunks, laid out as the boxes of the output tensor map: 64 columns x 32
+// rows of 128 bytes, chunk c of row r at c ^ (r mod 8) (the 128-byte
+// swizzle), columns 0-63 at stage0 and 64-127 at stage1 (4 KB each: the
+// warp's own rows of the query tile's two P~ halves, which only this warp
+// writes next).  by_map: the caller stores the boxes with bulk tensor stores;
+// otherwise the warp writes whole rows here, one store instruction covering
+// 512 contiguous bytes of two (D = 128) or four (D = 64) rows.
+template <int D, bool PV8>
 __device__ __forceinline__ void store_tile(uint16_t* orow0, long long ss, int nvalid, uint32_t stage0, uint32_t stage1,
                                            uint32_t ob, float inv_l, const float* vsc, const float* vmu, bool bf16,
                                            bool have_o, int lane, bool by_map) {
   constexpr int CH = 2 * D / 16;  // 16-byte chunks per row
   constexpr int RPI = 32 / CH;    // rows per warp store instruction
   auto chunk_addr = [&](int r, int k) -> uint32_t {
-    if (BOXED) return ((k >> 3) ? stage1 : stage0) + r * 128 + (((k & 7) ^ (r & 7)) << 4);
-    return (r < 16 ? stage0 : stage1) + (r & 15) * (2 * D) + ((k ^ (r & (CH - 1))) << 4);
+    return ((k >> 3) ? stage1 : stage0) + r * 128 + (((k & 7) ^ (r & 7)) << 4);
   };
 #pragma unroll
   for (int ch = 0; ch < D / 32; ++ch) {
@@ -333,7 +329,7 @@ __device__ __forceinline__ void store_tile(uint16_t* orow0, long long ss, int nv
       st_shared_v4(chunk_addr(lane, k), w[4 * kk], w[4 * kk + 1], w[4 * kk + 2], w[4 * kk + 3]);
     }
   }
-  if (BOXED && by_map) return;
+  if (by_map) return;
   __syncwarp();
 #pragma unroll
   for (int i = 0; i < 32 / RPI; ++i) {
@@ -706,9 +702,9 @@ __device__ __forceinline__ void softmax_role(const AttnParams& p, const CUtensor
       const uint32_t half = C::NPB == 2 ? (uint32_t)(NQ * C::PT) : (uint32_t)(C::PT / 2);
       const uint32_t stage0 = sb + C::OFF_P + q * C::PT + w * 4096;
       const int nvalid = min(32, max(0, io.Lq - row0));
-      const bool by_map = !ACC2 && p.use_out_map != 0;
-      store_tile<D, PV8, !ACC2>(orow0, p.os.ss, nvalid, stage0, stage0 + half, ob, l > 0.f ? 1.0f / l : 0.f, vsc, vmu,
-                         bf16, nq > 0, t & 31, by_map);
+      const bool by_map = p.use_out_map != 0;
+      store_tile<D, PV8>(orow0, p.os.ss, nvalid, stage0, stage0 + half, ob, l > 0.f ? 1.0f / l : 0.f, vsc, vmu, bf16,
+                         nq > 0, t & 31, by_map);
       if (by_map) {
         // dense: the boxes go out with asynchronous bulk tensor stores; the
         // staging area is reused only after they have read it (the wait at
