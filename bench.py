@@ -188,10 +188,42 @@ class Clocks:
                 "samples": len(sm)}
 
 
+def strip_comments(src: str) -> str:
+    """C/C++ source without its // and /* */ comments, every run of whitespace
+    outside string and character literals collapsed to one space, so that an
+    edit of comments or layout leaves the hash alone."""
+    out, i, n = [], 0, len(src)
+    while i < n:
+        c = src[i]
+        if c in "\"'":
+            j = i + 1
+            while j < n and src[j] != c:
+                j += 2 if src[j] == "\\" else 1
+            out.append(src[i:j + 1])
+            i = j + 1
+        elif src.startswith("//", i):
+            i = src.find("\n", i)
+            i = n if i < 0 else i
+        elif src.startswith("/*", i):
+            j = src.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+            out.append(" ")
+        elif c.isspace():
+            out.append(" ")
+            i += 1
+        else:
+            out.append(c)
+            i += 1
+    return " ".join("".join(out).split())
+
+
 def kernel_source_hash():
+    """Hash of the attention kernel's sources without comments: the recorded
+    ncu traffic is used only while it matches."""
     h = hashlib.sha256()
     for f in ("attn_fwd.cu", "sage_common.cuh", "sage_launch.cuh"):
-        h.update(open(os.path.join(ROOT, "quantized_attention_token_b200", "csrc", f), "rb").read())
+        src = open(os.path.join(ROOT, "quantized_attention_token_b200", "csrc", f), encoding="utf-8").read()
+        h.update(strip_comments(src).encode())
     return h.hexdigest()[:16]
 
 

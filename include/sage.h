@@ -317,7 +317,8 @@ int sage_debug_last_prepass_path(void);
 sage_status_t sage_debug_set_out_map(int on);
 
 /* Debug: the output store path of the calling thread's last attention launch:
- * 1 the tensor map, 2 per-warp stores, 0 none yet. */
+ * 1 the tensor map, 2 stores from the threads (per-warp rows in one-level
+ * modes, each thread's row in two-level modes), 0 none yet. */
 int sage_debug_last_out_path(void);
 
 /* Debug: the int32 scores of one 128x128 tile, S = Q_codes(q tile) *

@@ -344,6 +344,7 @@ def debug_set_out_map(on: bool):
 
 
 def debug_last_out_path():
-    """"tensor_map", "warp_stores" or None: the output store path of this
-    thread's last attention launch."""
+    """"tensor_map", "warp_stores" (stores from the threads: per-warp rows in
+    one-level modes, each thread's row in two-level modes) or None: the output
+    store path of this thread's last attention launch."""
     return OUT_PATH[lib().sage_debug_last_out_path()]

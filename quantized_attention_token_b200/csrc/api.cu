@@ -37,7 +37,7 @@ std::atomic<int> g_out_map{1};
 // kPrepassTwoLaunch, 0 none).
 thread_local int g_last_prepass_path = 0;
 // The output store path of the calling thread's last attention launch
-// (1 tensor map, 2 per-warp stores, 0 none).
+// (1 tensor map, 2 stores from the threads, 0 none).
 thread_local int g_last_out_path = 0;
 
 // ---------------------------------------------------------------- device check

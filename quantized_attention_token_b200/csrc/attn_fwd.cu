@@ -24,12 +24,16 @@
 //                 row of S and at once releases the S columns, so the next
 //                 tile's QK^T runs while it works; P~ goes to shared memory in
 //                 the swizzled K-major operand layout; in one-level mode it
-//                 also rescales O in TMEM and writes the epilogue;
+//                 also rescales O in TMEM and writes the epilogue (dense: the
+//                 rows staged as output tensor-map boxes and written with
+//                 bulk tensor stores);
 //   WG 2 (two-level mode, NQ = 1) correction: adds each tile's fresh partial
 //                 O (FP32, or binary16 in fp32+fp16 mode) into an FP32
 //                 register accumulator; epilogue.
 // Warpgroup 0 (loader, MMA, allocator) hands registers to WG 1..2 with
-// setmaxnreg (56 / 224 / 224 per thread).
+// setmaxnreg (56 / 224 / 224 per thread).  The softmax's template variants
+// (per_thread K scales, bf16 P~, smooth Q) sit behind a run-time switch in the
+// one-level kernels and get a kernel each in two-level mode (VAR).
 // Every mbarrier wait is bounded (sage_common.cuh): a wait that never ends sets
 // the device error word and the CTA tears down instead of hanging.
 #include "sage_launch.cuh"

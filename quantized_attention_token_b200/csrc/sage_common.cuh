@@ -298,7 +298,6 @@ __device__ __forceinline__ uint4 ld_shared_v4(uint32_t addr) {
                : "memory");
   return v;
 }
-// Fetch the line holding p into L1 (no register result).
 // Asynchronous bulk tensor store of one box from this CTA's shared memory (no
 // multicast), tracked in the issuing thread's bulk async-group; map is the
 // address of a tensor map in kernel parameter space.
@@ -312,6 +311,7 @@ __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.comm
 // The thread's bulk stores have read their shared-memory sources.
 __device__ __forceinline__ void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 
+// Fetch the line holding p into L1 (no register result).
 __device__ __forceinline__ void prefetch_l1(const void* p) {
   asm volatile("prefetch.global.L1 [%0];" ::"l"(p));
 }
